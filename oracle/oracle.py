@@ -1,0 +1,257 @@
+"""ctypes front end of the CPU oracle (``df11_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product package never
+imports this module, and this module never imports the product package.
+
+The steps follow "DFloat11: Kompresi inferensi GPU lossless ..."
+(id.news.hada.io/topic?id=20542); each C function names the section it
+restates.  ``build_format`` chains them in the page's order: split the BF16
+fields, histogram the exponents, Huffman code lengths (capped at 32 bits),
+canonical codes, bit-pack EncodedExponent, then the decoder metadata (Gaps,
+BlockOffset) and the hierarchical LUTs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "df11_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libdf11_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+MAX_CODE_LEN = 32  # "Kernel GPU 2 tahap": the longest code is 32 bits
+SEGMENT_BITS = 64  # "Kernel GPU 2 tahap": n = 8 bytes per thread
+
+
+def build(force: bool = False) -> str:
+    """Compiles the oracle with gcc into a shared object next to its source."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-Wall", "-o", tmp, _SRC],
+            check=True,
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        U64 = ctypes.c_uint64
+        lib.df11o_split.argtypes = [P, U64, P, P]
+        lib.df11o_split.restype = ctypes.c_int64
+        lib.df11o_histogram.argtypes = [P, U64, P]
+        lib.df11o_histogram.restype = None
+        lib.df11o_huffman_lengths.argtypes = [P, P]
+        lib.df11o_huffman_lengths.restype = ctypes.c_int
+        lib.df11o_package_merge.argtypes = [P, ctypes.c_int, P]
+        lib.df11o_package_merge.restype = ctypes.c_int
+        lib.df11o_code_lengths.argtypes = [P, ctypes.c_int, P]
+        lib.df11o_code_lengths.restype = ctypes.c_int
+        lib.df11o_canonical_codes.argtypes = [P, P]
+        lib.df11o_canonical_codes.restype = None
+        lib.df11o_encode.argtypes = [P, U64, P, P, P]
+        lib.df11o_encode.restype = U64
+        lib.df11o_metadata.argtypes = [P, U64, P, U64, ctypes.c_uint32, P, P]
+        lib.df11o_metadata.restype = ctypes.c_int
+        lib.df11o_pack_gaps.argtypes = [P, U64, P]
+        lib.df11o_pack_gaps.restype = None
+        lib.df11o_build_luts.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_int)]
+        lib.df11o_build_luts.restype = ctypes.c_int
+        lib.df11o_decode.argtypes = [P, U64, P, P, P, U64, P]
+        lib.df11o_decode.restype = ctypes.c_int
+        lib.df11o_decode_range.argtypes = [P, U64, U64, U64, P, P, P, U64]
+        lib.df11o_decode_range.restype = ctypes.c_int64
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+class UnsupportedExponent(ValueError):
+    """An element has an exponent in 240..255, the range reserved for LUT
+    pointers ("Decoding berbasis LUT hierarkis")."""
+
+
+def split(w: np.ndarray):
+    """BF16 bits -> (exponent bytes, sign/mantissa bytes)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).ravel()
+    exps = np.empty(w.size, np.uint8)
+    sm = np.empty(w.size, np.uint8)
+    bad = _load().df11o_split(_ptr(w), w.size, _ptr(exps), _ptr(sm))
+    if bad >= 0:
+        raise UnsupportedExponent(f"element {bad} has exponent >= 240")
+    return exps, sm
+
+
+def histogram(exps: np.ndarray) -> np.ndarray:
+    exps = np.ascontiguousarray(exps, dtype=np.uint8)
+    hist = np.zeros(256, np.uint64)
+    _load().df11o_histogram(_ptr(exps), exps.size, _ptr(hist))
+    return hist
+
+
+def huffman_lengths(hist) -> np.ndarray:
+    """Plain (uncapped) Huffman code lengths."""
+    hist = np.ascontiguousarray(hist, dtype=np.uint64)
+    lens = np.zeros(256, np.uint8)
+    _load().df11o_huffman_lengths(_ptr(hist), _ptr(lens))
+    return lens
+
+
+def package_merge(hist, max_len: int) -> np.ndarray:
+    """Optimal code lengths with every length <= max_len."""
+    hist = np.ascontiguousarray(hist, dtype=np.uint64)
+    lens = np.zeros(256, np.uint8)
+    if _load().df11o_package_merge(_ptr(hist), int(max_len), _ptr(lens)) != 0:
+        raise ValueError("no prefix code with this length cap")
+    return lens
+
+
+def code_lengths(hist, max_len: int = MAX_CODE_LEN) -> np.ndarray:
+    """The format's code lengths: Huffman, else package-merge at the cap."""
+    hist = np.ascontiguousarray(hist, dtype=np.uint64)
+    lens = np.zeros(256, np.uint8)
+    if _load().df11o_code_lengths(_ptr(hist), int(max_len), _ptr(lens)) < 0:
+        raise ValueError("no prefix code with this length cap")
+    return lens
+
+
+def canonical_codes(lens) -> np.ndarray:
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    codes = np.zeros(256, np.uint32)
+    _load().df11o_canonical_codes(_ptr(lens), _ptr(codes))
+    return codes
+
+
+def encode(exps, lens, codes):
+    """Returns (stream bytes, total bits); the stream has ceil(bits/8) bytes."""
+    exps = np.ascontiguousarray(exps, dtype=np.uint8)
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    total = int(np.sum(lens[exps].astype(np.uint64))) if exps.size else 0
+    stream = np.zeros(max((total + 7) // 8, 1), np.uint8)
+    bits = _load().df11o_encode(_ptr(exps), exps.size, _ptr(lens), _ptr(codes), _ptr(stream))
+    assert bits == total
+    return stream[: (total + 7) // 8], int(bits)
+
+
+def metadata(exps, lens, total_bits: int, threads_per_block: int):
+    """Returns (gaps: one uint8 per segment, block_offset: uint32[nblocks+1])."""
+    exps = np.ascontiguousarray(exps, dtype=np.uint8)
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    nseg = (total_bits + SEGMENT_BITS - 1) // SEGMENT_BITS
+    nblocks = (nseg + threads_per_block - 1) // threads_per_block
+    gaps = np.zeros(max(nseg, 1), np.uint8)
+    offs = np.zeros(nblocks + 1, np.uint32)
+    rc = _load().df11o_metadata(
+        _ptr(exps), exps.size, _ptr(lens), total_bits, threads_per_block, _ptr(gaps), _ptr(offs)
+    )
+    if rc != 0:
+        raise ValueError("a gap exceeds 31 bits")
+    return gaps[:nseg], offs
+
+
+def pack_gaps(gaps) -> np.ndarray:
+    """5-bit fields, LSB-first, into uint64 words (one spare word at the end)."""
+    gaps = np.ascontiguousarray(gaps, dtype=np.uint8)
+    words = np.zeros((5 * gaps.size + 63) // 64 + 1, np.uint64)
+    _load().df11o_pack_gaps(_ptr(gaps), gaps.size, _ptr(words))
+    return words
+
+
+def build_luts(lens, codes):
+    """Returns the k x 256 uint8 hierarchical LUTs."""
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    luts = np.zeros(17 * 256, np.uint8)
+    k = ctypes.c_int(0)
+    rc = _load().df11o_build_luts(_ptr(lens), _ptr(codes), _ptr(luts), ctypes.byref(k))
+    if rc == -2:
+        raise ValueError("more than 16 child LUTs")
+    if rc != 0:
+        raise ValueError("code lengths do not form a prefix code")
+    return luts[: k.value * 256].reshape(k.value, 256).copy()
+
+
+def decode(stream, total_bits: int, lens, codes, sm, n: int) -> np.ndarray:
+    """Bit-by-bit tree-walk decode back to BF16 bits (uint16)."""
+    stream = np.ascontiguousarray(stream, dtype=np.uint8)
+    if stream.size == 0:
+        stream = np.zeros(1, np.uint8)
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    sm = np.ascontiguousarray(sm, dtype=np.uint8)
+    if sm.size == 0:
+        sm = np.zeros(1, np.uint8)
+    out = np.empty(max(n, 1), np.uint16)
+    rc = _load().df11o_decode(
+        _ptr(stream), total_bits, _ptr(lens), _ptr(codes), _ptr(sm), n, _ptr(out)
+    )
+    if rc != 0:
+        raise ValueError("stream is inconsistent with the code")
+    return out[:n]
+
+
+def decode_range(stream, stream_bits: int, start_bit: int, end_bit: int, lens, codes) -> np.ndarray:
+    """Exponents of the codes that start in [start_bit, end_bit)."""
+    stream = np.ascontiguousarray(stream, dtype=np.uint8)
+    lens = np.ascontiguousarray(lens, dtype=np.uint8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    cap = max(end_bit - start_bit, 1)
+    out = np.empty(cap, np.uint8)
+    cnt = _load().df11o_decode_range(
+        _ptr(stream), stream_bits, start_bit, end_bit, _ptr(lens), _ptr(codes), _ptr(out), cap
+    )
+    if cnt < 0:
+        raise ValueError("stream is inconsistent with the code")
+    return out[:cnt].copy()
+
+
+def build_format(w: np.ndarray, threads_per_block: int = 256, max_len: int = MAX_CODE_LEN) -> dict:
+    """All DF11 arrays for one stream of BF16 bits, built step by step."""
+    exps, sm = split(w)
+    hist = histogram(exps)
+    lens = code_lengths(hist, max_len)
+    codes = canonical_codes(lens)
+    stream, total_bits = encode(exps, lens, codes)
+    gaps, offs = metadata(exps, lens, total_bits, threads_per_block)
+    luts = build_luts(lens, codes)
+    return {
+        "n": int(exps.size),
+        "hist": hist,
+        "code_lengths": lens,
+        "codes": codes,
+        "encoded_exponent": stream,
+        "total_bits": total_bits,
+        "packed_sign_mantissa": sm,
+        "gaps": gaps,
+        "gaps_packed": pack_gaps(gaps),
+        "block_offset": offs,
+        "luts": luts,
+        "threads_per_block": threads_per_block,
+    }
+
+
+def decode_format(fmt: dict) -> np.ndarray:
+    return decode(
+        fmt["encoded_exponent"], fmt["total_bits"], fmt["code_lengths"], fmt["codes"],
+        fmt["packed_sign_mantissa"], fmt["n"],
+    )
