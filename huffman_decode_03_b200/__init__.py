@@ -1,0 +1,295 @@
+"""B200-native DFloat11 (DF11) decompression: Python binding of the C ABI.
+
+Every entry point forwards to ``libdf11_b200.so`` (declared in
+``include/df11.h``); this module only marshals arguments.  PyTorch supplies
+device memory and CUDA streams.  There is no CPU fallback: if the library
+cannot be loaded, or the CUDA path is used without a GPU, the call raises.
+
+Names follow the DFloat11 page (id.news.hada.io/topic?id=20542): a stream's
+``encoded_exponent`` (EncodedExponent), ``packed_sign_mantissa``
+(PackedSignMantissa), ``gaps``, ``block_offset``, ``luts`` and
+``code_lengths`` (CodeLengths).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "Df11Error", "Format", "DeviceFormat", "build_format", "decompress",
+    "decompress_host", "read_status", "load_library",
+]
+
+DF11_OK = 0
+DF11_ERR_CORRUPT = 6
+
+
+class Df11Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        msg = _strerror(status)
+        super().__init__(f"{what}: {msg} (status {status})" if what else msg)
+
+
+class df11_arrays(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_uint64),
+        ("total_bits", ctypes.c_uint64),
+        ("num_segments", ctypes.c_uint64),
+        ("threads_per_block", ctypes.c_uint32),
+        ("num_blocks", ctypes.c_uint32),
+        ("num_luts", ctypes.c_uint32),
+        ("max_code_len", ctypes.c_uint32),
+        ("max_block_elems", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+        ("encoded_exponent", ctypes.c_void_p),
+        ("encoded_exponent_bytes", ctypes.c_uint64),
+        ("packed_sign_mantissa", ctypes.c_void_p),
+        ("packed_sign_mantissa_bytes", ctypes.c_uint64),
+        ("gaps", ctypes.c_void_p),
+        ("gaps_words", ctypes.c_uint64),
+        ("block_offset", ctypes.c_void_p),
+        ("luts", ctypes.c_void_p),
+        ("code_lengths", ctypes.c_void_p),
+    ]
+
+
+class df11_info(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_uint64),
+        ("total_bits", ctypes.c_uint64),
+        ("compressed_bytes", ctypes.c_uint64),
+        ("entropy_bits", ctypes.c_double),
+        ("avg_code_len", ctypes.c_double),
+        ("distinct_exponents", ctypes.c_uint32),
+        ("max_code_len", ctypes.c_uint32),
+        ("num_luts", ctypes.c_uint32),
+        ("threads_per_block", ctypes.c_uint32),
+        ("histogram", ctypes.c_uint64 * 256),
+    ]
+
+
+EXPORTS = (
+    "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
+    "df11_strerror", "df11_decompress", "df11_decompress_host", "df11_read_status",
+)
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Loads (building first when the sources are newer) the C-ABI library."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    if path is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path) or _build._stale():
+            _build.build()
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lib.df11_build_format.argtypes = [P, P, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(P)]
+    lib.df11_build_format.restype = ctypes.c_int
+    lib.df11_format_arrays.argtypes = [P, ctypes.POINTER(df11_arrays)]
+    lib.df11_format_arrays.restype = ctypes.c_int
+    lib.df11_format_info.argtypes = [P, ctypes.POINTER(df11_info)]
+    lib.df11_format_info.restype = ctypes.c_int
+    lib.df11_free.argtypes = [P]
+    lib.df11_free.restype = None
+    lib.df11_strerror.argtypes = [ctypes.c_int]
+    lib.df11_strerror.restype = ctypes.c_char_p
+    lib.df11_decompress.argtypes = [ctypes.POINTER(df11_arrays), P, P, P]
+    lib.df11_decompress.restype = ctypes.c_int
+    lib.df11_decompress_host.argtypes = [
+        ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_arrays), P, P, P, P]
+    lib.df11_decompress_host.restype = ctypes.c_int
+    lib.df11_read_status.argtypes = [P, P]
+    lib.df11_read_status.restype = ctypes.c_int
+    if path == _build.LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _strerror(status: int) -> str:
+    try:
+        return load_library().df11_strerror(int(status)).decode()
+    except OSError:
+        return f"status {status}"
+
+
+def _check(status: int, what: str):
+    if status != DF11_OK:
+        raise Df11Error(status, what)
+
+
+# --------------------------------------------------------------------- host
+class Format:
+    """A host-resident DF11 stream (handle from ``df11_build_format``)."""
+
+    def __init__(self, handle: int, lib):
+        self._h = ctypes.c_void_p(handle)
+        self._lib = lib
+        a = df11_arrays()
+        _check(lib.df11_format_arrays(self._h, ctypes.byref(a)), "df11_format_arrays")
+        self.c_arrays = a
+
+    def __del__(self):
+        self.free()
+
+    def free(self):
+        if getattr(self, "_h", None) and self._h.value:
+            self._lib.df11_free(self._h)
+            self._h = ctypes.c_void_p(0)
+
+    @property
+    def n(self) -> int:
+        return int(self.c_arrays.n)
+
+    def _view(self, ptr, count, dtype):
+        if count == 0 or not ptr:
+            return np.zeros(0, dtype)
+        nbytes = int(count) * np.dtype(dtype).itemsize
+        buf = (ctypes.c_uint8 * nbytes).from_address(ptr)
+        return np.frombuffer(buf, dtype=dtype, count=int(count))
+
+    def arrays(self) -> dict:
+        """Borrowed numpy views of the host arrays (valid while self lives)."""
+        a = self.c_arrays
+        return {
+            "encoded_exponent": self._view(a.encoded_exponent, a.encoded_exponent_bytes, np.uint8),
+            "packed_sign_mantissa": self._view(a.packed_sign_mantissa, a.packed_sign_mantissa_bytes, np.uint8),
+            "gaps": self._view(a.gaps, a.gaps_words, np.uint64),
+            "block_offset": self._view(a.block_offset, a.num_blocks + 1, np.uint32),
+            "luts": self._view(a.luts, a.num_luts * 256, np.uint8).reshape(a.num_luts, 256),
+            "code_lengths": self._view(a.code_lengths, 256, np.uint8),
+        }
+
+    def info(self) -> dict:
+        i = df11_info()
+        _check(self._lib.df11_format_info(self._h, ctypes.byref(i)), "df11_format_info")
+        return {
+            "n": int(i.n), "total_bits": int(i.total_bits), "compressed_bytes": int(i.compressed_bytes),
+            "entropy_bits": float(i.entropy_bits), "avg_code_len": float(i.avg_code_len),
+            "distinct_exponents": int(i.distinct_exponents), "max_code_len": int(i.max_code_len),
+            "num_luts": int(i.num_luts), "threads_per_block": int(i.threads_per_block),
+            "num_segments": int(self.c_arrays.num_segments), "num_blocks": int(self.c_arrays.num_blocks),
+            "max_block_elems": int(self.c_arrays.max_block_elems),
+            "histogram": np.array(i.histogram[:], np.uint64),
+        }
+
+    def scalars(self) -> dict:
+        a = self.c_arrays
+        return {f: int(getattr(a, f)) for f in (
+            "n", "total_bits", "num_segments", "threads_per_block", "num_blocks", "num_luts",
+            "max_code_len", "max_block_elems")}
+
+
+def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 256) -> Format:
+    """Compresses BF16 bit patterns (uint16 arrays, or torch bfloat16/int16
+    CPU tensors) into one DF11 stream; matrices are concatenated in order."""
+    lib = load_library()
+    if isinstance(mats, np.ndarray) or hasattr(mats, "data_ptr"):
+        mats = [mats]
+    keep = []
+    for m in mats:
+        if hasattr(m, "data_ptr"):  # torch tensor
+            m = m.detach().contiguous().cpu().view(-1)
+            import torch
+            m = m.view(torch.int16).numpy().view(np.uint16)
+        keep.append(np.ascontiguousarray(np.asarray(m).view(np.uint16).reshape(-1)))
+    k = len(keep)
+    ptrs = (ctypes.c_void_p * max(k, 1))(*[m.ctypes.data if m.size else None for m in keep])
+    counts = (ctypes.c_uint64 * max(k, 1))(*[m.size for m in keep])
+    h = ctypes.c_void_p()
+    _check(lib.df11_build_format(ptrs, counts, k, int(threads_per_block), ctypes.byref(h)),
+           "df11_build_format")
+    return Format(h.value, lib)
+
+
+# ------------------------------------------------------------------- device
+class DeviceFormat:
+    """A DF11 stream resident in device memory (arrays held as torch tensors)."""
+
+    def __init__(self, fmt: Format, device="cuda", pin_host: bool = False):
+        import torch
+
+        self.device = torch.device(device)
+        self.scalars = fmt.scalars()
+        arrs = fmt.arrays()
+        self.tensors = {}
+        self.host_tensors = {}
+        for name, arr in arrs.items():
+            t = torch.from_numpy(np.ascontiguousarray(arr).reshape(-1).view(np.uint8))
+            if pin_host:
+                t = t.pin_memory()
+                self.host_tensors[name] = t
+            self.tensors[name] = t.to(self.device, non_blocking=False)
+        self.c_arrays = self._struct(self.tensors)
+        self.c_host_arrays = self._struct(self.host_tensors) if pin_host else None
+
+    def _struct(self, ts) -> df11_arrays:
+        a = df11_arrays()
+        for k, v in self.scalars.items():
+            setattr(a, k, v)
+        a.encoded_exponent = ts["encoded_exponent"].data_ptr()
+        a.encoded_exponent_bytes = ts["encoded_exponent"].numel()
+        a.packed_sign_mantissa = ts["packed_sign_mantissa"].data_ptr()
+        a.packed_sign_mantissa_bytes = ts["packed_sign_mantissa"].numel()
+        a.gaps = ts["gaps"].data_ptr()
+        a.gaps_words = ts["gaps"].numel() // 8
+        a.block_offset = ts["block_offset"].data_ptr()
+        a.luts = ts["luts"].data_ptr()
+        a.code_lengths = ts["code_lengths"].data_ptr()
+        return a
+
+    @property
+    def n(self) -> int:
+        return self.scalars["n"]
+
+    def nbytes(self) -> int:
+        return sum(t.numel() for t in self.tensors.values())
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def decompress(dev: DeviceFormat, out=None, status=None, stream=None):
+    """Rebuilds the BF16 stream on the GPU (asynchronous, stream-ordered).
+    Returns ``out`` (a torch.bfloat16 tensor of n elements, allocated if None)."""
+    import torch
+
+    if out is None:
+        out = torch.empty(dev.n, dtype=torch.bfloat16, device=dev.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev.device)
+    assert out.is_cuda and out.is_contiguous() and out.numel() >= dev.n and out.element_size() == 2
+    _check(load_library().df11_decompress(ctypes.byref(dev.c_arrays), ctypes.c_void_p(out.data_ptr()),
+                                          ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
+           "df11_decompress")
+    return out
+
+
+def decompress_host(dev: DeviceFormat, out_dev, out_host, status, stream=None):
+    """Host-to-host decode: copies the pinned host arrays in, decodes, copies
+    the BF16 result to ``out_host`` (pinned, 2n bytes).  Asynchronous."""
+    assert dev.c_host_arrays is not None, "DeviceFormat(pin_host=True) required"
+    _check(load_library().df11_decompress_host(
+        ctypes.byref(dev.c_host_arrays), ctypes.byref(dev.c_arrays), ctypes.c_void_p(out_dev.data_ptr()),
+        ctypes.c_void_p(out_host.data_ptr()), ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
+        "df11_decompress_host")
+    return out_host
+
+
+def read_status(status, stream=None) -> int:
+    """Synchronises the stream and returns the kernel status (0 = ok)."""
+    return int(load_library().df11_read_status(ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)))

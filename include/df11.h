@@ -1,0 +1,191 @@
+/*
+ * df11.h -- C ABI of a B200-native DFloat11 (DF11) decompressor.
+ *
+ * DF11 ("DFloat11: Kompresi inferensi GPU lossless yang mengecilkan LLM
+ * menjadi 70% ukurannya", id.news.hada.io/topic?id=20542) stores a BFloat16
+ * matrix as two byte arrays: EncodedExponent, the 8-bit exponents Huffman
+ * coded and bit-packed, and PackedSignMantissa, sign and mantissa verbatim
+ * (section "Format DFloat11").  The GPU rebuilds the exact BF16 values right
+ * before they are used (section "Dekompresi yang disesuaikan untuk inferensi
+ * GPU"), helped by hierarchical 256-entry LUTs ("Decoding berbasis LUT
+ * hierarkis") and per-thread / per-block metadata ("Kernel GPU 2 tahap dan
+ * metadata bantu").
+ *
+ * The library has two halves:
+ *   - host: df11_build_format compresses BF16 matrices into the format;
+ *   - device: df11_decompress rebuilds the BF16 matrix on a CUDA stream.
+ * No entry point takes or returns framework types; all pointers are plain
+ * host or device addresses as stated per argument.
+ *
+ * Byte layout of the format (every reader of the arrays relies on it):
+ *   - element = BF16 bits w; exponent = (w >> 7) & 0xFF, which must be < 240
+ *     (240..255 are LUT pointers); PackedSignMantissa byte = (w >> 8 & 0x80)
+ *     | (w & 0x7F).
+ *   - code lengths: Huffman over the exponent histogram, ties merged by
+ *     smallest (weight, smallest symbol in subtree); if the longest code
+ *     exceeds 32 bits, optimal 32-bit-limited lengths by package-merge.  A
+ *     single distinct exponent gets length 1.
+ *   - codes: canonical (symbols sorted by (length, symbol) get increasing
+ *     values).  CodeLengths[256] therefore fixes the whole code.
+ *   - EncodedExponent: codes concatenated MSB-first; bit i of the stream is
+ *     bit (7 - i % 8) of byte i / 8.  Zero padded.
+ *   - segment s = stream bits [64 s, 64 s + 64) (8 bytes per GPU thread).
+ *     Gap[s] = (first code start >= 64 s, or total_bits if none) - 64 s, in
+ *     [0, 31]; stored as 5-bit fields LSB-first in uint64 words (field s at
+ *     bits 5 s .. 5 s + 4 of the little-endian word sequence).
+ *   - block b = segments [T b, T b + T).  BlockOffset[b] = number of codes
+ *     that start before bit 64 T b; BlockOffset[num_blocks] = n.
+ *   - LUTs: k tables of 256 bytes.  Table 0 is indexed by the first 8 bits
+ *     of the 32-bit window, a child table by the next 8 bits.  An entry is a
+ *     symbol (< 240) or a pointer 256 - j to table j (j = 1 .. 16); children
+ *     are numbered level by level in increasing order of their bit prefix.
+ *
+ * Threading: the host functions are thread-safe for distinct handles.  The
+ * device functions are stream-ordered and never synchronise except where
+ * stated (df11_read_status).
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DF11_ABI_VERSION 1
+#define DF11_MAX_CODE_LEN 32     /* longest code: Gaps are 5 bits wide */
+#define DF11_SEGMENT_BYTES 8     /* encoded bytes per GPU thread */
+#define DF11_MAX_LUTS 17         /* root + 16 children (pointers 240..255) */
+#define DF11_DEFAULT_THREADS 256 /* default segments (threads) per block */
+
+typedef enum df11_status {
+    DF11_OK = 0,
+    DF11_ERR_INVALID_ARG = 1,          /* bad pointer, size, alignment or T */
+    DF11_ERR_UNSUPPORTED_EXPONENT = 2, /* an input exponent is in 240..255 */
+    DF11_ERR_TOO_LARGE = 3,            /* n >= 2^32 elements in one stream */
+    DF11_ERR_TOO_MANY_LUTS = 4,        /* the code needs > 16 child LUTs */
+    DF11_ERR_CUDA = 5,                 /* a CUDA runtime call failed */
+    DF11_ERR_CORRUPT = 6,              /* the kernel found inconsistent data */
+    DF11_ERR_NO_MEMORY = 7             /* host allocation failed */
+} df11_status;
+
+/* Opaque handle: a host-resident compressed stream (owns its arrays). */
+typedef struct df11_format df11_format;
+
+/*
+ * The arrays of one compressed stream.  The same struct describes host
+ * copies (df11_format_arrays) or device copies (filled in by the caller after
+ * uploading each array).  Sizes include the padding the kernel relies on.
+ */
+typedef struct df11_arrays {
+    uint64_t n;                 /* BF16 elements in the stream */
+    uint64_t total_bits;        /* valid bits of encoded_exponent */
+    uint64_t num_segments;      /* ceil(total_bits / 64) */
+    uint32_t threads_per_block; /* T: segments per block (multiple of 32, 32..1024) */
+    uint32_t num_blocks;        /* ceil(num_segments / T) */
+    uint32_t num_luts;          /* k, 1 .. 17 */
+    uint32_t max_code_len;      /* longest code length, <= 32 */
+    uint32_t max_block_elems;   /* max_b BlockOffset[b+1] - BlockOffset[b] */
+    uint32_t reserved;
+    const uint8_t *encoded_exponent;     /* num_blocks*T*8 + 16 bytes, zero padded, 16-B aligned */
+    uint64_t encoded_exponent_bytes;
+    const uint8_t *packed_sign_mantissa; /* round_up(n, 16) + 16 bytes, 16-B aligned */
+    uint64_t packed_sign_mantissa_bytes;
+    const uint64_t *gaps;                /* ceil(5*num_blocks*T / 64) + 1 words */
+    uint64_t gaps_words;
+    const uint32_t *block_offset;        /* num_blocks + 1 entries */
+    const uint8_t *luts;                 /* num_luts * 256 bytes */
+    const uint8_t *code_lengths;         /* 256 bytes, indexed by exponent */
+} df11_arrays;
+
+/* Statistics of a built stream ("Ruang kompresi": exponent entropy and the
+ * number of exponent values in use; "Decoding berbasis LUT hierarkis": L, k). */
+typedef struct df11_info {
+    uint64_t n;
+    uint64_t total_bits;
+    uint64_t compressed_bytes; /* ceil(total_bits/8) + n + gaps + offsets + LUTs + 256 */
+    double entropy_bits;       /* Shannon entropy of the exponent histogram */
+    double avg_code_len;       /* total_bits / n */
+    uint32_t distinct_exponents;
+    uint32_t max_code_len;
+    uint32_t num_luts;
+    uint32_t threads_per_block;
+    uint64_t histogram[256];
+} df11_info;
+
+/*
+ * df11_build_format -- compress BF16 matrices into one DF11 stream
+ * ("Format DFloat11"; metadata per "Kernel GPU 2 tahap dan metadata bantu").
+ *   mats[i]   host pointer to counts[i] BF16 bit patterns (uint16), row-major;
+ *             matrix i occupies elements [sum_{j<i} counts[j], ...) of the
+ *             stream.  One Huffman code covers all matrices (a transformer
+ *             block is compressed as one stream, "Dekompresi per transformer
+ *             block").  NULL allowed when counts[i] == 0.
+ *   threads_per_block  T, a multiple of 32 in [32, 1024] (0 = default 256).
+ *   out       receives a new handle, owned by the caller (df11_free).
+ * Inputs are only read.  Errors: DF11_ERR_INVALID_ARG, _UNSUPPORTED_EXPONENT,
+ * _TOO_LARGE (total n >= 2^32), _TOO_MANY_LUTS, _NO_MEMORY; *out is NULL then.
+ * Runs on the host with up to hardware_concurrency threads; needs no GPU.
+ */
+df11_status df11_build_format(const uint16_t *const *mats, const uint64_t *counts,
+                              int num_mats, uint32_t threads_per_block,
+                              df11_format **out);
+
+/* Borrowed host views of a handle's arrays (valid until df11_free). */
+df11_status df11_format_arrays(const df11_format *f, df11_arrays *out);
+
+/* Statistics of a handle. */
+df11_status df11_format_info(const df11_format *f, df11_info *out);
+
+/* Frees a handle; NULL is allowed. */
+void df11_free(df11_format *f);
+
+/* Static English text for a status code. */
+const char *df11_strerror(df11_status s);
+
+/*
+ * df11_decompress -- rebuild the BF16 stream on the GPU
+ * ("Dekompresi yang disesuaikan untuk inferensi GPU", "Decoding berbasis LUT
+ * hierarkis", "Kernel GPU 2 tahap dan metadata bantu").
+ *   dev        arrays whose pointers are DEVICE addresses (sizes as in the
+ *              host view); only read.
+ *   dst        device pointer to dev->n uint16 BF16 outputs, 16-byte aligned;
+ *              written in full, nothing else is written.
+ *   status_dev device pointer to one uint32, OR-accumulated with
+ *              DF11_ERR_CORRUPT when the kernel meets inconsistent data (the
+ *              affected block's outputs are then left unwritten); zero it
+ *              before the first call.
+ *   stream     a cudaStream_t (NULL = legacy default stream).
+ * Asynchronous; returns DF11_ERR_INVALID_ARG for bad arguments (checked on
+ * the host, nothing launched) or DF11_ERR_CUDA when the launch fails.
+ * n == 0 launches nothing.  The kernel never traps and every loop is bounded.
+ */
+df11_status df11_decompress(const df11_arrays *dev, uint16_t *dst,
+                            uint32_t *status_dev, void *stream);
+
+/*
+ * df11_decompress_host -- the same decode, starting and ending in host
+ * memory: copies every array of *host (host pointers, ideally pinned) into
+ * the device buffers named by *dev_buffers (device pointers with at least the
+ * host sizes; they are overwritten although the struct's pointers are const),
+ * runs df11_decompress into dst_dev, then copies the n outputs to dst_host.
+ * All copies are cudaMemcpyAsync on `stream`; the call does not synchronise.
+ */
+df11_status df11_decompress_host(const df11_arrays *host, const df11_arrays *dev_buffers,
+                                 uint16_t *dst_dev, uint16_t *dst_host,
+                                 uint32_t *status_dev, void *stream);
+
+/*
+ * df11_read_status -- synchronises `stream`, reads *status_dev (device
+ * pointer) and returns DF11_OK or DF11_ERR_CORRUPT (DF11_ERR_CUDA if the
+ * copy fails).
+ */
+df11_status df11_read_status(const uint32_t *status_dev, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

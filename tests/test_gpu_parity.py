@@ -1,0 +1,248 @@
+"""GPU parity: the sm_100a decoder, called through the C ABI, against the CPU
+oracle and against the original BF16 bits (DF11 is lossless: "Format
+DFloat11" / "Hasil evaluasi" -- outputs are bit-identical).
+
+Small and mid-size cases compare every element with the oracle's own
+tree-walk decode of its own format (built independently from the same seeded
+input).  Full-size workloads compare every element with the original bits
+and a sample of blocks with the oracle's decode of that block's bit range.
+Corrupted inputs must raise the status word, never fault or hang: each
+corruption below stays inside the bounds the kernel checks (5-bit gaps,
+bounded loops, offset/capacity checks, LUT pointer range).
+"""
+import numpy as np
+import pytest
+
+import huffman_decode_03_b200 as df11
+from huffman_decode_03_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def torch_cuda():
+    import torch
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch
+
+
+def gpu_decode(mats, T=256, dev_fmt=None):
+    torch = torch_cuda()
+    fmt = df11.build_format(mats, T)
+    dev = dev_fmt or df11.DeviceFormat(fmt, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((max(dev.n, 1),), float("nan"), dtype=torch.bfloat16, device="cuda")
+    df11.decompress(dev, out, status)
+    st = df11.read_status(status)
+    got = out[: dev.n].view(torch.int16).cpu().numpy().view(np.uint16)
+    return got, st, fmt
+
+
+def check_against_oracle(oracle_mod, w, T=256):
+    got, st, _ = gpu_decode(w, T)
+    assert st == 0
+    ref = oracle_mod.decode_format(oracle_mod.build_format(w, T))
+    assert np.array_equal(ref, w)  # oracle round trip
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("n", [1, 2, 15, 16, 17, 63, 64, 65, 1000, 256 * 25 - 1, 256 * 25, 256 * 25 + 1, 100_003])
+def test_sizes(oracle_mod, n):
+    check_against_oracle(oracle_mod, inputs.gaussian(n, [21, n]))
+
+
+@pytest.mark.parametrize("T", [128, 256, 512])
+def test_threads_per_block(oracle_mod, T):
+    check_against_oracle(oracle_mod, inputs.gaussian(300_001, [22, T]), T)
+
+
+def test_empty_stream():
+    torch = torch_cuda()
+    fmt = df11.build_format(np.zeros(0, np.uint16))
+    dev = df11.DeviceFormat(fmt, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    df11.decompress(dev, out, status)
+    assert df11.read_status(status) == 0
+
+
+def test_every_bf16_pattern(oracle_mod):
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ok = allbits[((allbits >> 7) & 0xFF) < 240]
+    for seed in range(3):
+        check_against_oracle(oracle_mod, np.random.default_rng(seed).permutation(ok))
+
+
+def test_single_symbol(oracle_mod):
+    w = np.full(100_000, 0x3F80, np.uint16)
+    w[::3] |= 0x8000
+    w[::5] |= 0x0055
+    check_against_oracle(oracle_mod, w)
+
+
+def test_length_limited_code(oracle_mod):
+    f = [1, 1]
+    while len(f) < 34:
+        f.append(f[-1] + f[-2])
+    exps = np.repeat(np.arange(34, dtype=np.uint16) + 60, f)
+    exps = np.random.default_rng(5).permutation(exps)
+    mant = np.random.default_rng(6).integers(0, 256, exps.size).astype(np.uint16)
+    w = (exps << 7) | (mant & 0x7F) | ((mant & 0x80) << 8)
+    got, st, fmt = gpu_decode(w)
+    assert st == 0 and fmt.info()["max_code_len"] == 32
+    assert np.array_equal(got, w)
+
+
+def test_stress_small(oracle_mod):
+    check_against_oracle(oracle_mod, inputs.stress(1 << 21, key=(3, 7, 7)))
+
+
+def test_multi_matrix(oracle_mod):
+    mats = [inputs.gaussian(n, [23, n]) for n in (4096 * 3 + 5, 17, 0, 70_000)]
+    got, st, _ = gpu_decode(mats)
+    assert st == 0
+    ref = oracle_mod.decode_format(oracle_mod.build_format(np.concatenate(mats), 256))
+    assert np.array_equal(got, ref)
+
+
+def test_output_alignment_and_neighbours():
+    # decoding into the middle of a larger buffer writes exactly n elements
+    torch = torch_cuda()
+    w = inputs.gaussian(12_345, [24])
+    fmt = df11.build_format(w)
+    dev = df11.DeviceFormat(fmt, "cuda")
+    buf = torch.full((12_345 + 64,), 7, dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress(dev, buf[8:].view(torch.bfloat16), status)
+    assert df11.read_status(status) == 0
+    h = buf.cpu().numpy().view(np.uint16)
+    assert np.all(h[:8] == 7) and np.all(h[8 + 12_345:] == 7)
+    assert np.array_equal(h[8:8 + 12_345], w)
+
+
+def test_repeated_launches_are_identical():
+    torch = torch_cuda()
+    w = inputs.gaussian(1 << 20, [25])
+    fmt = df11.build_format(w)
+    dev = df11.DeviceFormat(fmt, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = [df11.decompress(dev, None, status).view(torch.int16).clone() for _ in range(3)]
+    assert df11.read_status(status) == 0
+    for o in outs:
+        assert torch.equal(o, outs[0])
+    assert np.array_equal(outs[0].cpu().numpy().view(np.uint16), w)
+
+
+# ----------------------------------------------------------------- corruption
+def _corrupt_run(w, mutate):
+    torch = torch_cuda()
+    fmt = df11.build_format(w)
+    dev = df11.DeviceFormat(fmt, "cuda")
+    mutate(dev, torch)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(dev.n, dtype=torch.bfloat16, device="cuda")
+    df11.decompress(dev, out, status)
+    return df11.read_status(status)
+
+
+def test_corrupt_block_offset_is_reported():
+    def mutate(dev, torch):
+        offs = dev.tensors["block_offset"].view(torch.int32)
+        offs[3] += 5
+    assert _corrupt_run(inputs.gaussian(200_000, [26]), mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_corrupt_gaps_is_reported():
+    def mutate(dev, torch):
+        g = dev.tensors["gaps"]
+        g[40:48] ^= 0x5A
+    assert _corrupt_run(inputs.gaussian(200_000, [27]), mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_corrupt_stream_is_reported():
+    def mutate(dev, torch):
+        s = dev.tensors["encoded_exponent"]
+        s[1000:1400] = 0xFF
+    assert _corrupt_run(inputs.gaussian(200_000, [28]), mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_dangling_lut_pointer_is_reported():
+    # long codes exist in the stress distribution: point one child entry past k
+    w = inputs.stress(1 << 20, key=(3, 8, 8))
+    fmt = df11.build_format(w)
+    luts = fmt.arrays()["luts"]
+    ptr_idx = int(np.nonzero(luts[0] >= 240)[0][0])
+
+    def mutate(dev, torch):
+        dev.tensors["luts"][ptr_idx] = 240  # child 16, beyond num_luts
+    assert _corrupt_run(w, mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_understated_capacity_is_reported():
+    def mutate(dev, torch):
+        dev.c_arrays.max_block_elems = 100
+    assert _corrupt_run(inputs.gaussian(200_000, [29]), mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_bad_arguments_launch_nothing():
+    torch = torch_cuda()
+    fmt = df11.build_format(inputs.gaussian(1000, [30]))
+    dev = df11.DeviceFormat(fmt, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(1000 + 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(df11.Df11Error) as e:
+        df11.decompress(dev, out[1:], status)  # 2-byte aligned only
+    assert e.value.status == 1
+    dev.c_arrays.num_blocks += 1
+    with pytest.raises(df11.Df11Error):
+        df11.decompress(dev, out, status)
+
+
+# ----------------------------------------------------------- full workloads
+def _full_check(oracle_mod, workload, block_id=0, sample_blocks=24):
+    torch = torch_cuda()
+    mats = [m for _, _, m in inputs.workload_arrays(workload, block_id)]
+    w = np.concatenate(mats) if len(mats) > 1 else mats[0]
+    got, st, fmt = gpu_decode(mats, 256)
+    assert st == 0
+    assert np.array_equal(got, w)
+    # oracle: its own format from the same input, then its tree walk over a
+    # sample of blocks' bit ranges
+    ref = oracle_mod.build_format(w, 256)
+    offs = ref["block_offset"].astype(np.int64)
+    nb = offs.size - 1
+    rng = np.random.default_rng(workload)
+    blocks = sorted(set([0, nb - 1] + rng.integers(0, nb, sample_blocks).tolist()))
+    gaps = ref["gaps"]
+    nseg = gaps.size
+    for b in blocks:
+        s0 = b * 256
+        s1 = min((b + 1) * 256, nseg)
+        a = 64 * s0 + int(gaps[s0])
+        e = 64 * s1 + int(gaps[s1]) if s1 < nseg else ref["total_bits"]
+        exps = oracle_mod.decode_range(ref["encoded_exponent"], ref["total_bits"], a, e,
+                                       ref["code_lengths"], ref["codes"])
+        sl = slice(int(offs[b]), int(offs[b + 1]))
+        assert exps.size == sl.stop - sl.start
+        assert np.array_equal((got[sl] >> 7) & 0xFF, exps)
+    return fmt
+
+
+def test_workload_single_matrix(oracle_mod):
+    w = inputs.single_matrix()
+    check_against_oracle(oracle_mod, w)
+
+
+def test_workload_llama3_8b_block(oracle_mod):
+    _full_check(oracle_mod, 2)
+
+
+def test_workload_stress(oracle_mod):
+    fmt = _full_check(oracle_mod, 3)
+    info = fmt.info()
+    assert info["max_code_len"] >= 24 and 4 <= info["num_luts"] <= 8
+
+
+@pytest.mark.slow
+def test_workload_llama3_70b_block(oracle_mod):
+    _full_check(oracle_mod, 4, sample_blocks=8)
