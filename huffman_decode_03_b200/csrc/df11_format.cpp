@@ -439,7 +439,7 @@ extern "C" df11_status df11_build_format(const uint16_t *const *mats, const uint
         f->offsets[nblocks] = (uint32_t)n;
 
         // ---- 4b. pack gaps: word w holds fields overlapping bits [64w, 64w+64)
-        uint64_t nwords = (5 * nblocks * T + 63) / 64 + 1;
+        uint64_t nwords = (5 * nblocks * T + 63) / 64 + 2;
         f->gaps.assign(nwords, 0);
         parallel_for((nwords + 4095) / 4096, [&](uint64_t blk) {
             for (uint64_t w = blk * 4096; w < std::min(nwords, (blk + 1) * 4096); w++) {

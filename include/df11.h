@@ -93,7 +93,7 @@ typedef struct df11_arrays {
     uint64_t encoded_exponent_bytes;
     const uint8_t *packed_sign_mantissa; /* round_up(n, 16) + 16 bytes, 16-B aligned */
     uint64_t packed_sign_mantissa_bytes;
-    const uint64_t *gaps;                /* ceil(5*num_blocks*T / 64) + 1 words */
+    const uint64_t *gaps;                /* ceil(5*num_blocks*T / 64) + 2 words */
     uint64_t gaps_words;
     const uint32_t *block_offset;        /* num_blocks + 1 entries */
     const uint8_t *luts;                 /* num_luts * 256 bytes */
