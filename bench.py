@@ -50,7 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5],
                     help="1 single 1024x1024, 2 Llama-3-8B block, 3 stress 64Mi, "
                          "4 Llama-3-70B block, 5 32 Llama-3-8B blocks streamed")
-    ap.add_argument("--threads-per-block", type=int, default=256)
+    ap.add_argument("--threads-per-block", type=int, default=32)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -376,7 +376,7 @@ def _oracle_sample(workload: int, elems: int):
     mats = [m for _, _, m in inputs.workload_arrays(1 if workload == 1 else (2 if workload == 5 else workload), 0)]
     w = np.concatenate(mats) if len(mats) > 1 else mats[0]
     w = np.ascontiguousarray(w[:elems])
-    return oracle, oracle.build_format(w, 256)
+    return oracle, oracle.build_format(w, 32)
 
 
 def cpu_baseline(workload: int, seconds: float) -> dict:

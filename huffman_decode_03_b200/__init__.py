@@ -189,7 +189,7 @@ class Format:
             "max_code_len", "max_block_elems")}
 
 
-def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 256) -> Format:
+def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 32) -> Format:
     """Compresses BF16 bit patterns (uint16 arrays, or torch bfloat16/int16
     CPU tensors) into one DF11 stream; matrices are concatenated in order."""
     lib = load_library()

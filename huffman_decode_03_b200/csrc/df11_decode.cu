@@ -6,18 +6,21 @@
 //        subtrees stored as 256-entry LUTs whose values 240..255 are pointers;
 //   "Kernel GPU 2 tahap dan metadata bantu" -- one thread per 8-byte segment
 //        of EncodedExponent, starting at the segment's Gap; stage 1 counts the
-//        codes of each segment, a block-wide prefix sum plus the block's stored
-//        output position gives each thread its first output index, stage 2
-//        decodes again and places the exponents in an on-chip write buffer,
-//        and the block's outputs leave in one coalesced write; the encoded
-//        stream is in shared memory before stage 1;
+//        codes of each segment, a prefix sum over the thread block plus the
+//        block's stored output position gives each thread its first output
+//        index, stage 2 decodes again and places the exponents in an on-chip
+//        write buffer, and the block's outputs leave in one coalesced write;
 //   "Format DFloat11" -- sign and mantissa come verbatim from
 //        PackedSignMantissa.
 //
 // B200 design (what differs from the page's kernel):
-//   * persistent CTAs (a multiple of the SM count) walk the blocks; each
-//     CTA stages the page's LUTs and CodeLengths once and derives two wider
-//     tables from them in shared memory:
+//   * the format's thread block is one warp (T = 32 segments): a block's
+//     prefix sum is five warp shuffles and its write buffer is private to
+//     the warp, so warps never wait for one another -- no block-wide barrier
+//     after set-up.  One persistent CTA of 32 warps runs per SM and every
+//     warp walks its own sequence of blocks;
+//   * the CTA stages the page's LUTs and CodeLengths once and derives two
+//     wider tables from them in shared memory, shared by its 32 warps:
 //       - a count table over the next 12 bits: how many whole codes they
 //         hold and how many bits those codes use (stage 1 advances about 10
 //         bits per lookup);
@@ -26,23 +29,18 @@
 //         lookup).  Exponents are stored rotated right by one bit, which
 //         turns the final BF16 merge into two bit-selects and two byte
 //         permutes per 4 elements.
-//     Codes longer than 12 bits fall back to the page's pointer-chasing LUTs.
+//     Codes longer than 12 bits fall back to the page's pointer-chasing LUTs;
 //   * stage 1 stops exactly at the thread's last code: the next segment's
 //     Gap gives the bit where the next thread starts; the final lookup masks
 //     the bits past that point to zeros, and the codes the zeros form (the
-//     all-zero code is the canonical first code) are subtracted.
+//     all-zero code is the canonical first code) are subtracted;
 //   * stage 2 runs until the thread has placed as many exponents as stage 1
-//     counted; no second end test is needed.
+//     counted;
 //   * each thread's 64 + 32 bits live in a three-register shift window: the
-//     table index is the top 12 bits, a step is three funnel shifts.
-//   * the next block's EncodedExponent slice, Gaps words and
-//     PackedSignMantissa slice are fetched by bulk asynchronous copies
-//     (cp.async.bulk, completion on an mbarrier) while the current block is
-//     decoded: two buffers per CTA.
-//   * the block prefix sum is a warp-shuffle scan plus a scan of warp totals
-//     (the page uses Blelloch's tree scan).
-// Every loop and every wait is bounded; inconsistent data sets a status word
-// and never traps.
+//     table index is the top 12 bits, a step is three funnel shifts;
+//   * the next block's stream words, Gaps words and offsets are loaded into
+//     registers while the current block is decoded.
+// Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -52,11 +50,13 @@
 
 namespace {
 
-constexpr int kIdxBits = 12;                // index width of both derived tables
+constexpr int kIdxBits = 12;  // index width of both derived tables
 constexpr int kIdxEntries = 1 << kIdxBits;
 constexpr int kLutBytes = DF11_MAX_LUTS * 256;
 constexpr uint32_t kPointerBase = 240;
-constexpr uint32_t kWaitTries = 1u << 22;   // bounded mbarrier polling
+constexpr int kBlockSegs = 32;  // segments per format block = lanes per warp
+constexpr int kWarps = 32;      // warps per CTA
+constexpr int kThreads = kWarps * 32;
 
 struct Params {
     const uint8_t *stream;
@@ -72,93 +72,25 @@ struct Params {
     uint64_t nseg;
     uint32_t nblocks;
     uint32_t num_luts;
-    uint32_t sm_cap;  // bytes of one PackedSignMantissa / exponent buffer
+    uint32_t cap;  // bytes of one warp's exponent buffer
 };
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
-// Per-block bytes of the Gaps slice: fields T b .. T b + T (the extra field
-// is the next block's first gap), whole 64-bit words, rounded to 16 bytes.
-__host__ __device__ constexpr uint32_t gaps_slice_bytes(uint32_t T) { return align16((5 * T) / 8 + 16); }
-__host__ __device__ constexpr uint32_t stream_slice_bytes(uint32_t T) { return T * 8 + 16; }
-
-// Shared-memory layout in bytes.  The derived tables sit at fixed offsets so
-// lookups need no base register.
-struct SmemLayout {
-    static constexpr uint32_t sym = 0;                              // uint32[4096]
-    static constexpr uint32_t cnt = sym + kIdxEntries * 4;          // uint8[4096]
-    static constexpr uint32_t luts = cnt + kIdxEntries;             // 17 * 256
-    static constexpr uint32_t cl = luts + kLutBytes;                // 256
-    static constexpr uint32_t ztab = cl + 256;                      // uint16[16]
-    static constexpr uint32_t warp = ztab + 32;                     // uint32[32]
-    static constexpr uint32_t bar = warp + 128;                     // 2 mbarriers
-    static constexpr uint32_t scal = bar + 16;                      // 2 x {o0, o1, bad, pad}
-    static constexpr uint32_t bufs = scal + 32;
-    uint32_t buf_stride, stream_off, gaps_off, sm_off, exps, total;
-    __host__ __device__ SmemLayout(uint32_t T, uint32_t sm_cap)
-    {
-        stream_off = 0;
-        gaps_off = stream_off + align16(stream_slice_bytes(T));
-        sm_off = gaps_off + gaps_slice_bytes(T);
-        buf_stride = sm_off + sm_cap;
-        exps = bufs + 2 * buf_stride;
-        total = exps + sm_cap;
-    }
+// Shared memory: tables at fixed offsets (lookups need no base register),
+// then one exponent buffer per warp.
+struct Smem {
+    static constexpr uint32_t sym = 0;                       // uint32[4096]
+    static constexpr uint32_t cnt = sym + kIdxEntries * 4;   // uint8[4096]
+    static constexpr uint32_t luts = cnt + kIdxEntries;      // 17 * 256
+    static constexpr uint32_t cl = luts + kLutBytes;         // 256
+    static constexpr uint32_t ztab = cl + 256;               // uint16[16]
+    static constexpr uint32_t bufs = ztab + 32;
+    static constexpr uint32_t bytes(uint32_t cap) { return bufs + kWarps * cap; }
 };
-static_assert(SmemLayout::bufs % 16 == 0, "buffers must be 16-byte aligned");
+static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// Bounded wait for the phase with the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
-{
-    for (uint32_t i = 0; i < kWaitTries; i++) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
-
-// Bulk global -> shared copy (no multicast), completion counted in bytes on
-// the mbarrier.  Addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t load_be32(const uint8_t *p)
-{
-    return __byte_perm(*reinterpret_cast<const uint32_t *>(p), 0, 0x0123);
-}
+__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
 __device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
 
@@ -195,38 +127,6 @@ __device__ __forceinline__ void shift_window(uint32_t &h, uint32_t &m, uint32_t 
     l = __funnelshift_lc(0u, l, c);
 }
 
-// Exclusive prefix sum over the block; *total receives the block sum.
-template <int T>
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t *total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, d);
-        if (lane >= d)
-            x += y;
-    }
-    if (lane == 31)
-        warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t s = lane < T / 32 ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, s, d);
-            if (lane >= d)
-                s += y;
-        }
-        if (lane < T / 32)
-            warp_sums[lane] = s;
-    }
-    __syncthreads();
-    uint32_t before = warp ? warp_sums[warp - 1] : 0;
-    *total = warp_sums[T / 32 - 1];
-    return before + x - v;
-}
-
 // Four BF16 values from four sign/mantissa bytes S and four rotated exponent
 // bytes E (ror8(e) = e >> 1 | (e & 1) << 7):
 //   high byte = sign | e >> 1,  low byte = (e & 1) << 7 | mantissa.
@@ -243,64 +143,47 @@ __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
     return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
 }
 
-template <int T>
-__global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
+// Registers one lane holds for one block: its stream words (raw), the Gaps
+// word pair holding its field and the next one, and the block's offsets.
+struct BlockRegs {
+    uint2 s01;
+    uint32_t s2;
+    uint64_t g0, g1;
+    uint32_t o0, o1;
+};
+
+__device__ __forceinline__ void load_block(const Params &p, uint32_t b, int lane, BlockRegs &r)
+{
+    const uint8_t *s = p.stream + (uint64_t)b * (kBlockSegs * 8) + 8 * lane;
+    r.s01 = __ldg(reinterpret_cast<const uint2 *>(s));
+    r.s2 = __ldg(reinterpret_cast<const uint32_t *>(s + 8));
+    const uint64_t bit = 5ull * ((uint64_t)b * kBlockSegs + lane);
+    const uint64_t w = bit >> 6;
+    r.g0 = __ldg(p.gaps + w);
+    r.g1 = __ldg(p.gaps + w + 1);
+    r.o0 = __ldg(p.offs + b);
+    r.o1 = __ldg(p.offs + b + 1);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    const SmemLayout L(T, p.sm_cap);
-    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + SmemLayout::sym);
-    uint8_t *cnt_tab = smem + SmemLayout::cnt;
-    uint8_t *luts = smem + SmemLayout::luts;
-    uint8_t *cl = smem + SmemLayout::cl;
-    uint16_t *ztab = reinterpret_cast<uint16_t *>(smem + SmemLayout::ztab);
-    uint32_t *warp_sums = reinterpret_cast<uint32_t *>(smem + SmemLayout::warp);
-    uint32_t *scal = reinterpret_cast<uint32_t *>(smem + SmemLayout::scal);
-    uint8_t *exp_s = smem + L.exps;
-    const uint32_t bar0 = smem_addr(smem + SmemLayout::bar);
-    const int tid = threadIdx.x;
-    const uint32_t G = gridDim.x;
+    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
+    uint8_t *cnt_tab = smem + Smem::cnt;
+    uint8_t *luts = smem + Smem::luts;
+    uint8_t *cl = smem + Smem::cl;
+    uint16_t *ztab = reinterpret_cast<uint16_t *>(smem + Smem::ztab);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *exp_s = smem + Smem::bufs + warp * p.cap;
 
-    // thread 0: fetch block b into buffer k (offsets from registers o0, o1)
-    auto issue = [&](uint32_t b, int k, uint32_t o0, uint32_t o1) {
-        uint8_t *buf = smem + SmemLayout::bufs + k * L.buf_stride;
-        const uint32_t bar = bar0 + 8 * k;
-        const uint32_t base = o0 & ~15u;
-        const uint64_t end16 = ((uint64_t)o1 + 15u) & ~(uint64_t)15u;
-        const bool ok = o1 >= o0 && (uint64_t)o1 <= p.n && end16 - base <= p.sm_cap;
-        const uint32_t sm_bytes = ok ? (uint32_t)(end16 - base) : 0u;
-        scal[4 * k + 0] = o0;
-        scal[4 * k + 1] = o1;
-        scal[4 * k + 2] = ok ? 0u : 1u;
-        fence_proxy_async();
-        mbar_arrive_expect_tx(bar, stream_slice_bytes(T) + gaps_slice_bytes(T) + sm_bytes);
-        bulk_copy(smem_addr(buf + L.stream_off), p.stream + (uint64_t)b * T * 8, stream_slice_bytes(T), bar);
-        bulk_copy(smem_addr(buf + L.gaps_off), reinterpret_cast<const uint8_t *>(p.gaps) + (uint64_t)b * (5 * T / 8),
-                  gaps_slice_bytes(T), bar);
-        if (sm_bytes)
-            bulk_copy(smem_addr(buf + L.sm_off), p.sm + base, sm_bytes, bar);
-    };
-
-    // ---- once per CTA: barriers, the page's LUTs, derived tables
-    uint32_t next_o0 = 0, next_o1 = 0;
-    if (tid == 0) {
-        mbar_init(bar0, 1);
-        mbar_init(bar0 + 8, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        fence_proxy_async();
-        const uint32_t b = blockIdx.x;
-        issue(b, 0, __ldg(p.offs + b), __ldg(p.offs + b + 1));
-        if (b + G < p.nblocks) {
-            next_o0 = __ldg(p.offs + b + G);
-            next_o1 = __ldg(p.offs + b + G + 1);
-        }
-    }
+    // ---- once per CTA: the page's LUTs and CodeLengths, derived tables
     const uint32_t lut_bytes = p.num_luts * 256u;
-    for (uint32_t i = tid; i < lut_bytes; i += T)
+    for (uint32_t i = tid; i < lut_bytes; i += kThreads)
         luts[i] = p.luts[i];
-    for (uint32_t i = tid; i < 256; i += T)
+    for (uint32_t i = tid; i < 256; i += kThreads)
         cl[i] = p.cl[i];
     __syncthreads();
-    for (uint32_t i = tid; i < kIdxEntries; i += T) {
+    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
         const uint32_t w = i << (32 - kIdxBits);
         uint32_t pos = 0, ncodes = 0, syms = 0, sym_bits = 0, sym_n = 0;
         for (int it = 0; it < kIdxBits; it++) {
@@ -318,11 +201,12 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
             pos += len;
         }
         cnt_tab[i] = (uint8_t)(ncodes | (pos << 4));
-        sym_tab[i] = syms | (sym_bits << 24) | (sym_n << 28);
+        // exponents in bytes 0..2, count in bits 24..25, total length in 28..31
+        sym_tab[i] = syms | (sym_n << 24) | (sym_bits << 28);
     }
     if (tid <= kIdxBits) {
-        // codes formed by r..11 zero bits after a code boundary: the all-zero
-        // code (the canonical first code) repeated; count | bits << 8
+        // codes formed by the zero bits r..11 after a code boundary: the
+        // all-zero code (the canonical first code) repeated; count | bits << 8
         bool bad = false;
         const uint32_t lmin = lut_decode(0u, luts, cl, p.num_luts, &bad) >> 8;
         const uint32_t z = (lmin >= 1 && !bad) ? (kIdxBits - tid) / lmin : 0u;
@@ -330,49 +214,33 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
     }
     __syncthreads();
 
-    uint32_t i = 0;
-    for (uint32_t b = blockIdx.x; b < p.nblocks; b += G, i++) {
-        const int k = i & 1;
-        if (tid == 0 && b + G < p.nblocks) {
-            issue(b + G, k ^ 1, next_o0, next_o1);
-            if (b + 2 * G < p.nblocks) {
-                next_o0 = __ldg(p.offs + b + 2 * G);
-                next_o1 = __ldg(p.offs + b + 2 * G + 1);
-            }
-        }
-        const bool timed_out = !mbar_wait(bar0 + 8 * k, (i >> 1) & 1);
-        if (__syncthreads_or(timed_out)) {
-            if (tid == 0)
-                atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
-            mbar_wait(bar0 + 8 * (k ^ 1), ((i + 1) >> 1) & 1);  // bounded: copies still in flight
-            return;
-        }
-        const uint8_t *buf = smem + SmemLayout::bufs + k * L.buf_stride;
-        const uint8_t *stream_s = buf + L.stream_off;
-        const uint64_t *gaps_s = reinterpret_cast<const uint64_t *>(buf + L.gaps_off);
-        const uint8_t *sm_s = buf + L.sm_off;
-        const uint32_t o0 = scal[4 * k + 0], o1 = scal[4 * k + 1];
-        const bool offs_bad = scal[4 * k + 2] != 0;
+    // ---- each warp walks its own blocks; no block-wide barrier from here on
+    const uint32_t stride = gridDim.x * kWarps;
+    uint32_t b = blockIdx.x * kWarps + warp;
+    BlockRegs cur, nxt;
+    if (b < p.nblocks)
+        load_block(p, b, lane, cur);
+    for (; b < p.nblocks; b += stride) {
+        if (b + stride < p.nblocks)
+            load_block(p, b + stride, lane, nxt);
+        const uint32_t o0 = cur.o0, o1 = cur.o1;
         const uint32_t lo_off = o0 & 15u;
 
-        // ---- locate: this thread's codes start in [pos0, pend) of its window
-        const uint64_t seg = (uint64_t)b * T + tid;
+        // ---- locate: this lane's codes start in [pos0, pend) of its window
+        const uint64_t seg = (uint64_t)b * kBlockSegs + lane;
         int pos0 = 0, pend = 0;
         {
-            const uint32_t bit = 5u * tid;
-            const uint32_t w = bit >> 6, off = bit & 63u;
-            uint64_t v = gaps_s[w] >> off;
-            if (off > 54)  // fields tid and tid + 1 reach into the next word
-                v |= gaps_s[w + 1] << (64 - off);
-            const uint32_t g0 = (uint32_t)v & 31u, g1 = (uint32_t)(v >> 5) & 31u;
+            const uint32_t off = (uint32_t)((5ull * seg) & 63);
+            uint64_t v = cur.g0 >> off;
+            if (off > 54)  // this field and the next reach into the second word
+                v |= cur.g1 << (64 - off);
+            const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
             if (seg < p.nseg) {
-                pos0 = (int)g0;
-                pend = seg + 1 < p.nseg ? 64 + (int)g1 : (int)(p.total_bits - 64 * seg);
+                pos0 = (int)gap;
+                pend = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
             }
         }
-        const uint32_t w0 = load_be32(stream_s + 8 * tid);
-        const uint32_t w1 = load_be32(stream_s + 8 * tid + 4);
-        const uint32_t w2 = load_be32(stream_s + 8 * tid + 8);
+        const uint32_t w0 = bswap32(cur.s01.x), w1 = bswap32(cur.s01.y), w2 = bswap32(cur.s2);
 
         // ---- stage 1: count the codes starting in [pos0, pend)
         bool bad = false;
@@ -381,11 +249,13 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
             uint32_t h = w0, m = w1, l = w2;
             shift_window(h, m, l, (uint32_t)pos0);
             int pos = pos0;
-            for (int it = 0; it < 64 && pend - pos > kIdxBits; it++) {
+            const int bulk_end = pend - kIdxBits;
+            while (pos < bulk_end) {  // pos strictly increases: at most 95 steps
                 uint32_t e = cnt_tab[h >> (32 - kIdxBits)];
                 uint32_t c = e >> 4;
                 if (c == 0) {  // a code longer than 12 bits
                     c = lut_decode(h, luts, cl, p.num_luts, &bad) >> 8;
+                    c = c ? c : 1u;
                     e = 1;
                 }
                 cnt += e & 15u;
@@ -393,9 +263,7 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
                 shift_window(h, m, l, c);
             }
             const int r = pend - pos;
-            if (r > kIdxBits) {
-                bad = true;  // the loop bound ran out: not a valid segment
-            } else if (r > 0) {
+            if (r > 0) {
                 // the last r <= 12 bits hold whole codes; mask the rest to zeros
                 const uint32_t idx = (h >> (32 - kIdxBits)) & ((0xFFFu << (kIdxBits - r)) & 0xFFFu);
                 const uint32_t e = cnt_tab[idx];
@@ -407,52 +275,56 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
             }
         }
 
-        uint32_t total;
-        const uint32_t first = block_exclusive_scan<T>(cnt, warp_sums, &total);
-        const bool block_bad = __syncthreads_or(bad) || offs_bad || total != o1 - o0 ||
-                               lo_off + total + 16u > p.sm_cap;
+        // ---- warp prefix sum of the counts
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d)
+                incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+        const uint32_t first = incl - cnt;
+        const bool block_bad = __any_sync(0xffffffffu, bad) || o1 < o0 || (uint64_t)o1 > p.n ||
+                               total != o1 - o0 || lo_off + total + 16u > p.cap;
         if (block_bad) {
-            if (tid == 0)
+            if (lane == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
-            __syncthreads();
-            continue;
-        }
-
-        // ---- stage 2: decode again, place rotated exponents
-        {
-            uint32_t h = w0, m = w1, l = w2;
-            shift_window(h, m, l, (uint32_t)pos0);
-            uint32_t q = lo_off + first;
-            const uint32_t qend = q + cnt;
-            for (int it = 0; it < 64 && q < qend; it++) {
-                uint32_t e = sym_tab[h >> (32 - kIdxBits)];
-                uint32_t c = (e >> 24) & 15u, nsym = e >> 28;
-                if (nsym == 0) {  // a code longer than 12 bits
-                    const uint32_t d = lut_decode(h, luts, cl, p.num_luts, &bad);
-                    e = ror8(d & 0xFFu);
-                    c = d >> 8;
-                    nsym = 1;
+        } else {
+            // ---- stage 2: decode again, place rotated exponents
+            {
+                uint32_t h = w0, m = w1, l = w2;
+                shift_window(h, m, l, (uint32_t)pos0);
+                uint32_t q = lo_off + first;
+                const uint32_t qend = q + cnt;
+                while (q < qend) {  // q strictly increases
+                    uint32_t e = sym_tab[h >> (32 - kIdxBits)];
+                    uint32_t c = e >> 28, nsym = (e >> 24) & 3u;
+                    if (nsym == 0) {  // a code longer than 12 bits
+                        const uint32_t d = lut_decode(h, luts, cl, p.num_luts, &bad);
+                        e = ror8(d & 0xFFu);
+                        c = d >> 8;
+                        nsym = 1;
+                    }
+                    exp_s[q] = (uint8_t)e;
+                    if (q + 1 < qend)
+                        exp_s[q + 1] = (uint8_t)(e >> 8);
+                    if (q + 2 < qend)
+                        exp_s[q + 2] = (uint8_t)(e >> 16);
+                    q += nsym;
+                    shift_window(h, m, l, c);
                 }
-                exp_s[q] = (uint8_t)e;
-                if (q + 1 < qend)
-                    exp_s[q + 1] = (uint8_t)(e >> 8);
-                if (q + 2 < qend)
-                    exp_s[q + 2] = (uint8_t)(e >> 16);
-                q += nsym;
-                shift_window(h, m, l, c);
             }
-        }
-        __syncthreads();
+            __syncwarp();
 
-        // ---- merge with sign/mantissa, coalesced 16-byte stores
-        {
+            // ---- merge with sign/mantissa, coalesced 16-byte stores
             const uint32_t hi = lo_off + total;
             const uint64_t g0 = (uint64_t)o0 - lo_off;  // multiple of 16
             const uint32_t nchunks = (hi + 15) / 16;
-            for (uint32_t c = tid; c < nchunks; c += T) {
+            for (uint32_t c = lane; c < nchunks; c += 32) {
                 const uint32_t l0 = 16 * c;
                 if (l0 >= lo_off && l0 + 16 <= hi) {
-                    const uint4 s = *reinterpret_cast<const uint4 *>(sm_s + l0);
+                    const uint4 s = __ldg(reinterpret_cast<const uint4 *>(p.sm + g0 + l0));
                     const uint4 e = *reinterpret_cast<const uint4 *>(exp_s + l0);
                     uint4 r0, r1;
                     merge4(s.x, e.x, r0.x, r0.y);
@@ -462,16 +334,19 @@ __global__ void __launch_bounds__(T) df11_decode_kernel(const Params p)
                     uint4 *d = reinterpret_cast<uint4 *>(p.dst + g0 + l0);
                     d[0] = r0;
                     d[1] = r1;
-                } else {
-                    for (uint32_t j = 0; j < 16; j++) {
-                        const uint32_t l = l0 + j;
-                        if (l >= lo_off && l < hi)
-                            p.dst[g0 + l] = merge1(sm_s[l], exp_s[l]);
-                    }
                 }
             }
+            // partial first / last chunk: one element per lane
+            {
+                const uint32_t chunk = lane < 16 ? 0u : nchunks - 1;
+                const uint32_t l = 16 * chunk + (lane & 15);
+                const bool partial = lo_off > 16 * chunk || 16 * chunk + 16 > hi;
+                if ((lane < 16 || nchunks > 1) && partial && l >= lo_off && l < hi)
+                    p.dst[g0 + l] = merge1(__ldg(p.sm + g0 + l), exp_s[l]);
+            }
+            __syncwarp();
         }
-        __syncthreads();
+        cur = nxt;
     }
 }
 
@@ -497,27 +372,6 @@ df11_status device_sms(int *sms)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-template <int T>
-df11_status launch(const Params &prm, cudaStream_t stream)
-{
-    const SmemLayout L(T, prm.sm_cap);
-    auto kern = df11_decode_kernel<T>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total) != cudaSuccess)
-        return DF11_ERR_CUDA;
-    int sms = 0;
-    df11_status st = device_sms(&sms);
-    if (st != DF11_OK)
-        return st;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, L.total) != cudaSuccess || per_sm < 1)
-        return DF11_ERR_CUDA;
-    uint64_t grid = (uint64_t)sms * (uint64_t)per_sm;
-    if (grid > prm.nblocks)
-        grid = prm.nblocks;
-    kern<<<(unsigned)grid, T, L.total, stream>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream)
@@ -526,25 +380,24 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
         return DF11_ERR_INVALID_ARG;
     if (a->n == 0)
         return DF11_OK;
-    const uint32_t T = a->threads_per_block;
-    if (T != 128 && T != 256 && T != 512)
+    if (a->threads_per_block != kBlockSegs)
         return DF11_ERR_INVALID_ARG;
     if (!dst || !a->encoded_exponent || !a->packed_sign_mantissa || !a->gaps || !a->block_offset || !a->luts ||
         !a->code_lengths)
         return DF11_ERR_INVALID_ARG;
     if (!aligned(dst, 16) || !aligned(a->encoded_exponent, 16) || !aligned(a->packed_sign_mantissa, 16) ||
-        !aligned(a->gaps, 16) || !aligned(a->block_offset, 4))
+        !aligned(a->gaps, 8) || !aligned(a->block_offset, 4))
         return DF11_ERR_INVALID_ARG;
     if (a->num_luts < 1 || a->num_luts > DF11_MAX_LUTS || a->n >= (1ull << 32))
         return DF11_ERR_INVALID_ARG;
     const uint64_t nseg = (a->total_bits + 63) / 64;
-    if (nseg != a->num_segments || (nseg + T - 1) / T != a->num_blocks || a->num_blocks == 0)
+    if (nseg != a->num_segments || (nseg + kBlockSegs - 1) / kBlockSegs != a->num_blocks || a->num_blocks == 0)
         return DF11_ERR_INVALID_ARG;
-    // every bulk copy must stay inside its array
-    if (a->encoded_exponent_bytes < (uint64_t)a->num_blocks * T * 8 + 16 ||
+    // every load stays inside its array
+    if (a->encoded_exponent_bytes < (uint64_t)a->num_blocks * kBlockSegs * 8 + 16 ||
         a->packed_sign_mantissa_bytes < ((a->n + 15) / 16) * 16 ||
-        a->gaps_words * 8 < (uint64_t)(a->num_blocks - 1) * (5 * T / 8) + gaps_slice_bytes(T) ||
-        a->max_block_elems > 64u * T)
+        a->gaps_words < (5ull * a->num_blocks * kBlockSegs + 63) / 64 + 2 ||
+        a->max_block_elems > 64u * kBlockSegs)
         return DF11_ERR_INVALID_ARG;
 
     Params prm;
@@ -561,13 +414,26 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     prm.nseg = nseg;
     prm.nblocks = a->num_blocks;
     prm.num_luts = a->num_luts;
-    prm.sm_cap = align16(a->max_block_elems + 32);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    switch (T) {
-    case 128: return launch<128>(prm, s);
-    case 256: return launch<256>(prm, s);
-    default: return launch<512>(prm, s);
-    }
+    prm.cap = align16(a->max_block_elems + 32);
+
+    const uint32_t smem = Smem::bytes(prm.cap);
+    if (cudaFuncSetAttribute(df11_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return DF11_ERR_CUDA;
+    int sms = 0;
+    df11_status st = device_sms(&sms);
+    if (st != DF11_OK)
+        return st;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, df11_decode_kernel, kThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        return DF11_ERR_CUDA;
+    uint64_t grid = (uint64_t)sms * (uint64_t)per_sm;
+    const uint64_t need = (a->num_blocks + kWarps - 1) / kWarps;
+    if (grid > need)
+        grid = need;
+    df11_decode_kernel<<<(unsigned)grid, kThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
 extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arrays *d, uint16_t *dst_dev,
