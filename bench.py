@@ -50,7 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5],
                     help="1 single 1024x1024, 2 Llama-3-8B block, 3 stress 64Mi, "
                          "4 Llama-3-70B block, 5 32 Llama-3-8B blocks streamed")
-    ap.add_argument("--threads-per-block", type=int, default=32)
+    ap.add_argument("--threads-per-block", type=int, default=64)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -75,6 +75,22 @@ def shard(workload: int, rank: int, world: int):
     if workload == 5:
         return [(5, b) for b in range(32) if b % world == rank]
     return [(workload, rank)]
+
+
+def reduce_over_ranks(ms_step, e2e_ms, n_elems, good, device, world):
+    """Whole-job numbers: the slowest rank's times, the elements of all
+    ranks, and bit-exactness only if every rank was exact."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms_step, e2e_ms], dtype=torch.float64, device=device)
+    n = torch.tensor([float(n_elems)], dtype=torch.float64, device=device)
+    g = torch.tensor([1.0 if good else 0.0], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+        dist.all_reduce(g, op=dist.ReduceOp.MIN)
+    return float(t[0]), float(t[1]), float(n[0]), bool(g[0] > 0)
 
 
 def scaling_kind(workload: int) -> str:
@@ -284,17 +300,7 @@ def run_gpu(args):
     ok = ok and df11.read_status(status) == 0
     clocks = sampler.stop() if sampler else None
 
-    # reduce over ranks: max time, summed elements
-    stats = torch.tensor([ms_mean, e2e_ms, float(n_total), float(exact and ok)], dtype=torch.float64, device=device)
-    if world > 1:
-        t_max = stats[:2].clone()
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-        n_sum = stats[2:3].clone()
-        dist.all_reduce(n_sum, op=dist.ReduceOp.SUM)
-        good = stats[3:4].clone()
-        dist.all_reduce(good, op=dist.ReduceOp.MIN)
-        stats = torch.cat([t_max, n_sum, good])
-    ms_step, e2e_ms, n_all, good = stats.tolist()
+    ms_step, e2e_ms, n_all, good = reduce_over_ranks(ms_mean, e2e_ms, n_total, exact and ok, device, world)
 
     if rank == 0:
         info0 = prepared[0]["info"]
@@ -376,7 +382,7 @@ def _oracle_sample(workload: int, elems: int):
     mats = [m for _, _, m in inputs.workload_arrays(1 if workload == 1 else (2 if workload == 5 else workload), 0)]
     w = np.concatenate(mats) if len(mats) > 1 else mats[0]
     w = np.ascontiguousarray(w[:elems])
-    return oracle, oracle.build_format(w, 32)
+    return oracle, oracle.build_format(w, 64)
 
 
 def cpu_baseline(workload: int, seconds: float) -> dict:

@@ -142,9 +142,10 @@ class Format:
         self.free()
 
     def free(self):
-        if getattr(self, "_h", None) and self._h.value:
-            self._lib.df11_free(self._h)
-            self._h = ctypes.c_void_p(0)
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.df11_free(h)
+            self._h = None
 
     @property
     def n(self) -> int:
@@ -189,7 +190,7 @@ class Format:
             "max_code_len", "max_block_elems")}
 
 
-def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 32) -> Format:
+def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 64) -> Format:
     """Compresses BF16 bit patterns (uint16 arrays, or torch bfloat16/int16
     CPU tensors) into one DF11 stream; matrices are concatenated in order."""
     lib = load_library()

@@ -14,13 +14,16 @@
 //        PackedSignMantissa.
 //
 // B200 design (what differs from the page's kernel):
-//   * the format's thread block is one warp (T = 32 segments): a block's
-//     prefix sum is five warp shuffles and its write buffer is private to
-//     the warp, so warps never wait for one another -- no block-wide barrier
-//     after set-up.  One persistent CTA of 32 warps runs per SM and every
-//     warp walks its own sequence of blocks;
+//   * the format's thread block is one warp (T = 32 or 64 segments; with 64
+//     each lane decodes two segments as two independent chains, which keeps
+//     two lookups in flight per thread): a block's prefix sum is five warp
+//     shuffles and its write buffer is private to the warp, so warps never
+//     wait for one another -- no block-wide barrier after set-up.  One
+//     persistent CTA of 32 warps runs per SM and every warp walks its own
+//     sequence of blocks;
 //   * the CTA stages the page's LUTs and CodeLengths once and derives two
-//     wider tables from them in shared memory, shared by its 32 warps:
+//     wider tables from them in shared memory, shared by its 32 warps (via a
+//     scratch table of the first code of every 12-bit window):
 //       - a count table over the next 12 bits: how many whole codes they
 //         hold and how many bits those codes use (stage 1 advances about 10
 //         bits per lookup);
@@ -38,8 +41,14 @@
 //     counted;
 //   * each thread's 64 + 32 bits live in a three-register shift window: the
 //     table index is the top 12 bits, a step is three funnel shifts;
+//   * the two decode loops are hand-written PTX: both chains of a lane step
+//     in one predicated loop, so the warp runs max(chain A, chain B) passes;
+//     stage 1 adds raw table entries (codes + 16 * bits) and recovers the
+//     count from the bits advanced;
 //   * the next block's stream words, Gaps words and offsets are loaded into
-//     registers while the current block is decoded.
+//     registers while the current block is decoded; the current block's
+//     sign/mantissa bytes arrive in shared memory by asynchronous copies
+//     (cp.async) during the two decode stages.
 // Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
 
@@ -50,18 +59,16 @@
 
 namespace {
 
-constexpr int kIdxBits = 12;  // index width of both derived tables
+constexpr int kIdxBits = 12;  // index width of the derived tables
 constexpr int kIdxEntries = 1 << kIdxBits;
 constexpr int kLutBytes = DF11_MAX_LUTS * 256;
 constexpr uint32_t kPointerBase = 240;
-constexpr int kBlockSegs = 32;  // segments per format block = lanes per warp
-constexpr int kWarps = 32;      // warps per CTA
-constexpr int kThreads = kWarps * 32;
+constexpr int kMaxWarps = 32;  // warps per CTA (fewer when a block's buffers are large)
 
 struct Params {
     const uint8_t *stream;
     const uint8_t *sm;
-    const uint64_t *gaps;
+    const uint32_t *gaps;  // the uint64 Gaps words read as little-endian halves
     const uint32_t *offs;
     const uint8_t *luts;
     const uint8_t *cl;
@@ -72,13 +79,14 @@ struct Params {
     uint64_t nseg;
     uint32_t nblocks;
     uint32_t num_luts;
-    uint32_t cap;  // bytes of one warp's exponent buffer
+    uint32_t cap;  // bytes of one warp's exponent (and sign/mantissa) buffer
 };
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
 // Shared memory: tables at fixed offsets (lookups need no base register),
-// then one exponent buffer per warp.
+// then two buffers per warp: placed exponents and the block's
+// sign/mantissa bytes.
 struct Smem {
     static constexpr uint32_t sym = 0;                       // uint32[4096]
     static constexpr uint32_t cnt = sym + kIdxEntries * 4;   // uint8[4096]
@@ -86,7 +94,7 @@ struct Smem {
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
     static constexpr uint32_t ztab = cl + 256;               // uint16[16]
     static constexpr uint32_t bufs = ztab + 32;
-    static constexpr uint32_t bytes(uint32_t cap) { return bufs + kWarps * cap; }
+    static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * 2 * cap; }
 };
 static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
 
@@ -143,30 +151,161 @@ __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
     return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
 }
 
-// Registers one lane holds for one block: its stream words (raw), the Gaps
-// word pair holding its field and the next one, and the block's offsets.
+__device__ __forceinline__ void cp_async16(uint8_t *dst_smem, const void *src)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+
+// Stage-1 bulk loop for two chains (A, B) of one lane, in PTX so that each
+// lookup costs a fixed, short instruction sequence.  Per active chain and
+// lookup: index = top 12 bits of the window (mad.hi adds the table base),
+// entry = codes | bits << 4, sum += entry (the code count is recovered as
+// sum - 16 * bits), advance the 96-bit window.  A chain is active while
+// pos < bulk_end.  Leaves early, state intact, when an active chain meets a
+// code longer than 12 bits (entry bits == 0); the caller resolves it.
+__device__ __forceinline__ void count_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &sA, int &posA,
+                                            uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &sB, int &posB,
+                                            int bendA, int bendB, uint32_t cnt_base)
+{
+    asm volatile(
+        "{\n\t"
+        ".reg .pred pa, pb, pz, pl;\n\t"
+        ".reg .u32 ea, eb, ca, cb;\n\t"
+        "CB_TOP:\n\t"
+        "setp.lt.s32 pa, %4, %10;\n\t"
+        "setp.lt.s32 pb, %9, %11;\n\t"
+        "or.pred pz, pa, pb;\n\t"
+        "@!pz bra CB_END;\n\t"
+        "@pa mad.hi.u32 ea, %0, 4096, %12;\n\t"
+        "@pb mad.hi.u32 eb, %5, 4096, %12;\n\t"
+        "@pa ld.shared.u8 ea, [ea];\n\t"
+        "@pb ld.shared.u8 eb, [eb];\n\t"
+        "@pa shr.u32 ca, ea, 4;\n\t"
+        "@pb shr.u32 cb, eb, 4;\n\t"
+        "setp.eq.and.u32 pl, ca, 0, pa;\n\t"
+        "setp.eq.and.u32 pz, cb, 0, pb;\n\t"
+        "or.pred pl, pl, pz;\n\t"
+        "@pl bra CB_END;\n\t"
+        "@pa add.u32 %3, %3, ea;\n\t"
+        "@pa add.s32 %4, %4, ca;\n\t"
+        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
+        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
+        "@pa shl.b32 %2, %2, ca;\n\t"
+        "@pb add.u32 %8, %8, eb;\n\t"
+        "@pb add.s32 %9, %9, cb;\n\t"
+        "@pb shf.l.wrap.b32 %5, %6, %5, cb;\n\t"
+        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
+        "@pb shl.b32 %7, %7, cb;\n\t"
+        "bra CB_TOP;\n\t"
+        "CB_END:\n\t"
+        "}"
+        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(sA), "+r"(posA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(sB), "+r"(posB)
+        : "r"(bendA), "r"(bendB), "r"(cnt_base)
+        : "memory");
+}
+
+// Stage-2 loop for two chains, in PTX.  Symbol-table entry: up to three
+// rotated exponents in bytes 0..2, their total length in bits 24..28, their
+// number in bits 29..30 (0 = a code longer than 12 bits).  The length is
+// used as a funnel-shift amount in wrap mode, which reads only its low five
+// bits, so (entry >> 24) serves directly.  Each active chain stores one to
+// three exponent bytes at its shared-memory cursor q (q < qend), bytes two
+// and three only while they stay below qend.  Leaves early, state intact,
+// when an active chain meets a long code.
+__device__ __forceinline__ void place_loop2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA,
+                                            uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
+                                            uint32_t qendA, uint32_t qend1A, uint32_t qend2A, uint32_t qendB,
+                                            uint32_t qend1B, uint32_t qend2B, uint32_t sym_base)
+{
+    asm volatile(
+        "{\n\t"
+        ".reg .pred pa, pb, pz, pl, p1, p2;\n\t"
+        ".reg .u32 ea, eb, ca, cb, na, nb, t;\n\t"
+        "PL_TOP:\n\t"
+        "setp.lt.u32 pa, %3, %8;\n\t"
+        "setp.lt.u32 pb, %7, %11;\n\t"
+        "or.pred pz, pa, pb;\n\t"
+        "@!pz bra PL_END;\n\t"
+        "@pa shr.u32 ea, %0, 20;\n\t"
+        "@pb shr.u32 eb, %4, 20;\n\t"
+        "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"
+        "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"
+        "@pa ld.shared.u32 ea, [ea];\n\t"
+        "@pb ld.shared.u32 eb, [eb];\n\t"
+        "setp.eq.and.u32 pl, ea, 0, pa;\n\t"
+        "setp.eq.and.u32 pz, eb, 0, pb;\n\t"
+        "or.pred pl, pl, pz;\n\t"
+        "@pl bra PL_END;\n\t"
+        "@pa shr.u32 ca, ea, 24;\n\t"
+        "@pa shr.u32 na, ea, 29;\n\t"
+        "@pa st.shared.u8 [%3], ea;\n\t"
+        "setp.lt.and.u32 p1, %3, %9, pa;\n\t"
+        "setp.lt.and.u32 p2, %3, %10, pa;\n\t"
+        "@p1 shr.u32 t, ea, 8;\n\t"
+        "@p1 st.shared.u8 [%3+1], t;\n\t"
+        "@p2 shr.u32 t, ea, 16;\n\t"
+        "@p2 st.shared.u8 [%3+2], t;\n\t"
+        "@pa add.u32 %3, %3, na;\n\t"
+        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
+        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
+        "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
+        "@pb shr.u32 cb, eb, 24;\n\t"
+        "@pb shr.u32 nb, eb, 29;\n\t"
+        "@pb st.shared.u8 [%7], eb;\n\t"
+        "setp.lt.and.u32 p1, %7, %12, pb;\n\t"
+        "setp.lt.and.u32 p2, %7, %13, pb;\n\t"
+        "@p1 shr.u32 t, eb, 8;\n\t"
+        "@p1 st.shared.u8 [%7+1], t;\n\t"
+        "@p2 shr.u32 t, eb, 16;\n\t"
+        "@p2 st.shared.u8 [%7+2], t;\n\t"
+        "@pb add.u32 %7, %7, nb;\n\t"
+        "@pb shf.l.wrap.b32 %4, %5, %4, cb;\n\t"
+        "@pb shf.l.wrap.b32 %5, %6, %5, cb;\n\t"
+        "@pb shf.l.wrap.b32 %6, 0, %6, cb;\n\t"
+        "bra PL_TOP;\n\t"
+        "PL_END:\n\t"
+        "}"
+        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB)
+        : "r"(qendA), "r"(qend1A), "r"(qend2A), "r"(qendB), "r"(qend1B), "r"(qend2B), "r"(sym_base)
+        : "memory");
+}
+
+// Registers one lane holds for one block: per chain its 12 stream bytes and
+// the Gaps words holding its field and the next one; the block's offsets.
+template <int C>
 struct BlockRegs {
-    uint2 s01;
-    uint32_t s2;
-    uint64_t g0, g1;
+    uint2 s01[C];
+    uint32_t s2[C];
+    uint32_t g0[C], g1[C];
     uint32_t o0, o1;
 };
 
-__device__ __forceinline__ void load_block(const Params &p, uint32_t b, int lane, BlockRegs &r)
+template <int C>
+__device__ __forceinline__ void load_block(const Params &p, uint32_t b, int lane, BlockRegs<C> &r)
 {
-    const uint8_t *s = p.stream + (uint64_t)b * (kBlockSegs * 8) + 8 * lane;
-    r.s01 = __ldg(reinterpret_cast<const uint2 *>(s));
-    r.s2 = __ldg(reinterpret_cast<const uint32_t *>(s + 8));
-    const uint64_t bit = 5ull * ((uint64_t)b * kBlockSegs + lane);
-    const uint64_t w = bit >> 6;
-    r.g0 = __ldg(p.gaps + w);
-    r.g1 = __ldg(p.gaps + w + 1);
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+        const uint64_t seg = (uint64_t)b * (32 * C) + lane + 32 * k;
+        const uint8_t *s = p.stream + 8 * seg;
+        r.s01[k] = __ldg(reinterpret_cast<const uint2 *>(s));
+        r.s2[k] = __ldg(reinterpret_cast<const uint32_t *>(s + 8));
+        const uint64_t w = (5 * seg) >> 5;
+        r.g0[k] = __ldg(p.gaps + w);
+        r.g1[k] = __ldg(p.gaps + w + 1);
+    }
     r.o0 = __ldg(p.offs + b);
     r.o1 = __ldg(p.offs + b + 1);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p)
+// C = segments per lane: the format block is 32 * C segments, one warp; lane
+// l decodes segments l, l + 32, ... as C independent chains.  WARPS warps per
+// CTA, one CTA per SM.
+template <int C, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params p)
 {
+    constexpr int kWarps = WARPS, kThreads = WARPS * 32;
+    constexpr uint32_t T = 32 * C;
     extern __shared__ __align__(128) uint8_t smem[];
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
     uint8_t *cnt_tab = smem + Smem::cnt;
@@ -174,7 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p
     uint8_t *cl = smem + Smem::cl;
     uint16_t *ztab = reinterpret_cast<uint16_t *>(smem + Smem::ztab);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint8_t *exp_s = smem + Smem::bufs + warp * p.cap;
+    uint8_t *exp_s = smem + Smem::bufs + warp * 2 * p.cap;
+    uint8_t *sm_s = exp_s + p.cap;
 
     // ---- once per CTA: the page's LUTs and CodeLengths, derived tables
     const uint32_t lut_bytes = p.num_luts * 256u;
@@ -183,14 +323,25 @@ __global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p
     for (uint32_t i = tid; i < 256; i += kThreads)
         cl[i] = p.cl[i];
     __syncthreads();
+    // first code of every 12-bit window (zero filled): symbol | length << 8,
+    // length 0 when the code is longer than 12 bits.  Kept in the per-warp
+    // buffers, which are free until the blocks start.
+    uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
     for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
-        const uint32_t w = i << (32 - kIdxBits);
+        bool bad = false;
+        const uint32_t e = lut_decode(i << (32 - kIdxBits), luts, cl, p.num_luts, &bad);
+        const uint32_t len = e >> 8;
+        first_code[i] = (!bad && len >= 1 && len <= kIdxBits) ? (uint16_t)e : (uint16_t)0;
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
         uint32_t pos = 0, ncodes = 0, syms = 0, sym_bits = 0, sym_n = 0;
         for (int it = 0; it < kIdxBits; it++) {
-            bool bad = false;
-            const uint32_t e = lut_decode(w << pos, luts, cl, p.num_luts, &bad);
+            // the window after `pos` bits; its tail is zero filled, and a code
+            // found there is genuine only if it ends inside the 12 bits
+            const uint32_t e = first_code[(i << pos) & (kIdxEntries - 1)];
             const uint32_t len = e >> 8;
-            if (bad || len < 1 || pos + len > kIdxBits)
+            if (len == 0 || pos + len > kIdxBits)
                 break;
             if (ncodes < 3) {
                 syms |= ror8(e & 0xFFu) << (8 * ncodes);
@@ -201,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p
             pos += len;
         }
         cnt_tab[i] = (uint8_t)(ncodes | (pos << 4));
-        // exponents in bytes 0..2, count in bits 24..25, total length in 28..31
-        sym_tab[i] = syms | (sym_n << 24) | (sym_bits << 28);
+        // exponents in bytes 0..2, total length in bits 24..28, count in 29..30
+        sym_tab[i] = syms | (sym_bits << 24) | (sym_n << 29);
     }
     if (tid <= kIdxBits) {
         // codes formed by the zero bits r..11 after a code boundary: the
@@ -217,132 +368,197 @@ __global__ void __launch_bounds__(kThreads, 1) df11_decode_kernel(const Params p
     // ---- each warp walks its own blocks; no block-wide barrier from here on
     const uint32_t stride = gridDim.x * kWarps;
     uint32_t b = blockIdx.x * kWarps + warp;
-    BlockRegs cur, nxt;
+    BlockRegs<C> cur, nxt;
     if (b < p.nblocks)
-        load_block(p, b, lane, cur);
+        load_block<C>(p, b, lane, cur);
     for (; b < p.nblocks; b += stride) {
         if (b + stride < p.nblocks)
-            load_block(p, b + stride, lane, nxt);
+            load_block<C>(p, b + stride, lane, nxt);
         const uint32_t o0 = cur.o0, o1 = cur.o1;
         const uint32_t lo_off = o0 & 15u;
+        const uint64_t g0 = (uint64_t)o0 - lo_off;  // multiple of 16
+        const bool offs_ok = o1 >= o0 && (uint64_t)o1 <= p.n && (uint64_t)lo_off + (o1 - o0) + 16u <= p.cap;
 
-        // ---- locate: this lane's codes start in [pos0, pend) of its window
-        const uint64_t seg = (uint64_t)b * kBlockSegs + lane;
-        int pos0 = 0, pend = 0;
-        {
-            const uint32_t off = (uint32_t)((5ull * seg) & 63);
-            uint64_t v = cur.g0 >> off;
-            if (off > 54)  // this field and the next reach into the second word
-                v |= cur.g1 << (64 - off);
-            const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
-            if (seg < p.nseg) {
-                pos0 = (int)gap;
-                pend = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
-            }
+        // ---- the block's sign/mantissa bytes: asynchronous copy, waited for
+        // just before the merge
+        if (offs_ok) {
+            const uint32_t nbytes = align16(lo_off + (o1 - o0));
+            for (uint32_t off = 16 * lane; off < nbytes; off += 16 * 32)
+                cp_async16(sm_s + off, p.sm + g0 + off);
         }
-        const uint32_t w0 = bswap32(cur.s01.x), w1 = bswap32(cur.s01.y), w2 = bswap32(cur.s2);
+        asm volatile("cp.async.commit_group;" ::: "memory");
 
-        // ---- stage 1: count the codes starting in [pos0, pend)
+        // ---- locate: chain k's codes start in [pos0, pend) of its window
         bool bad = false;
-        uint32_t cnt = 0;
-        {
-            uint32_t h = w0, m = w1, l = w2;
-            shift_window(h, m, l, (uint32_t)pos0);
-            int pos = pos0;
-            const int bulk_end = pend - kIdxBits;
-            while (pos < bulk_end) {  // pos strictly increases: at most 95 steps
-                uint32_t e = cnt_tab[h >> (32 - kIdxBits)];
-                uint32_t c = e >> 4;
-                if (c == 0) {  // a code longer than 12 bits
-                    c = lut_decode(h, luts, cl, p.num_luts, &bad) >> 8;
-                    c = c ? c : 1u;
-                    e = 1;
-                }
-                cnt += e & 15u;
-                pos += (int)c;
-                shift_window(h, m, l, c);
+        int pos0[C], pend[C];
+        uint32_t w0[C], w1[C], w2[C], cnt[C];
+#pragma unroll
+        for (int k = 0; k < C; k++) {
+            const uint64_t seg = (uint64_t)b * T + lane + 32 * k;
+            const uint32_t off = (uint32_t)((5 * seg) & 31);
+            const uint64_t v = (((uint64_t)cur.g1[k] << 32) | cur.g0[k]) >> off;
+            const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
+            pos0[k] = 0;
+            pend[k] = 0;
+            if (seg < p.nseg) {
+                pos0[k] = (int)gap;
+                pend[k] = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
             }
-            const int r = pend - pos;
-            if (r > 0) {
-                // the last r <= 12 bits hold whole codes; mask the rest to zeros
-                const uint32_t idx = (h >> (32 - kIdxBits)) & ((0xFFFu << (kIdxBits - r)) & 0xFFFu);
-                const uint32_t e = cnt_tab[idx];
-                const uint32_t z = ztab[r];
-                cnt += (e & 15u) - (z & 0xFFu);
-                bad |= (e >> 4) - (z >> 8) != (uint32_t)r;
-            } else if (r < 0) {
-                bad = true;
+            w0[k] = bswap32(cur.s01[k].x);
+            w1[k] = bswap32(cur.s01[k].y);
+            w2[k] = bswap32(cur.s2[k]);
+            cnt[k] = 0;
+        }
+
+        // ---- stage 1: count the codes of each chain, chains interleaved
+        {
+            const uint32_t cnt_base = static_cast<uint32_t>(__cvta_generic_to_shared(cnt_tab));
+            uint32_t h[2], m[2], l[2], sum[2] = {0u, 0u}, nlong[2] = {0u, 0u}, blong[2] = {0u, 0u};
+            int pos[2], bend[2];
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const bool on = k < C;
+                h[k] = on ? w0[k < C ? k : 0] : 0u;
+                m[k] = on ? w1[k < C ? k : 0] : 0u;
+                l[k] = on ? w2[k < C ? k : 0] : 0u;
+                pos[k] = on ? pos0[k < C ? k : 0] : 0;
+                bend[k] = on ? pend[k < C ? k : 0] - kIdxBits : 0;
+                shift_window(h[k], m[k], l[k], (uint32_t)pos[k]);
+            }
+            for (;;) {  // each pass resolves >= 1 code or ends both chains
+                count_bulk2(h[0], m[0], l[0], sum[0], pos[0], h[1], m[1], l[1], sum[1], pos[1], bend[0], bend[1],
+                            cnt_base);
+                bool any_long = false;
+#pragma unroll
+                for (int k = 0; k < 2; k++) {
+                    if (pos[k] < bend[k] && (cnt_tab[h[k] >> (32 - kIdxBits)] >> 4) == 0) {
+                        // a code longer than 12 bits: the page's LUTs
+                        uint32_t c = lut_decode(h[k], luts, cl, p.num_luts, &bad) >> 8;
+                        c = c ? c : 1u;
+                        nlong[k] += 1;
+                        blong[k] += c;
+                        pos[k] += (int)c;
+                        shift_window(h[k], m[k], l[k], c);
+                        any_long = true;
+                    }
+                }
+                if (!any_long)
+                    break;
+            }
+#pragma unroll
+            for (int k = 0; k < C; k++) {
+                // table lookups added codes + 16 * bits
+                cnt[k] = sum[k] - 16u * ((uint32_t)(pos[k] - pos0[k]) - blong[k]) + nlong[k];
+                const int r = pend[k] - pos[k];
+                if (r > 0) {
+                    // the last r <= 12 bits hold whole codes; mask the rest
+                    const uint32_t idx = (h[k] >> (32 - kIdxBits)) & ((0xFFFu << (kIdxBits - r)) & 0xFFFu);
+                    const uint32_t e = cnt_tab[idx];
+                    const uint32_t z = ztab[r];
+                    cnt[k] += (e & 15u) - (z & 0xFFu);
+                    bad |= (e >> 4) - (z >> 8) != (uint32_t)r;
+                } else if (r < 0) {
+                    bad = true;
+                }
             }
         }
 
-        // ---- warp prefix sum of the counts
-        uint32_t incl = cnt;
+        // ---- warp prefix sum of the counts; both chains in one packed scan
+        // (a chain's block total is at most 64 * 32 < 2^16)
+        static_assert(C == 1 || C == 2, "one or two chains per lane");
+        uint32_t packed = 0;
+#pragma unroll
+        for (int k = 0; k < C; k++)
+            packed |= (cnt[k] & 0xFFFFu) << (16 * k);
+        uint32_t incl = packed;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
             if (lane >= d)
                 incl += y;
         }
-        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-        const uint32_t first = incl - cnt;
-        const bool block_bad = __any_sync(0xffffffffu, bad) || o1 < o0 || (uint64_t)o1 > p.n ||
-                               total != o1 - o0 || lo_off + total + 16u > p.cap;
+        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t first[C];
+        uint32_t total = 0;
+#pragma unroll
+        for (int k = 0; k < C; k++) {
+            first[k] = total + ((incl >> (16 * k)) & 0xFFFFu) - cnt[k];
+            total += (tot >> (16 * k)) & 0xFFFFu;
+        }
+#pragma unroll
+        for (int k = 0; k < C; k++)
+            bad |= cnt[k] > 64u;
+        const bool block_bad = __any_sync(0xffffffffu, bad) || !offs_ok || total != o1 - o0;
         if (block_bad) {
             if (lane == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            __syncwarp();
         } else {
             // ---- stage 2: decode again, place rotated exponents
             {
-                uint32_t h = w0, m = w1, l = w2;
-                shift_window(h, m, l, (uint32_t)pos0);
-                uint32_t q = lo_off + first;
-                const uint32_t qend = q + cnt;
-                while (q < qend) {  // q strictly increases
-                    uint32_t e = sym_tab[h >> (32 - kIdxBits)];
-                    uint32_t c = e >> 28, nsym = (e >> 24) & 3u;
-                    if (nsym == 0) {  // a code longer than 12 bits
-                        const uint32_t d = lut_decode(h, luts, cl, p.num_luts, &bad);
-                        e = ror8(d & 0xFFu);
-                        c = d >> 8;
-                        nsym = 1;
+                const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(sym_tab));
+                const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
+                uint32_t h[2], m[2], l[2], q[2], qend[2], qend1[2], qend2[2];
+#pragma unroll
+                for (int k = 0; k < 2; k++) {
+                    const bool on = k < C;
+                    const int kk = k < C ? k : 0;
+                    h[k] = w0[kk];
+                    m[k] = w1[kk];
+                    l[k] = w2[kk];
+                    shift_window(h[k], m[k], l[k], (uint32_t)pos0[kk]);
+                    // shared-memory byte addresses (never near 0, so q - 2 cannot wrap)
+                    q[k] = exp_base + lo_off + first[kk];
+                    qend[k] = on ? q[k] + cnt[kk] : q[k];
+                    qend1[k] = qend[k] - 1;  // a second exponent fits while q < qend - 1
+                    qend2[k] = qend[k] - 2;  // a third one while q < qend - 2
+                }
+                for (;;) {  // each pass places >= 1 exponent or ends both chains
+                    place_loop2(h[0], m[0], l[0], q[0], h[1], m[1], l[1], q[1], qend[0], qend1[0], qend2[0], qend[1],
+                                qend1[1], qend2[1], sym_base);
+                    bool any_long = false;
+#pragma unroll
+                    for (int k = 0; k < 2; k++) {
+                        if (q[k] < qend[k] && sym_tab[h[k] >> (32 - kIdxBits)] == 0) {
+                            const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
+                            exp_s[q[k] - exp_base] = (uint8_t)ror8(d & 0xFFu);
+                            q[k] += 1;
+                            shift_window(h[k], m[k], l[k], d >> 8);
+                            any_long = true;
+                        }
                     }
-                    exp_s[q] = (uint8_t)e;
-                    if (q + 1 < qend)
-                        exp_s[q + 1] = (uint8_t)(e >> 8);
-                    if (q + 2 < qend)
-                        exp_s[q + 2] = (uint8_t)(e >> 16);
-                    q += nsym;
-                    shift_window(h, m, l, c);
+                    if (!any_long)
+                        break;
                 }
             }
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
 
             // ---- merge with sign/mantissa, coalesced 16-byte stores
             const uint32_t hi = lo_off + total;
-            const uint64_t g0 = (uint64_t)o0 - lo_off;  // multiple of 16
-            const uint32_t nchunks = (hi + 15) / 16;
-            for (uint32_t c = lane; c < nchunks; c += 32) {
+            const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
+            for (uint32_t c = c_first + lane; c < c_end; c += 32) {
                 const uint32_t l0 = 16 * c;
-                if (l0 >= lo_off && l0 + 16 <= hi) {
-                    const uint4 s = __ldg(reinterpret_cast<const uint4 *>(p.sm + g0 + l0));
-                    const uint4 e = *reinterpret_cast<const uint4 *>(exp_s + l0);
-                    uint4 r0, r1;
-                    merge4(s.x, e.x, r0.x, r0.y);
-                    merge4(s.y, e.y, r0.z, r0.w);
-                    merge4(s.z, e.z, r1.x, r1.y);
-                    merge4(s.w, e.w, r1.z, r1.w);
-                    uint4 *d = reinterpret_cast<uint4 *>(p.dst + g0 + l0);
-                    d[0] = r0;
-                    d[1] = r1;
-                }
+                const uint4 s = *reinterpret_cast<const uint4 *>(sm_s + l0);
+                const uint4 e = *reinterpret_cast<const uint4 *>(exp_s + l0);
+                uint4 r0, r1;
+                merge4(s.x, e.x, r0.x, r0.y);
+                merge4(s.y, e.y, r0.z, r0.w);
+                merge4(s.z, e.z, r1.x, r1.y);
+                merge4(s.w, e.w, r1.z, r1.w);
+                uint4 *d = reinterpret_cast<uint4 *>(p.dst + g0 + l0);
+                d[0] = r0;
+                d[1] = r1;
             }
-            // partial first / last chunk: one element per lane
+            // partial first chunk (lanes 0..15) and partial last chunk
+            // (lanes 16..31): one element per lane
             {
-                const uint32_t chunk = lane < 16 ? 0u : nchunks - 1;
-                const uint32_t l = 16 * chunk + (lane & 15);
-                const bool partial = lo_off > 16 * chunk || 16 * chunk + 16 > hi;
-                if ((lane < 16 || nchunks > 1) && partial && l >= lo_off && l < hi)
-                    p.dst[g0 + l] = merge1(__ldg(p.sm + g0 + l), exp_s[l]);
+                const bool head = lane < 16;
+                const uint32_t l = head ? lane : 16 * c_end + (lane - 16);
+                const bool want = head ? (lo_off != 0 || hi < 16) : (c_end > 0 && (hi & 15u) != 0);
+                if (want && l >= lo_off && l < hi)
+                    p.dst[g0 + l] = merge1(sm_s[l], exp_s[l]);
             }
             __syncwarp();
         }
@@ -372,6 +588,45 @@ df11_status device_sms(int *sms)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+template <int C, int WARPS>
+df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem)
+{
+    auto kern = df11_decode_kernel<C, WARPS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    int sms = 0;
+    df11_status st = device_sms(&sms);
+    if (st != DF11_OK)
+        return st;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, smem) != cudaSuccess || per_sm < 1)
+        return DF11_ERR_CUDA;
+    uint64_t grid = (uint64_t)sms * (uint64_t)per_sm;
+    const uint64_t need = (prm.nblocks + WARPS - 1) / WARPS;
+    if (grid > need)
+        grid = need;
+    kern<<<(unsigned)grid, WARPS * 32, smem, stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+// 32 warps per CTA unless their buffers do not fit in shared memory (blocks of
+// very short codes hold up to 64 outputs per segment): then 16 or 8.
+template <int C>
+df11_status launch(const Params &prm, cudaStream_t stream)
+{
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return DF11_ERR_CUDA;
+    if (Smem::bytes(prm.cap, 32) <= (uint32_t)optin)
+        return launch_warps<C, 32>(prm, stream, Smem::bytes(prm.cap, 32));
+    if (Smem::bytes(prm.cap, 16) <= (uint32_t)optin)
+        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16));
+    if (Smem::bytes(prm.cap, 8) <= (uint32_t)optin)
+        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8));
+    return DF11_ERR_INVALID_ARG;
+}
+
 }  // namespace
 
 extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream)
@@ -380,7 +635,8 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
         return DF11_ERR_INVALID_ARG;
     if (a->n == 0)
         return DF11_OK;
-    if (a->threads_per_block != kBlockSegs)
+    const uint32_t T = a->threads_per_block;
+    if (T != 32 && T != 64)
         return DF11_ERR_INVALID_ARG;
     if (!dst || !a->encoded_exponent || !a->packed_sign_mantissa || !a->gaps || !a->block_offset || !a->luts ||
         !a->code_lengths)
@@ -391,19 +647,18 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     if (a->num_luts < 1 || a->num_luts > DF11_MAX_LUTS || a->n >= (1ull << 32))
         return DF11_ERR_INVALID_ARG;
     const uint64_t nseg = (a->total_bits + 63) / 64;
-    if (nseg != a->num_segments || (nseg + kBlockSegs - 1) / kBlockSegs != a->num_blocks || a->num_blocks == 0)
+    if (nseg != a->num_segments || (nseg + T - 1) / T != a->num_blocks || a->num_blocks == 0)
         return DF11_ERR_INVALID_ARG;
     // every load stays inside its array
-    if (a->encoded_exponent_bytes < (uint64_t)a->num_blocks * kBlockSegs * 8 + 16 ||
+    if (a->encoded_exponent_bytes < (uint64_t)a->num_blocks * T * 8 + 16 ||
         a->packed_sign_mantissa_bytes < ((a->n + 15) / 16) * 16 ||
-        a->gaps_words < (5ull * a->num_blocks * kBlockSegs + 63) / 64 + 2 ||
-        a->max_block_elems > 64u * kBlockSegs)
+        a->gaps_words < (5ull * a->num_blocks * T + 63) / 64 + 2 || a->max_block_elems > 64u * T)
         return DF11_ERR_INVALID_ARG;
 
     Params prm;
     prm.stream = a->encoded_exponent;
     prm.sm = a->packed_sign_mantissa;
-    prm.gaps = a->gaps;
+    prm.gaps = reinterpret_cast<const uint32_t *>(a->gaps);
     prm.offs = a->block_offset;
     prm.luts = a->luts;
     prm.cl = a->code_lengths;
@@ -414,26 +669,13 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     prm.nseg = nseg;
     prm.nblocks = a->num_blocks;
     prm.num_luts = a->num_luts;
+    // at least 8 KB of buffers even with 8 warps: they hold a 4096-entry
+    // scratch table during set-up
     prm.cap = align16(a->max_block_elems + 32);
-
-    const uint32_t smem = Smem::bytes(prm.cap);
-    if (cudaFuncSetAttribute(df11_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return DF11_ERR_CUDA;
-    int sms = 0;
-    df11_status st = device_sms(&sms);
-    if (st != DF11_OK)
-        return st;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, df11_decode_kernel, kThreads, smem) != cudaSuccess ||
-        per_sm < 1)
-        return DF11_ERR_CUDA;
-    uint64_t grid = (uint64_t)sms * (uint64_t)per_sm;
-    const uint64_t need = (a->num_blocks + kWarps - 1) / kWarps;
-    if (grid > need)
-        grid = need;
-    df11_decode_kernel<<<(unsigned)grid, kThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+    if (prm.cap * 2 * 8 < kIdxEntries * 2)
+        prm.cap = kIdxEntries / 8;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
 }
 
 extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arrays *d, uint16_t *dst_dev,

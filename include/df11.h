@@ -58,7 +58,7 @@ extern "C" {
 #define DF11_MAX_CODE_LEN 32     /* longest code: Gaps are 5 bits wide */
 #define DF11_SEGMENT_BYTES 8     /* encoded bytes per GPU thread */
 #define DF11_MAX_LUTS 17         /* root + 16 children (pointers 240..255) */
-#define DF11_DEFAULT_THREADS 32  /* default segments (threads) per block */
+#define DF11_DEFAULT_THREADS 64  /* default segments (threads) per block */
 
 typedef enum df11_status {
     DF11_OK = 0,
@@ -84,7 +84,7 @@ typedef struct df11_arrays {
     uint64_t total_bits;        /* valid bits of encoded_exponent */
     uint64_t num_segments;      /* ceil(total_bits / 64) */
     uint32_t threads_per_block; /* T: segments per block (multiple of 32, 32..1024;
-                                   the decoder takes T = 32, one warp) */
+                                   the decoder takes T = 32 or 64: one warp) */
     uint32_t num_blocks;        /* ceil(num_segments / T) */
     uint32_t num_luts;          /* k, 1 .. 17 */
     uint32_t max_code_len;      /* longest code length, <= 32 */
@@ -124,8 +124,8 @@ typedef struct df11_info {
  *             stream.  One Huffman code covers all matrices (a transformer
  *             block is compressed as one stream, "Dekompresi per transformer
  *             block").  NULL allowed when counts[i] == 0.
- *   threads_per_block  T, a multiple of 32 in [32, 1024] (0 = default 32).
- *             df11_decompress requires T = 32 (a block is one warp).
+ *   threads_per_block  T, a multiple of 32 in [32, 1024] (0 = default 64).
+ *             df11_decompress requires T = 32 or 64 (a block is one warp).
  *   out       receives a new handle, owned by the caller (df11_free).
  * Inputs are only read.  Errors: DF11_ERR_INVALID_ARG, _UNSUPPORTED_EXPONENT,
  * _TOO_LARGE (total n >= 2^32), _TOO_MANY_LUTS, _NO_MEMORY; *out is NULL then.

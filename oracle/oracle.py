@@ -225,7 +225,7 @@ def decode_range(stream, stream_bits: int, start_bit: int, end_bit: int, lens, c
     return out[:cnt].copy()
 
 
-def build_format(w: np.ndarray, threads_per_block: int = 32, max_len: int = MAX_CODE_LEN) -> dict:
+def build_format(w: np.ndarray, threads_per_block: int = 64, max_len: int = MAX_CODE_LEN) -> dict:
     """All DF11 arrays for one stream of BF16 bits, built step by step."""
     exps, sm = split(w)
     hist = histogram(exps)

@@ -26,7 +26,7 @@ def torch_cuda():
     return torch
 
 
-def gpu_decode(mats, T=32, dev_fmt=None):
+def gpu_decode(mats, T=64, dev_fmt=None):
     torch = torch_cuda()
     fmt = df11.build_format(mats, T)
     dev = dev_fmt or df11.DeviceFormat(fmt, "cuda")
@@ -38,7 +38,7 @@ def gpu_decode(mats, T=32, dev_fmt=None):
     return got, st, fmt
 
 
-def check_against_oracle(oracle_mod, w, T=32):
+def check_against_oracle(oracle_mod, w, T=64):
     got, st, _ = gpu_decode(w, T)
     assert st == 0
     ref = oracle_mod.decode_format(oracle_mod.build_format(w, T))
@@ -52,10 +52,17 @@ def test_sizes(oracle_mod, n):
     check_against_oracle(oracle_mod, inputs.gaussian(n, [21, n]))
 
 
-@pytest.mark.parametrize("T", [64, 128, 256])
+@pytest.mark.parametrize("T", [32, 64])
+@pytest.mark.parametrize("n", [1, 65, 32 * 64 + 1, 300_007])
+def test_block_sizes(oracle_mod, T, n):
+    # one warp decodes a block of T segments: T = 64 runs two chains per lane
+    check_against_oracle(oracle_mod, inputs.gaussian(n, [31, T, n]), T)
+
+
+@pytest.mark.parametrize("T", [96, 128, 256])
 def test_other_block_sizes_are_rejected(T):
-    # the decoder's thread block is one warp: formats built with T != 32 are
-    # refused on the host, nothing is launched
+    # the decoder's thread block is one warp of one or two chains per lane:
+    # other block sizes are refused on the host, nothing is launched
     torch = torch_cuda()
     fmt = df11.build_format(inputs.gaussian(10_000, [22, T]), T)
     dev = df11.DeviceFormat(fmt, "cuda")
@@ -65,9 +72,10 @@ def test_other_block_sizes_are_rejected(T):
     assert e.value.status == 1
 
 
-def test_many_blocks_per_warp(oracle_mod):
+@pytest.mark.parametrize("T", [32, 64])
+def test_many_blocks_per_warp(oracle_mod, T):
     # more blocks than resident warps: every warp walks several blocks
-    check_against_oracle(oracle_mod, inputs.gaussian(6_000_011, [22, 1]))
+    check_against_oracle(oracle_mod, inputs.gaussian(6_000_011, [22, 1]), T)
 
 
 def test_empty_stream():
@@ -107,15 +115,16 @@ def test_length_limited_code(oracle_mod):
     assert np.array_equal(got, w)
 
 
-def test_stress_small(oracle_mod):
-    check_against_oracle(oracle_mod, inputs.stress(1 << 21, key=(3, 7, 7)))
+@pytest.mark.parametrize("T", [32, 64])
+def test_stress_small(oracle_mod, T):
+    check_against_oracle(oracle_mod, inputs.stress(1 << 21, key=(3, 7, 7)), T)
 
 
 def test_multi_matrix(oracle_mod):
     mats = [inputs.gaussian(n, [23, n]) for n in (4096 * 3 + 5, 17, 0, 70_000)]
     got, st, _ = gpu_decode(mats)
     assert st == 0
-    ref = oracle_mod.decode_format(oracle_mod.build_format(np.concatenate(mats), 32))
+    ref = oracle_mod.decode_format(oracle_mod.build_format(np.concatenate(mats), 64))
     assert np.array_equal(got, ref)
 
 
@@ -217,12 +226,12 @@ def _full_check(oracle_mod, workload, block_id=0, sample_blocks=200):
     torch = torch_cuda()
     mats = [m for _, _, m in inputs.workload_arrays(workload, block_id)]
     w = np.concatenate(mats) if len(mats) > 1 else mats[0]
-    got, st, fmt = gpu_decode(mats, 32)
+    got, st, fmt = gpu_decode(mats, 64)
     assert st == 0
     assert np.array_equal(got, w)
     # oracle: its own format from the same input, then its tree walk over a
     # sample of blocks' bit ranges
-    ref = oracle_mod.build_format(w, 32)
+    ref = oracle_mod.build_format(w, 64)
     offs = ref["block_offset"].astype(np.int64)
     nb = offs.size - 1
     rng = np.random.default_rng(workload)
@@ -230,8 +239,8 @@ def _full_check(oracle_mod, workload, block_id=0, sample_blocks=200):
     gaps = ref["gaps"]
     nseg = gaps.size
     for b in blocks:
-        s0 = b * 32
-        s1 = min((b + 1) * 32, nseg)
+        s0 = b * 64
+        s1 = min((b + 1) * 64, nseg)
         a = 64 * s0 + int(gaps[s0])
         e = 64 * s1 + int(gaps[s1]) if s1 < nseg else ref["total_bits"]
         exps = oracle_mod.decode_range(ref["encoded_exponent"], ref["total_bits"], a, e,

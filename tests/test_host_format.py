@@ -44,7 +44,7 @@ def compare(fmt, ref):
 @pytest.mark.parametrize("n", [0, 1, 2, 7, 63, 64, 65, 1000, 32 * 25 - 1, 32 * 25, 32 * 25 + 1, 256 * 25 + 1, 100_003])
 def test_gaussian_sizes(oracle_mod, n):
     w = inputs.gaussian(n, [11, n])
-    compare(df11.build_format(w), oracle_mod.build_format(w, 32))
+    compare(df11.build_format(w), oracle_mod.build_format(w, 64))
 
 
 @pytest.mark.parametrize("T", [32, 64, 128, 256, 512, 1024])
@@ -56,7 +56,7 @@ def test_threads_per_block(oracle_mod, T):
 def test_stress_distribution(oracle_mod):
     w = inputs.stress(1 << 20, key=(3, 9, 9))
     fmt = df11.build_format(w)
-    compare(fmt, oracle_mod.build_format(w, 32))
+    compare(fmt, oracle_mod.build_format(w, 64))
     info = fmt.info()
     assert info["max_code_len"] >= 18 and info["num_luts"] >= 3
 
@@ -65,21 +65,21 @@ def test_chunk_boundaries_many_threads(oracle_mod):
     # > 4 Mi elements: the encoder splits work into several chunks whose
     # boundary bytes are shared
     w = inputs.gaussian((1 << 22) * 2 + 12345, [13, 0])
-    compare(df11.build_format(w), oracle_mod.build_format(w, 32))
+    compare(df11.build_format(w), oracle_mod.build_format(w, 64))
 
 
 def test_every_bf16_pattern(oracle_mod):
     allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     ok = allbits[((allbits >> 7) & 0xFF) < 240]
     w = np.random.default_rng(3).permutation(ok)
-    compare(df11.build_format(w), oracle_mod.build_format(w, 32))
+    compare(df11.build_format(w), oracle_mod.build_format(w, 64))
 
 
 def test_single_symbol(oracle_mod):
     w = np.full(5000, 0x3F80, np.uint16)
     w[::7] = 0xBF80  # sign differs, exponent the same
     fmt = df11.build_format(w)
-    compare(fmt, oracle_mod.build_format(w, 32))
+    compare(fmt, oracle_mod.build_format(w, 64))
     assert fmt.info()["max_code_len"] == 1
 
 
@@ -91,7 +91,7 @@ def test_length_limited_code(oracle_mod):
     exps = np.random.default_rng(5).permutation(exps)
     w = (exps << 7).astype(np.uint16)
     fmt = df11.build_format(w)
-    ref = oracle_mod.build_format(w, 32)
+    ref = oracle_mod.build_format(w, 64)
     compare(fmt, ref)
     assert fmt.info()["max_code_len"] == 32
 
@@ -99,7 +99,7 @@ def test_length_limited_code(oracle_mod):
 def test_multi_matrix_equals_concatenation(oracle_mod):
     mats = [inputs.gaussian(n, [14, n]) for n in (1000, 0, 4097, 33)]
     fmt = df11.build_format(mats)
-    compare(fmt, oracle_mod.build_format(np.concatenate(mats), 32))
+    compare(fmt, oracle_mod.build_format(np.concatenate(mats), 64))
 
 
 def test_info_statistics(oracle_mod):
