@@ -44,7 +44,10 @@
 //   * the two decode loops are hand-written PTX: both chains of a lane step
 //     in one predicated loop, so the warp runs max(chain A, chain B) passes;
 //     stage 1 adds raw table entries (codes + 16 * bits) and recovers the
-//     count from the bits advanced;
+//     count from the bits advanced; right shifts by constants that are off
+//     the loop's dependency chain are written as mul.hi (x >> k ==
+//     mul.hi(x, 2^(32-k))), which runs on the FMA pipe and leaves the integer
+//     ALU pipe -- the busier one here -- to the funnel shifts and compares;
 //   * the next block's stream words, Gaps words and offsets are loaded into
 //     registers while the current block is decoded; the current block's
 //     sign/mantissa bytes arrive in shared memory by asynchronous copies
@@ -238,26 +241,26 @@ __device__ __forceinline__ void place_loop2(uint32_t &hA, uint32_t &mA, uint32_t
         "or.pred pl, pl, pz;\n\t"
         "@pl bra PL_END;\n\t"
         "@pa shr.u32 ca, ea, 24;\n\t"
-        "@pa shr.u32 na, ea, 29;\n\t"
+        "@pa mul.hi.u32 na, ea, 8;\n\t"
         "@pa st.shared.u8 [%3], ea;\n\t"
         "setp.lt.and.u32 p1, %3, %9, pa;\n\t"
         "setp.lt.and.u32 p2, %3, %10, pa;\n\t"
-        "@p1 shr.u32 t, ea, 8;\n\t"
+        "@p1 mul.hi.u32 t, ea, 16777216;\n\t"
         "@p1 st.shared.u8 [%3+1], t;\n\t"
-        "@p2 shr.u32 t, ea, 16;\n\t"
+        "@p2 mul.hi.u32 t, ea, 65536;\n\t"
         "@p2 st.shared.u8 [%3+2], t;\n\t"
         "@pa add.u32 %3, %3, na;\n\t"
         "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
         "@pb shr.u32 cb, eb, 24;\n\t"
-        "@pb shr.u32 nb, eb, 29;\n\t"
+        "@pb mul.hi.u32 nb, eb, 8;\n\t"
         "@pb st.shared.u8 [%7], eb;\n\t"
         "setp.lt.and.u32 p1, %7, %12, pb;\n\t"
         "setp.lt.and.u32 p2, %7, %13, pb;\n\t"
-        "@p1 shr.u32 t, eb, 8;\n\t"
+        "@p1 mul.hi.u32 t, eb, 16777216;\n\t"
         "@p1 st.shared.u8 [%7+1], t;\n\t"
-        "@p2 shr.u32 t, eb, 16;\n\t"
+        "@p2 mul.hi.u32 t, eb, 65536;\n\t"
         "@p2 st.shared.u8 [%7+2], t;\n\t"
         "@pb add.u32 %7, %7, nb;\n\t"
         "@pb shf.l.wrap.b32 %4, %5, %4, cb;\n\t"
@@ -316,6 +319,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     uint8_t *exp_s = smem + Smem::bufs + warp * 2 * p.cap;
     uint8_t *sm_s = exp_s + p.cap;
 
+    // the first block's registers load while the tables are built
+    const uint32_t stride = gridDim.x * kWarps;
+    uint32_t b = blockIdx.x * kWarps + warp;
+    BlockRegs<C> cur, nxt;
+    if (b < p.nblocks)
+        load_block<C>(p, b, lane, cur);
+
     // ---- once per CTA: the page's LUTs and CodeLengths, derived tables
     const uint32_t lut_bytes = p.num_luts * 256u;
     for (uint32_t i = tid; i < lut_bytes; i += kThreads)
@@ -323,37 +333,60 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     for (uint32_t i = tid; i < 256; i += kThreads)
         cl[i] = p.cl[i];
     __syncthreads();
-    // first code of every 12-bit window (zero filled): symbol | length << 8,
-    // length 0 when the code is longer than 12 bits.  Kept in the per-warp
-    // buffers, which are free until the blocks start.
+    // Derived tables.  first_code[i]: the first code of the 12-bit window i
+    // (bits past 12 taken as zeros): symbol | length << 8, or 0 when that code
+    // is longer than 12 bits.  A code found in a zero-filled window is genuine
+    // when it ends inside the window (prefix property).  Scratch lives in the
+    // per-warp buffers, which are free until the blocks start.
     uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
+    uint16_t *greedy = first_code + kIdxEntries;  // levels r = 0..11, 2^r entries each
     for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
         bool bad = false;
         const uint32_t e = lut_decode(i << (32 - kIdxBits), luts, cl, p.num_luts, &bad);
         const uint32_t len = e >> 8;
         first_code[i] = (!bad && len >= 1 && len <= kIdxBits) ? (uint16_t)e : (uint16_t)0;
     }
+    if (tid == 0)
+        greedy[0] = 0;
     __syncthreads();
-    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
-        uint32_t pos = 0, ncodes = 0, syms = 0, sym_bits = 0, sym_n = 0;
-        for (int it = 0; it < kIdxBits; it++) {
-            // the window after `pos` bits; its tail is zero filled, and a code
-            // found there is genuine only if it ends inside the 12 bits
-            const uint32_t e = first_code[(i << pos) & (kIdxEntries - 1)];
-            const uint32_t len = e >> 8;
-            if (len == 0 || pos + len > kIdxBits)
-                break;
-            if (ncodes < 3) {
-                syms |= ror8(e & 0xFFu) << (8 * ncodes);
-                sym_bits = pos + len;
-                sym_n = ncodes + 1;
+    // Count table by levels: G_r(v) = whole codes (and their bits) read
+    // greedily from the r-bit value v; G_r(v) = 1 + G_{r-l}(v without its
+    // first code of length l), or nothing when that code needs more than r
+    // bits.  G_12 is the count table (codes | bits << 4).
+    for (uint32_t r = 1; r <= kIdxBits; r++) {
+        const uint32_t nv = 1u << r;
+        for (uint32_t v = tid; v < nv; v += kThreads) {
+            const uint32_t fc = first_code[(v << (kIdxBits - r)) & (kIdxEntries - 1)];
+            const uint32_t len = fc >> 8;
+            uint32_t g = 0;  // codes | bits << 8
+            if (len != 0 && len <= r) {
+                const uint32_t rest = r - len;
+                const uint32_t gr = greedy[(1u << rest) - 1 + (v & ((1u << rest) - 1))];
+                g = (1u + (gr & 0xFFu)) | ((len + (gr >> 8)) << 8);
             }
-            ncodes++;
-            pos += len;
+            if (r < kIdxBits)
+                greedy[nv - 1 + v] = (uint16_t)g;
+            else
+                cnt_tab[v] = (uint8_t)((g & 0xFFu) | ((g >> 8) << 4));
         }
-        cnt_tab[i] = (uint8_t)(ncodes | (pos << 4));
+        __syncthreads();
+    }
+    // Symbol table: the first three codes of each window, by three dependent
+    // first_code lookups.
+    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
+        uint32_t syms = 0, bits = 0, n = 0;
+#pragma unroll
+        for (int j = 0; j < 3; j++) {
+            const uint32_t fc = first_code[(i << bits) & (kIdxEntries - 1)];
+            const uint32_t len = fc >> 8;
+            if (len != 0 && len + bits <= kIdxBits && n == (uint32_t)j) {
+                syms |= ror8(fc & 0xFFu) << (8 * j);
+                bits += len;
+                n++;
+            }
+        }
         // exponents in bytes 0..2, total length in bits 24..28, count in 29..30
-        sym_tab[i] = syms | (sym_bits << 24) | (sym_n << 29);
+        sym_tab[i] = syms | (bits << 24) | (n << 29);
     }
     if (tid <= kIdxBits) {
         // codes formed by the zero bits r..11 after a code boundary: the
@@ -366,11 +399,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     __syncthreads();
 
     // ---- each warp walks its own blocks; no block-wide barrier from here on
-    const uint32_t stride = gridDim.x * kWarps;
-    uint32_t b = blockIdx.x * kWarps + warp;
-    BlockRegs<C> cur, nxt;
-    if (b < p.nblocks)
-        load_block<C>(p, b, lane, cur);
     for (; b < p.nblocks; b += stride) {
         if (b + stride < p.nblocks)
             load_block<C>(p, b + stride, lane, nxt);
@@ -567,41 +595,53 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 }
 
 // ------------------------------------------------------------- host side
+// Per-device launch facts, looked up once: SM count and the opt-in shared
+// memory limit; per kernel instantiation, the largest dynamic shared memory
+// size already granted.
+struct DeviceFacts {
+    int sms = 0;
+    int smem_optin = 0;
+    uint32_t granted[2][3] = {};  // [C - 1][warps 32 / 16 / 8]
+};
 std::mutex g_mu;
-int g_sms[64];
+DeviceFacts g_dev[64];
 
-df11_status device_sms(int *sms)
+df11_status device_facts(DeviceFacts **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return DF11_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_sms[dev]) {
-        int v = 0;
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    DeviceFacts &f = g_dev[dev];
+    if (!f.sms) {
+        int sms = 0, optin = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return DF11_ERR_CUDA;
-        g_sms[dev] = v;
+        f.smem_optin = optin;
+        f.sms = sms;
     }
-    *sms = g_sms[dev];
+    *out = &f;
     return DF11_OK;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 template <int C, int WARPS>
-df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem)
+df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, DeviceFacts *f, uint32_t &granted)
 {
     auto kern = df11_decode_kernel<C, WARPS>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return DF11_ERR_CUDA;
-    int sms = 0;
-    df11_status st = device_sms(&sms);
-    if (st != DF11_OK)
-        return st;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WARPS * 32, smem) != cudaSuccess || per_sm < 1)
-        return DF11_ERR_CUDA;
-    uint64_t grid = (uint64_t)sms * (uint64_t)per_sm;
+    if (smem > granted) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (smem > granted) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return DF11_ERR_CUDA;
+            granted = smem;
+        }
+    }
+    // one persistent CTA per SM: __launch_bounds__(WARPS * 32, 1) and the
+    // shared-memory footprint allow no second one
+    uint64_t grid = (uint64_t)f->sms;
     const uint64_t need = (prm.nblocks + WARPS - 1) / WARPS;
     if (grid > need)
         grid = need;
@@ -614,16 +654,17 @@ df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem)
 template <int C>
 df11_status launch(const Params &prm, cudaStream_t stream)
 {
-    int dev = 0, optin = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-        return DF11_ERR_CUDA;
-    if (Smem::bytes(prm.cap, 32) <= (uint32_t)optin)
-        return launch_warps<C, 32>(prm, stream, Smem::bytes(prm.cap, 32));
-    if (Smem::bytes(prm.cap, 16) <= (uint32_t)optin)
-        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16));
-    if (Smem::bytes(prm.cap, 8) <= (uint32_t)optin)
-        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8));
+    DeviceFacts *f = nullptr;
+    df11_status st = device_facts(&f);
+    if (st != DF11_OK)
+        return st;
+    const uint32_t optin = (uint32_t)f->smem_optin;
+    if (Smem::bytes(prm.cap, 32) <= optin)
+        return launch_warps<C, 32>(prm, stream, Smem::bytes(prm.cap, 32), f, f->granted[C - 1][0]);
+    if (Smem::bytes(prm.cap, 16) <= optin)
+        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[C - 1][1]);
+    if (Smem::bytes(prm.cap, 8) <= optin)
+        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[C - 1][2]);
     return DF11_ERR_INVALID_ARG;
 }
 
@@ -669,11 +710,11 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     prm.nseg = nseg;
     prm.nblocks = a->num_blocks;
     prm.num_luts = a->num_luts;
-    // at least 8 KB of buffers even with 8 warps: they hold a 4096-entry
-    // scratch table during set-up
+    // at least 16 KB of buffers even with 8 warps: they hold set-up scratch
+    // (two 4096-entry uint16 tables)
     prm.cap = align16(a->max_block_elems + 32);
-    if (prm.cap * 2 * 8 < kIdxEntries * 2)
-        prm.cap = kIdxEntries / 8;
+    if (prm.cap < 1024)
+        prm.cap = 1024;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
 }
