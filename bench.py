@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAME = "df11_decode_kernel"
 KERNEL_SOURCE = os.path.join(ROOT, "huffman_decode_03_b200", "csrc", "df11_decode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILES = os.path.join(ROOT, "profiles")
 
 
 # ----------------------------------------------------------------- helpers
@@ -113,19 +113,27 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(workload: int, n_elems: int):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken of
-    the current kernel source; scaled by elements when captured smaller."""
+    """DRAM bytes per launch from a committed ncu capture (profiles/traffic_*.txt),
+    if it was taken of the current kernel source; scaled by elements when the
+    capture covered a different number of outputs."""
     try:
-        with open(TRAFFIC_FILE) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+        names = sorted(os.listdir(PROFILES))
+    except OSError:
         return None
-    if d.get("kernel_source_sha256_16") != kernel_source_hash():
-        return None
-    rec = d.get("captures", {}).get(str(workload))
-    if not rec:
-        return None
-    return float(rec["dram_bytes"]) * n_elems / float(rec["elements"])
+    for name in names:
+        if not (name.startswith("traffic_") and name.endswith(".txt")):
+            continue
+        rec = {}
+        with open(os.path.join(PROFILES, name)) as f:
+            for line in f:
+                if line.strip() and not line.startswith("#") and ":" in line:
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.strip()
+        if rec.get("kernel_source_sha256_16") != kernel_source_hash() or rec.get("workload") != str(workload):
+            continue
+        dram = float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
+        return dram * n_elems / float(rec["elements"])
+    return None
 
 
 def stream_algorithmic_bytes(s: dict) -> int:
