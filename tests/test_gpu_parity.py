@@ -269,3 +269,35 @@ def test_workload_stress(oracle_mod):
 @pytest.mark.slow
 def test_workload_llama3_70b_block(oracle_mod):
     _full_check(oracle_mod, 4, sample_blocks=100)
+
+
+@pytest.mark.slow
+def test_workload_stream_of_32_blocks():
+    # 32 independent Llama-3-8B blocks, each with its own code, decoded back to
+    # back into ONE reused BF16 buffer (the streaming launch configuration);
+    # every block is checked against its original bits before the next
+    # overwrites the buffer ("Dekompresi per transformer block").
+    torch = torch_cuda()
+    from concurrent.futures import ThreadPoolExecutor
+
+    n = inputs.block_elements(5)
+    out = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def prepare(b):
+        mats = [m for _, _, m in inputs.workload_arrays(5, b)]
+        return np.concatenate(mats), df11.build_format(mats)
+
+    with ThreadPoolExecutor(1) as ex:
+        nxt = ex.submit(prepare, 0)
+        for b in range(32):
+            w, fmt = nxt.result()
+            if b + 1 < 32:
+                nxt = ex.submit(prepare, b + 1)
+            dev = df11.DeviceFormat(fmt, "cuda")
+            fmt.free()
+            df11.decompress(dev, out, status)
+            ref = torch.from_numpy(w.view(np.int16)).to("cuda")
+            assert torch.equal(out.view(torch.int16), ref), f"block {b}"
+            del dev, ref
+    assert df11.read_status(status) == 0
