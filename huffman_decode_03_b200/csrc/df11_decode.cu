@@ -5,53 +5,50 @@
 //        instead of a bit-by-bit tree walk; the tree is cut into height-8
 //        subtrees stored as 256-entry LUTs whose values 240..255 are pointers;
 //   "Kernel GPU 2 tahap dan metadata bantu" -- one thread per 8-byte segment
-//        of EncodedExponent, starting at the segment's Gap; stage 1 counts the
-//        codes of each segment, a prefix sum over the thread block plus the
-//        block's stored output position gives each thread its first output
-//        index, stage 2 decodes again and places the exponents in an on-chip
-//        write buffer, and the block's outputs leave in one coalesced write;
+//        of EncodedExponent, starting at the segment's Gap; the number of codes
+//        of each thread, prefix-summed over the thread block and added to the
+//        block's stored output position, gives each thread its first output
+//        index; exponents are placed in an on-chip write buffer and the block's
+//        outputs leave in one coalesced write;
 //   "Format DFloat11" -- sign and mantissa come verbatim from
 //        PackedSignMantissa.
 //
 // B200 design (what differs from the page's kernel):
-//   * the format's thread block is one warp (T = 32 or 64 segments; with 64
-//     each lane decodes two segments as two independent chains, which keeps
+//   * the format's thread block is one warp (T = 64 segments by default; lane
+//     l decodes segments l and l + 32 as two independent chains, which keeps
 //     two lookups in flight per thread): a block's prefix sum is five warp
-//     shuffles and its write buffer is private to the warp, so warps never
-//     wait for one another -- no block-wide barrier after set-up.  One
-//     persistent CTA of 32 warps runs per SM and every warp walks its own
-//     sequence of blocks;
-//   * the CTA stages the page's LUTs and CodeLengths once and derives two
-//     wider tables from them in shared memory, shared by its 32 warps (via a
-//     scratch table of the first code of every 12-bit window):
-//       - a count table over the next 12 bits: how many whole codes they
-//         hold and how many bits those codes use (stage 1 advances about 10
-//         bits per lookup);
-//       - a symbol table over the next 12 bits: up to 3 whole codes, their
-//         total length and their exponents (stage 2 places ~3 exponents per
-//         lookup).  Exponents are stored rotated right by one bit, which
-//         turns the final BF16 merge into two bit-selects and two byte
-//         permutes per 4 elements.
-//     Codes longer than 12 bits fall back to the page's pointer-chasing LUTs;
-//   * stage 1 stops exactly at the thread's last code: the next segment's
-//     Gap gives the bit where the next thread starts; the final lookup masks
-//     the bits past that point to zeros, and the codes the zeros form (the
-//     all-zero code is the canonical first code) are subtracted;
-//   * stage 2 runs until the thread has placed as many exponents as stage 1
-//     counted;
-//   * each thread's 64 + 32 bits live in a three-register shift window: the
+//     shuffles and its buffers are private to the warp, so warps never wait
+//     for one another -- no block-wide barrier after set-up.  One persistent
+//     CTA per SM; every warp walks its own sequence of blocks;
+//   * decode once, not twice: the page counts the codes of every segment in
+//     a first pass and decodes them again in a second.  Here every chain
+//     decodes once into a private staging slot in shared memory (slots 68
+//     bytes apart, so the 32 lanes of a warp store to distinct banks), its
+//     code count falls out of that pass, and after the warp prefix sum each
+//     chain copies its slot into the block's write buffer a 32-bit word at a
+//     time;
+//   * the CTA stages the page's LUTs and CodeLengths once and derives from
+//     them a symbol table over the next 12 bits of the stream: up to 3 whole
+//     codes, their total length and their exponents (~3 exponents per shared
+//     memory lookup).  Exponents are stored rotated right by one bit, which
+//     turns the final BF16 merge into two bit-selects and two byte permutes
+//     per 4 elements.  Codes longer than 12 bits fall back to the page's
+//     pointer-chasing LUTs;
+//   * a chain stops exactly at its last code: the next segment's Gap gives the
+//     bit where the next chain starts; the lookups of the last <= 12 bits
+//     mask the bits past that point to zeros, and the codes the zeros form
+//     (the all-zero code is the canonical first code) are discounted;
+//   * each chain's 64 + 32 bits live in a three-register shift window: the
 //     table index is the top 12 bits, a step is three funnel shifts;
-//   * the two decode loops are hand-written PTX: both chains of a lane step
-//     in one predicated loop, so the warp runs max(chain A, chain B) passes;
-//     stage 1 adds raw table entries (codes + 16 * bits) and recovers the
-//     count from the bits advanced; right shifts by constants that are off
-//     the loop's dependency chain are written as mul.hi (x >> k ==
-//     mul.hi(x, 2^(32-k))), which runs on the FMA pipe and leaves the integer
-//     ALU pipe -- the busier one here -- to the funnel shifts and compares;
+//   * the decode loop is hand-written PTX: both chains of a lane step in one
+//     predicated loop; right shifts by constants that are off the loop's
+//     dependency chain are written as mul.hi (x >> k == mul.hi(x, 2^(32-k))),
+//     which runs on the FMA pipe and leaves the integer ALU pipe to the
+//     funnel shifts and compares;
 //   * the next block's stream words, Gaps words and offsets are loaded into
 //     registers while the current block is decoded; the current block's
 //     sign/mantissa bytes arrive in shared memory by asynchronous copies
-//     (cp.async) during the two decode stages.
+//     (cp.async) during decoding.
 // Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
 
@@ -62,11 +59,15 @@
 
 namespace {
 
-constexpr int kIdxBits = 12;  // index width of the derived tables
+constexpr int kIdxBits = 12;  // index width of the derived table
 constexpr int kIdxEntries = 1 << kIdxBits;
 constexpr int kLutBytes = DF11_MAX_LUTS * 256;
 constexpr uint32_t kPointerBase = 240;
-constexpr int kMaxWarps = 32;  // warps per CTA (fewer when a block's buffers are large)
+constexpr uint32_t kSlotStride = 68;  // bytes per lane's staging slot (64 codes + 2 spill + 2)
+// per warp: two chains x 32 lanes, plus 32 bytes so that a chain of
+// inconsistent data (up to 95 one-bit codes + 2 spill bytes) stays inside the
+// warp's own slots; such a block is reported and writes nothing
+constexpr uint32_t kSlotBytes = 2 * 32 * kSlotStride + 32;
 
 struct Params {
     const uint8_t *stream;
@@ -87,19 +88,19 @@ struct Params {
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
-// Shared memory: tables at fixed offsets (lookups need no base register),
-// then two buffers per warp: placed exponents and the block's
-// sign/mantissa bytes.
+// Shared memory: tables at fixed offsets, then per warp: the exponent write
+// buffer, the block's sign/mantissa bytes and the chains' staging slots.
 struct Smem {
     static constexpr uint32_t sym = 0;                       // uint32[4096]
-    static constexpr uint32_t cnt = sym + kIdxEntries * 4;   // uint8[4096]
-    static constexpr uint32_t luts = cnt + kIdxEntries;      // 17 * 256
+    static constexpr uint32_t luts = sym + kIdxEntries * 4;  // 17 * 256
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
-    static constexpr uint32_t ztab = cl + 256;               // uint16[16]
-    static constexpr uint32_t bufs = ztab + 32;
-    static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * 2 * cap; }
+    static constexpr uint32_t zq = cl + 256;                 // uint8[16]
+    static constexpr uint32_t bufs = zq + 16;
+    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap) { return 2 * cap + kSlotBytes; }
+    __host__ __device__ static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * per_warp(cap); }
 };
 static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
+static_assert(kSlotBytes % 16 == 0, "slots keep the buffers 16-byte aligned");
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
@@ -160,117 +161,99 @@ __device__ __forceinline__ void cp_async16(uint8_t *dst_smem, const void *src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
 }
 
-// Stage-1 bulk loop for two chains (A, B) of one lane, in PTX so that each
-// lookup costs a fixed, short instruction sequence.  Per active chain and
-// lookup: index = top 12 bits of the window (mad.hi adds the table base),
-// entry = codes | bits << 4, sum += entry (the code count is recovered as
-// sum - 16 * bits), advance the 96-bit window.  A chain is active while
-// pos < bulk_end.  Leaves early, state intact, when an active chain meets a
-// code longer than 12 bits (entry bits == 0); the caller resolves it.
-__device__ __forceinline__ void count_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &sA, int &posA,
-                                            uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &sB, int &posB,
-                                            int bendA, int bendB, uint32_t cnt_base)
+// Shared-memory accesses by 32-bit address.  They are volatile (kept in
+// program order with each other and with the PTX loops); the staging slots
+// and write buffers they touch are not accessed through C++ pointers.
+__device__ __forceinline__ void st_u8(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
+__device__ __forceinline__ uint32_t ld_u8(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void st_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
+// Bulk decode loop for two chains (A, B) of one lane, in PTX.  Symbol-table
+// entry: up to three rotated exponents in bytes 0..2, their total length in
+// bits 24..28, their number in bits 29..30 (0 = a code longer than 12 bits).
+// A chain is active while pos < bend (its last 12 bits are left to the
+// caller).  Per lookup: the three exponent bytes go to the chain's staging
+// slot at q unconditionally (bytes past the codes found are overwritten by
+// the next lookup or never read), q advances by the count, the window and pos
+// by the length.  (entry >> 24) serves as the funnel-shift amount directly:
+// wrap mode reads only its low five bits.  Leaves early, state intact, when an
+// active chain meets a long code.
+__device__ __forceinline__ void decode_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA, int &posA,
+                                             uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB, int &posB,
+                                             int bendA, int bendB, uint32_t sym_base)
 {
     asm volatile(
         "{\n\t"
         ".reg .pred pa, pb, pz, pl;\n\t"
-        ".reg .u32 ea, eb, ca, cb;\n\t"
-        "CB_TOP:\n\t"
+        ".reg .u32 ea, eb, ca, cb, t;\n\t"
+        "DB_TOP:\n\t"
         "setp.lt.s32 pa, %4, %10;\n\t"
         "setp.lt.s32 pb, %9, %11;\n\t"
         "or.pred pz, pa, pb;\n\t"
-        "@!pz bra CB_END;\n\t"
-        "@pa mad.hi.u32 ea, %0, 4096, %12;\n\t"
-        "@pb mad.hi.u32 eb, %5, 4096, %12;\n\t"
-        "@pa ld.shared.u8 ea, [ea];\n\t"
-        "@pb ld.shared.u8 eb, [eb];\n\t"
-        "@pa shr.u32 ca, ea, 4;\n\t"
-        "@pb shr.u32 cb, eb, 4;\n\t"
-        "setp.eq.and.u32 pl, ca, 0, pa;\n\t"
-        "setp.eq.and.u32 pz, cb, 0, pb;\n\t"
-        "or.pred pl, pl, pz;\n\t"
-        "@pl bra CB_END;\n\t"
-        "@pa add.u32 %3, %3, ea;\n\t"
-        "@pa add.s32 %4, %4, ca;\n\t"
-        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
-        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
-        "@pa shl.b32 %2, %2, ca;\n\t"
-        "@pb add.u32 %8, %8, eb;\n\t"
-        "@pb add.s32 %9, %9, cb;\n\t"
-        "@pb shf.l.wrap.b32 %5, %6, %5, cb;\n\t"
-        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
-        "@pb shl.b32 %7, %7, cb;\n\t"
-        "bra CB_TOP;\n\t"
-        "CB_END:\n\t"
-        "}"
-        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(sA), "+r"(posA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(sB), "+r"(posB)
-        : "r"(bendA), "r"(bendB), "r"(cnt_base)
-        : "memory");
-}
-
-// Stage-2 loop for two chains, in PTX.  Symbol-table entry: up to three
-// rotated exponents in bytes 0..2, their total length in bits 24..28, their
-// number in bits 29..30 (0 = a code longer than 12 bits).  The length is
-// used as a funnel-shift amount in wrap mode, which reads only its low five
-// bits, so (entry >> 24) serves directly.  Each active chain stores one to
-// three exponent bytes at its shared-memory cursor q (q < qend), bytes two
-// and three only while they stay below qend.  Leaves early, state intact,
-// when an active chain meets a long code.
-__device__ __forceinline__ void place_loop2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA,
-                                            uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
-                                            uint32_t qendA, uint32_t qend1A, uint32_t qend2A, uint32_t qendB,
-                                            uint32_t qend1B, uint32_t qend2B, uint32_t sym_base)
-{
-    asm volatile(
-        "{\n\t"
-        ".reg .pred pa, pb, pz, pl, p1, p2;\n\t"
-        ".reg .u32 ea, eb, ca, cb, na, nb, t;\n\t"
-        "PL_TOP:\n\t"
-        "setp.lt.u32 pa, %3, %8;\n\t"
-        "setp.lt.u32 pb, %7, %11;\n\t"
-        "or.pred pz, pa, pb;\n\t"
-        "@!pz bra PL_END;\n\t"
+        "@!pz bra DB_END;\n\t"
         "@pa shr.u32 ea, %0, 20;\n\t"
-        "@pb shr.u32 eb, %4, 20;\n\t"
-        "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"
-        "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"
+        "@pb shr.u32 eb, %5, 20;\n\t"
+        "@pa mad.lo.u32 ea, ea, 4, %12;\n\t"
+        "@pb mad.lo.u32 eb, eb, 4, %12;\n\t"
         "@pa ld.shared.u32 ea, [ea];\n\t"
         "@pb ld.shared.u32 eb, [eb];\n\t"
         "setp.eq.and.u32 pl, ea, 0, pa;\n\t"
         "setp.eq.and.u32 pz, eb, 0, pb;\n\t"
         "or.pred pl, pl, pz;\n\t"
-        "@pl bra PL_END;\n\t"
-        "@pa shr.u32 ca, ea, 24;\n\t"
-        "@pa mul.hi.u32 na, ea, 8;\n\t"
+        "@pl bra DB_END;\n\t"
+        // chain A
         "@pa st.shared.u8 [%3], ea;\n\t"
-        "setp.lt.and.u32 p1, %3, %9, pa;\n\t"
-        "setp.lt.and.u32 p2, %3, %10, pa;\n\t"
-        "@p1 mul.hi.u32 t, ea, 16777216;\n\t"
-        "@p1 st.shared.u8 [%3+1], t;\n\t"
-        "@p2 mul.hi.u32 t, ea, 65536;\n\t"
-        "@p2 st.shared.u8 [%3+2], t;\n\t"
-        "@pa add.u32 %3, %3, na;\n\t"
+        "@pa mul.hi.u32 t, ea, 16777216;\n\t"
+        "@pa st.shared.u8 [%3+1], t;\n\t"
+        "@pa mul.hi.u32 t, ea, 65536;\n\t"
+        "@pa st.shared.u8 [%3+2], t;\n\t"
+        "@pa shr.u32 ca, ea, 24;\n\t"
+        "@pa mul.hi.u32 t, ea, 8;\n\t"
+        "@pa add.u32 %3, %3, t;\n\t"
+        "@pa and.b32 t, ca, 31;\n\t"
+        "@pa add.s32 %4, %4, t;\n\t"
         "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
+        // chain B
+        "@pb st.shared.u8 [%8], eb;\n\t"
+        "@pb mul.hi.u32 t, eb, 16777216;\n\t"
+        "@pb st.shared.u8 [%8+1], t;\n\t"
+        "@pb mul.hi.u32 t, eb, 65536;\n\t"
+        "@pb st.shared.u8 [%8+2], t;\n\t"
         "@pb shr.u32 cb, eb, 24;\n\t"
-        "@pb mul.hi.u32 nb, eb, 8;\n\t"
-        "@pb st.shared.u8 [%7], eb;\n\t"
-        "setp.lt.and.u32 p1, %7, %12, pb;\n\t"
-        "setp.lt.and.u32 p2, %7, %13, pb;\n\t"
-        "@p1 mul.hi.u32 t, eb, 16777216;\n\t"
-        "@p1 st.shared.u8 [%7+1], t;\n\t"
-        "@p2 mul.hi.u32 t, eb, 65536;\n\t"
-        "@p2 st.shared.u8 [%7+2], t;\n\t"
-        "@pb add.u32 %7, %7, nb;\n\t"
-        "@pb shf.l.wrap.b32 %4, %5, %4, cb;\n\t"
+        "@pb mul.hi.u32 t, eb, 8;\n\t"
+        "@pb add.u32 %8, %8, t;\n\t"
+        "@pb and.b32 t, cb, 31;\n\t"
+        "@pb add.s32 %9, %9, t;\n\t"
         "@pb shf.l.wrap.b32 %5, %6, %5, cb;\n\t"
-        "@pb shf.l.wrap.b32 %6, 0, %6, cb;\n\t"
-        "bra PL_TOP;\n\t"
-        "PL_END:\n\t"
+        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
+        "@pb shf.l.wrap.b32 %7, 0, %7, cb;\n\t"
+        "bra DB_TOP;\n\t"
+        "DB_END:\n\t"
         "}"
-        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB)
-        : "r"(qendA), "r"(qend1A), "r"(qend2A), "r"(qendB), "r"(qend1B), "r"(qend2B), "r"(sym_base)
+        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB), "+r"(posB)
+        : "r"(bendA), "r"(bendB), "r"(sym_base)
         : "memory");
 }
 
@@ -301,23 +284,71 @@ __device__ __forceinline__ void load_block(const Params &p, uint32_t b, int lane
     r.o1 = __ldg(p.offs + b + 1);
 }
 
+// Copies each of two chains' staging slots (shared address src[k], 4-byte
+// aligned, len[k] bytes) to the write buffer at shared address dst[k]: the up
+// to three bytes before dst's first word boundary and after its last one
+// singly (those words are shared with neighbouring chains), the words in
+// between as 32-bit stores assembled by funnel shifts; both chains step
+// through one loop.
+__device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32_t src0[2], const uint32_t len0[2])
+{
+    uint32_t dst[2], src[2], nw[2], sh[2], sa[2], cur[2], tail[2];
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        uint32_t head = (4u - (dst0[k] & 3u)) & 3u;
+        head = head < len0[k] ? head : len0[k];
+#pragma unroll
+        for (uint32_t i = 0; i < 3; i++)
+            if (i < head)
+                st_u8(dst0[k] + i, ld_u8(src0[k] + i));
+        dst[k] = dst0[k] + head;
+        src[k] = src0[k] + head;
+        const uint32_t len = len0[k] - head;
+        nw[k] = len >> 2;
+        tail[k] = len & 3u;
+        sh[k] = 8u * (src[k] & 3u);
+        sa[k] = src[k] & ~3u;
+        cur[k] = ld_u32(sa[k]);
+    }
+    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
+    for (uint32_t w = 0; w < nmax; w++) {
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            if (w < nw[k]) {
+                const uint32_t nxt = ld_u32(sa[k] + 4 * w + 4);
+                st_u32(dst[k] + 4 * w, __funnelshift_r(cur[k], nxt, sh[k]));
+                cur[k] = nxt;
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        const uint32_t o = 4 * nw[k];
+#pragma unroll
+        for (uint32_t i = 0; i < 3; i++)
+            if (i < tail[k])
+                st_u8(dst[k] + o + i, ld_u8(src[k] + o + i));
+    }
+}
+
 // C = segments per lane: the format block is 32 * C segments, one warp; lane
 // l decodes segments l, l + 32, ... as C independent chains.  WARPS warps per
 // CTA, one CTA per SM.
 template <int C, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params p)
 {
+    static_assert(C == 1 || C == 2, "one or two chains per lane");
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
     constexpr uint32_t T = 32 * C;
     extern __shared__ __align__(128) uint8_t smem[];
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
-    uint8_t *cnt_tab = smem + Smem::cnt;
     uint8_t *luts = smem + Smem::luts;
     uint8_t *cl = smem + Smem::cl;
-    uint16_t *ztab = reinterpret_cast<uint16_t *>(smem + Smem::ztab);
+    uint8_t *zq = smem + Smem::zq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint8_t *exp_s = smem + Smem::bufs + warp * 2 * p.cap;
+    uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
     uint8_t *sm_s = exp_s + p.cap;
+    uint8_t *slots = sm_s + p.cap;
 
     // the first block's registers load while the tables are built
     const uint32_t stride = gridDim.x * kWarps;
@@ -333,44 +364,19 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     for (uint32_t i = tid; i < 256; i += kThreads)
         cl[i] = p.cl[i];
     __syncthreads();
-    // Derived tables.  first_code[i]: the first code of the 12-bit window i
-    // (bits past 12 taken as zeros): symbol | length << 8, or 0 when that code
-    // is longer than 12 bits.  A code found in a zero-filled window is genuine
-    // when it ends inside the window (prefix property).  Scratch lives in the
-    // per-warp buffers, which are free until the blocks start.
+    // first_code[i]: the first code of the 12-bit window i (bits past 12 taken
+    // as zeros): symbol | length << 8, or 0 when that code is longer than 12
+    // bits.  A code found in a zero-filled window is genuine when it ends
+    // inside the window (prefix property).  Scratch in the per-warp buffers,
+    // which are free until the blocks start.
     uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
-    uint16_t *greedy = first_code + kIdxEntries;  // levels r = 0..11, 2^r entries each
     for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
         bool bad = false;
         const uint32_t e = lut_decode(i << (32 - kIdxBits), luts, cl, p.num_luts, &bad);
         const uint32_t len = e >> 8;
         first_code[i] = (!bad && len >= 1 && len <= kIdxBits) ? (uint16_t)e : (uint16_t)0;
     }
-    if (tid == 0)
-        greedy[0] = 0;
     __syncthreads();
-    // Count table by levels: G_r(v) = whole codes (and their bits) read
-    // greedily from the r-bit value v; G_r(v) = 1 + G_{r-l}(v without its
-    // first code of length l), or nothing when that code needs more than r
-    // bits.  G_12 is the count table (codes | bits << 4).
-    for (uint32_t r = 1; r <= kIdxBits; r++) {
-        const uint32_t nv = 1u << r;
-        for (uint32_t v = tid; v < nv; v += kThreads) {
-            const uint32_t fc = first_code[(v << (kIdxBits - r)) & (kIdxEntries - 1)];
-            const uint32_t len = fc >> 8;
-            uint32_t g = 0;  // codes | bits << 8
-            if (len != 0 && len <= r) {
-                const uint32_t rest = r - len;
-                const uint32_t gr = greedy[(1u << rest) - 1 + (v & ((1u << rest) - 1))];
-                g = (1u + (gr & 0xFFu)) | ((len + (gr >> 8)) << 8);
-            }
-            if (r < kIdxBits)
-                greedy[nv - 1 + v] = (uint16_t)g;
-            else
-                cnt_tab[v] = (uint8_t)((g & 0xFFu) | ((g >> 8) << 4));
-        }
-        __syncthreads();
-    }
     // Symbol table: the first three codes of each window, by three dependent
     // first_code lookups.
     for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
@@ -388,15 +394,20 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         // exponents in bytes 0..2, total length in bits 24..28, count in 29..30
         sym_tab[i] = syms | (bits << 24) | (n << 29);
     }
-    if (tid <= kIdxBits) {
-        // codes formed by the zero bits r..11 after a code boundary: the
-        // all-zero code (the canonical first code) repeated; count | bits << 8
+    if (tid < 16) {
+        // codes formed by d trailing zero bits, d = 0..15: the all-zero code
+        // (the canonical first code, of length lmin) repeated d / lmin times;
+        // bit 7 flags d as a multiple of lmin
         bool bad = false;
         const uint32_t lmin = lut_decode(0u, luts, cl, p.num_luts, &bad) >> 8;
-        const uint32_t z = (lmin >= 1 && !bad) ? (kIdxBits - tid) / lmin : 0u;
-        ztab[tid] = (uint16_t)(z | ((z * lmin) << 8));
+        const uint32_t d = (uint32_t)tid;
+        zq[tid] = (lmin >= 1 && !bad) ? (uint8_t)((d / lmin) | ((d % lmin == 0) << 7)) : (uint8_t)0;
     }
     __syncthreads();
+
+    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(sym_tab));
+    const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
+    const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * kSlotStride;
 
     // ---- each warp walks its own blocks; no block-wide barrier from here on
     for (; b < p.nblocks; b += stride) {
@@ -418,82 +429,99 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 
         // ---- locate: chain k's codes start in [pos0, pend) of its window
         bool bad = false;
-        int pos0[C], pend[C];
-        uint32_t w0[C], w1[C], w2[C], cnt[C];
+        int pos0[2] = {0, 0}, pend[2] = {0, 0};
+        uint32_t h[2] = {0u, 0u}, m[2] = {0u, 0u}, l[2] = {0u, 0u};
 #pragma unroll
         for (int k = 0; k < C; k++) {
             const uint64_t seg = (uint64_t)b * T + lane + 32 * k;
             const uint32_t off = (uint32_t)((5 * seg) & 31);
             const uint64_t v = (((uint64_t)cur.g1[k] << 32) | cur.g0[k]) >> off;
             const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
-            pos0[k] = 0;
-            pend[k] = 0;
             if (seg < p.nseg) {
                 pos0[k] = (int)gap;
                 pend[k] = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
             }
-            w0[k] = bswap32(cur.s01[k].x);
-            w1[k] = bswap32(cur.s01[k].y);
-            w2[k] = bswap32(cur.s2[k]);
-            cnt[k] = 0;
+            h[k] = bswap32(cur.s01[k].x);
+            m[k] = bswap32(cur.s01[k].y);
+            l[k] = bswap32(cur.s2[k]);
+            shift_window(h[k], m[k], l[k], (uint32_t)pos0[k]);
         }
 
-        // ---- stage 1: count the codes of each chain, chains interleaved
+        // ---- decode each chain once into its staging slot
+        uint32_t cnt[2];
         {
-            const uint32_t cnt_base = static_cast<uint32_t>(__cvta_generic_to_shared(cnt_tab));
-            uint32_t h[2], m[2], l[2], sum[2] = {0u, 0u}, nlong[2] = {0u, 0u}, blong[2] = {0u, 0u};
+            uint32_t q[2], q0[2];
             int pos[2], bend[2];
 #pragma unroll
             for (int k = 0; k < 2; k++) {
-                const bool on = k < C;
-                h[k] = on ? w0[k < C ? k : 0] : 0u;
-                m[k] = on ? w1[k < C ? k : 0] : 0u;
-                l[k] = on ? w2[k < C ? k : 0] : 0u;
-                pos[k] = on ? pos0[k < C ? k : 0] : 0;
-                bend[k] = on ? pend[k < C ? k : 0] - kIdxBits : 0;
-                shift_window(h[k], m[k], l[k], (uint32_t)pos[k]);
+                q0[k] = slot_base + k * (32 * kSlotStride);
+                q[k] = q0[k];
+                pos[k] = pos0[k];
+                bend[k] = pend[k] - kIdxBits;
             }
-            for (;;) {  // each pass resolves >= 1 code or ends both chains
-                count_bulk2(h[0], m[0], l[0], sum[0], pos[0], h[1], m[1], l[1], sum[1], pos[1], bend[0], bend[1],
-                            cnt_base);
+            for (;;) {  // each pass resolves >= 1 code or ends both bulk loops
+                decode_bulk2(h[0], m[0], l[0], q[0], pos[0], h[1], m[1], l[1], q[1], pos[1], bend[0], bend[1],
+                             sym_base);
                 bool any_long = false;
 #pragma unroll
                 for (int k = 0; k < 2; k++) {
-                    if (pos[k] < bend[k] && (cnt_tab[h[k] >> (32 - kIdxBits)] >> 4) == 0) {
+                    if (pos[k] < bend[k] && sym_tab[h[k] >> (32 - kIdxBits)] == 0) {
                         // a code longer than 12 bits: the page's LUTs
-                        uint32_t c = lut_decode(h[k], luts, cl, p.num_luts, &bad) >> 8;
-                        c = c ? c : 1u;
-                        nlong[k] += 1;
-                        blong[k] += c;
-                        pos[k] += (int)c;
-                        shift_window(h[k], m[k], l[k], c);
+                        const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
+                        const uint32_t len = (d >> 8) ? (d >> 8) : 1u;
+                        st_u8(q[k], ror8(d & 0xFFu));
+                        q[k] += 1;
+                        pos[k] += (int)len;
+                        shift_window(h[k], m[k], l[k], len);
                         any_long = true;
                     }
                 }
                 if (!any_long)
                     break;
             }
+            // the last <= 12 bits of each chain: lookups on the masked window,
+            // both chains per pass
+            for (int it = 0; it < kIdxBits; it++) {
+                bool any = false;
 #pragma unroll
-            for (int k = 0; k < C; k++) {
-                // table lookups added codes + 16 * bits
-                cnt[k] = sum[k] - 16u * ((uint32_t)(pos[k] - pos0[k]) - blong[k]) + nlong[k];
-                const int r = pend[k] - pos[k];
-                if (r > 0) {
-                    // the last r <= 12 bits hold whole codes; mask the rest
+                for (int k = 0; k < 2; k++) {
+                    if (pos[k] >= pend[k])
+                        continue;
+                    any = true;
+                    const int r0 = pend[k] - pos[k];  // 1..12 for consistent data
+                    const int r = r0 < kIdxBits ? r0 : kIdxBits;
                     const uint32_t idx = (h[k] >> (32 - kIdxBits)) & ((0xFFFu << (kIdxBits - r)) & 0xFFFu);
-                    const uint32_t e = cnt_tab[idx];
-                    const uint32_t z = ztab[r];
-                    cnt[k] += (e & 15u) - (z & 0xFFu);
-                    bad |= (e >> 4) - (z >> 8) != (uint32_t)r;
-                } else if (r < 0) {
-                    bad = true;
+                    const uint32_t e = sym_tab[idx];
+                    uint32_t n = e >> 29, c = (e >> 24) & 31u;
+                    if (c > (uint32_t)r) {  // the entry read into the zero fill
+                        const uint32_t z = zq[(c - r) & 15u];
+                        const uint32_t zn = z & 0x7Fu;
+                        bad |= !(z & 0x80u) || zn >= n;
+                        n = zn < n ? n - zn : 1u;
+                        c = (uint32_t)r;
+                    }
+                    bad |= n == 0 || r0 > kIdxBits;
+                    n = n ? n : 1u;
+                    c = c ? c : 1u;
+                    st_u8(q[k], e);
+                    st_u8(q[k] + 1, e >> 8);
+                    st_u8(q[k] + 2, e >> 16);
+                    q[k] += n;
+                    pos[k] += (int)c;
+                    shift_window(h[k], m[k], l[k], c);
                 }
+                if (!any)
+                    break;
+            }
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                bad |= pos[k] != pend[k];
+                cnt[k] = q[k] - q0[k];
             }
         }
 
         // ---- warp prefix sum of the counts; both chains in one packed scan
-        // (a chain's block total is at most 64 * 32 < 2^16)
-        static_assert(C == 1 || C == 2, "one or two chains per lane");
+        // (a chain holds at most 64 codes, a block at most 2048 per chain)
         uint32_t packed = 0;
 #pragma unroll
         for (int k = 0; k < C; k++)
@@ -506,16 +534,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
                 incl += y;
         }
         const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-        uint32_t first[C];
+        uint32_t first[2] = {0u, 0u};
         uint32_t total = 0;
 #pragma unroll
         for (int k = 0; k < C; k++) {
             first[k] = total + ((incl >> (16 * k)) & 0xFFFFu) - cnt[k];
             total += (tot >> (16 * k)) & 0xFFFFu;
-        }
-#pragma unroll
-        for (int k = 0; k < C; k++)
             bad |= cnt[k] > 64u;
+        }
         const bool block_bad = __any_sync(0xffffffffu, bad) || !offs_ok || total != o1 - o0;
         if (block_bad) {
             if (lane == 0)
@@ -523,42 +549,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
         } else {
-            // ---- stage 2: decode again, place rotated exponents
+            // ---- place: each chain's slot into the write buffer
             {
-                const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(sym_tab));
-                const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
-                uint32_t h[2], m[2], l[2], q[2], qend[2], qend1[2], qend2[2];
-#pragma unroll
-                for (int k = 0; k < 2; k++) {
-                    const bool on = k < C;
-                    const int kk = k < C ? k : 0;
-                    h[k] = w0[kk];
-                    m[k] = w1[kk];
-                    l[k] = w2[kk];
-                    shift_window(h[k], m[k], l[k], (uint32_t)pos0[kk]);
-                    // shared-memory byte addresses (never near 0, so q - 2 cannot wrap)
-                    q[k] = exp_base + lo_off + first[kk];
-                    qend[k] = on ? q[k] + cnt[kk] : q[k];
-                    qend1[k] = qend[k] - 1;  // a second exponent fits while q < qend - 1
-                    qend2[k] = qend[k] - 2;  // a third one while q < qend - 2
-                }
-                for (;;) {  // each pass places >= 1 exponent or ends both chains
-                    place_loop2(h[0], m[0], l[0], q[0], h[1], m[1], l[1], q[1], qend[0], qend1[0], qend2[0], qend[1],
-                                qend1[1], qend2[1], sym_base);
-                    bool any_long = false;
-#pragma unroll
-                    for (int k = 0; k < 2; k++) {
-                        if (q[k] < qend[k] && sym_tab[h[k] >> (32 - kIdxBits)] == 0) {
-                            const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
-                            exp_s[q[k] - exp_base] = (uint8_t)ror8(d & 0xFFu);
-                            q[k] += 1;
-                            shift_window(h[k], m[k], l[k], d >> 8);
-                            any_long = true;
-                        }
-                    }
-                    if (!any_long)
-                        break;
-                }
+                const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
+                const uint32_t srcs[2] = {slot_base, slot_base + 32 * kSlotStride};
+                copy_slots2(dsts, srcs, cnt);
             }
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
@@ -601,7 +596,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 struct DeviceFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][3] = {};  // [C - 1][warps 32 / 16 / 8]
+    uint32_t granted[2][4] = {};  // [C - 1][warps 32 / 24 / 16 / 8]
 };
 std::mutex g_mu;
 DeviceFacts g_dev[64];
@@ -649,8 +644,8 @@ df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, 
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
-// 32 warps per CTA unless their buffers do not fit in shared memory (blocks of
-// very short codes hold up to 64 outputs per segment): then 16 or 8.
+// As many warps per CTA (32, 24, 16 or 8) as the per-warp buffers allow in
+// shared memory; blocks of very short codes hold up to 64 outputs per segment.
 template <int C>
 df11_status launch(const Params &prm, cudaStream_t stream)
 {
@@ -661,10 +656,12 @@ df11_status launch(const Params &prm, cudaStream_t stream)
     const uint32_t optin = (uint32_t)f->smem_optin;
     if (Smem::bytes(prm.cap, 32) <= optin)
         return launch_warps<C, 32>(prm, stream, Smem::bytes(prm.cap, 32), f, f->granted[C - 1][0]);
+    if (Smem::bytes(prm.cap, 24) <= optin)
+        return launch_warps<C, 24>(prm, stream, Smem::bytes(prm.cap, 24), f, f->granted[C - 1][1]);
     if (Smem::bytes(prm.cap, 16) <= optin)
-        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[C - 1][1]);
+        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[C - 1][2]);
     if (Smem::bytes(prm.cap, 8) <= optin)
-        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[C - 1][2]);
+        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[C - 1][3]);
     return DF11_ERR_INVALID_ARG;
 }
 
@@ -710,11 +707,8 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     prm.nseg = nseg;
     prm.nblocks = a->num_blocks;
     prm.num_luts = a->num_luts;
-    // at least 16 KB of buffers even with 8 warps: they hold set-up scratch
-    // (two 4096-entry uint16 tables)
+    // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
     prm.cap = align16(a->max_block_elems + 32);
-    if (prm.cap < 1024)
-        prm.cap = 1024;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
 }
