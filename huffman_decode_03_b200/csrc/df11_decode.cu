@@ -188,47 +188,46 @@ __device__ __forceinline__ void st_u32(uint32_t addr, uint32_t v)
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
 }
 
-// Bulk decode loop for two chains (A, B) of one lane, in PTX.  Symbol-table
+// Decode loop for two chains (A, B) of one lane, in PTX.  Symbol-table
 // entry: up to three rotated exponents in bytes 0..2, their total length in
 // bits 24..28, their number in bits 29..30 (0 = a code longer than 12 bits).
-// A chain is active while pos < bend (its last 12 bits are left to the
-// caller).  Per lookup: the three exponent bytes go to the chain's staging
-// slot at q unconditionally (bytes past the codes found are overwritten by
-// the next lookup or never read), q advances by the count, the window and pos
-// by the length.  (entry >> 24) serves as the funnel-shift amount directly:
-// wrap mode reads only its low five bits.  Leaves early, state intact, when an
-// active chain meets a long code.
+// A chain is active while pos < pend and its last entry was not 0; the bits
+// of its window past pend are zeros.  Per lookup: the three exponent bytes go
+// to the chain's staging slot at q unconditionally (bytes past the codes
+// found are overwritten by the next lookup or never read), q advances by the
+// count, the window and pos by the length.  (entry >> 24) serves as the
+// funnel-shift amount directly: wrap mode reads only its low five bits.  An
+// entry of 0 changes nothing and stops its chain: the caller resolves that
+// long code, resets the chain's entry to non-zero and calls again.
 __device__ __forceinline__ void decode_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA, int &posA,
-                                             uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB, int &posB,
-                                             int bendA, int bendB, uint32_t sym_base)
+                                             uint32_t &eA, uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
+                                             int &posB, uint32_t &eB, int pendA, int pendB, uint32_t sym_base)
 {
     asm volatile(
         "{\n\t"
-        ".reg .pred pa, pb, pz, pl;\n\t"
-        ".reg .u32 ea, eb, ca, cb, t;\n\t"
+        ".reg .pred pa, pb, pz;\n\t"
+        ".reg .u32 ca, cb, t;\n\t"
         "DB_TOP:\n\t"
-        "setp.lt.s32 pa, %4, %10;\n\t"
-        "setp.lt.s32 pb, %9, %11;\n\t"
+        "setp.lt.s32 pa, %4, %12;\n\t"
+        "setp.lt.s32 pb, %10, %13;\n\t"
+        "setp.ne.and.u32 pa, %5, 0, pa;\n\t"
+        "setp.ne.and.u32 pb, %11, 0, pb;\n\t"
         "or.pred pz, pa, pb;\n\t"
         "@!pz bra DB_END;\n\t"
-        "@pa shr.u32 ea, %0, 20;\n\t"
-        "@pb shr.u32 eb, %5, 20;\n\t"
-        "@pa mad.lo.u32 ea, ea, 4, %12;\n\t"
-        "@pb mad.lo.u32 eb, eb, 4, %12;\n\t"
-        "@pa ld.shared.u32 ea, [ea];\n\t"
-        "@pb ld.shared.u32 eb, [eb];\n\t"
-        "setp.eq.and.u32 pl, ea, 0, pa;\n\t"
-        "setp.eq.and.u32 pz, eb, 0, pb;\n\t"
-        "or.pred pl, pl, pz;\n\t"
-        "@pl bra DB_END;\n\t"
+        "@pa shr.u32 %5, %0, 20;\n\t"
+        "@pb shr.u32 %11, %6, 20;\n\t"
+        "@pa mad.lo.u32 %5, %5, 4, %14;\n\t"
+        "@pb mad.lo.u32 %11, %11, 4, %14;\n\t"
+        "@pa ld.shared.u32 %5, [%5];\n\t"
+        "@pb ld.shared.u32 %11, [%11];\n\t"
         // chain A
-        "@pa st.shared.u8 [%3], ea;\n\t"
-        "@pa mul.hi.u32 t, ea, 16777216;\n\t"
+        "@pa st.shared.u8 [%3], %5;\n\t"
+        "@pa mul.hi.u32 t, %5, 16777216;\n\t"
         "@pa st.shared.u8 [%3+1], t;\n\t"
-        "@pa mul.hi.u32 t, ea, 65536;\n\t"
+        "@pa mul.hi.u32 t, %5, 65536;\n\t"
         "@pa st.shared.u8 [%3+2], t;\n\t"
-        "@pa shr.u32 ca, ea, 24;\n\t"
-        "@pa mul.hi.u32 t, ea, 8;\n\t"
+        "@pa shr.u32 ca, %5, 24;\n\t"
+        "@pa mul.hi.u32 t, %5, 8;\n\t"
         "@pa add.u32 %3, %3, t;\n\t"
         "@pa and.b32 t, ca, 31;\n\t"
         "@pa add.s32 %4, %4, t;\n\t"
@@ -236,24 +235,25 @@ __device__ __forceinline__ void decode_bulk2(uint32_t &hA, uint32_t &mA, uint32_
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
         // chain B
-        "@pb st.shared.u8 [%8], eb;\n\t"
-        "@pb mul.hi.u32 t, eb, 16777216;\n\t"
-        "@pb st.shared.u8 [%8+1], t;\n\t"
-        "@pb mul.hi.u32 t, eb, 65536;\n\t"
-        "@pb st.shared.u8 [%8+2], t;\n\t"
-        "@pb shr.u32 cb, eb, 24;\n\t"
-        "@pb mul.hi.u32 t, eb, 8;\n\t"
-        "@pb add.u32 %8, %8, t;\n\t"
+        "@pb st.shared.u8 [%9], %11;\n\t"
+        "@pb mul.hi.u32 t, %11, 16777216;\n\t"
+        "@pb st.shared.u8 [%9+1], t;\n\t"
+        "@pb mul.hi.u32 t, %11, 65536;\n\t"
+        "@pb st.shared.u8 [%9+2], t;\n\t"
+        "@pb shr.u32 cb, %11, 24;\n\t"
+        "@pb mul.hi.u32 t, %11, 8;\n\t"
+        "@pb add.u32 %9, %9, t;\n\t"
         "@pb and.b32 t, cb, 31;\n\t"
-        "@pb add.s32 %9, %9, t;\n\t"
-        "@pb shf.l.wrap.b32 %5, %6, %5, cb;\n\t"
+        "@pb add.s32 %10, %10, t;\n\t"
         "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
-        "@pb shf.l.wrap.b32 %7, 0, %7, cb;\n\t"
+        "@pb shf.l.wrap.b32 %7, %8, %7, cb;\n\t"
+        "@pb shf.l.wrap.b32 %8, 0, %8, cb;\n\t"
         "bra DB_TOP;\n\t"
         "DB_END:\n\t"
         "}"
-        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB), "+r"(posB)
-        : "r"(bendA), "r"(bendB), "r"(sym_base)
+        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(eA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB),
+          "+r"(posB), "+r"(eB)
+        : "r"(pendA), "r"(pendB), "r"(sym_base)
         : "memory");
 }
 
@@ -328,6 +328,57 @@ __device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32
         for (uint32_t i = 0; i < 3; i++)
             if (i < tail[k])
                 st_u8(dst[k] + o + i, ld_u8(src[k] + o + i));
+    }
+}
+
+// Places every chain's staging slot in the write buffer with 32-bit stores
+// only; valid when every chain of the block holds >= 3 codes.  Chain c covers
+// bytes [s_c, s_c + cnt_c) of the buffer.  It writes the words from the one
+// holding s_c up to, not including, the word that holds its own last byte
+// (the next chain writes that one); the block's last chain also writes its
+// final partial word.  The bytes of a chain's first word that precede s_c are
+// the previous chain's last bytes: each chain reads its last four slot bytes
+// as one word and passes it on by shuffle.  src[k]: the chain's slot (4-byte
+// aligned shared address); s[k]: its byte offset in the buffer at shared
+// address exp_base.
+template <int C>
+__device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[2], const uint32_t src[2],
+                                            const uint32_t cnt[2], int lane)
+{
+    uint32_t last[2] = {0u, 0u}, prev[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+        const uint32_t t = src[k] + cnt[k] - 4u;  // >= src[k] - 1: inside the shared buffers
+        const uint32_t a = t & ~3u;
+        last[k] = __funnelshift_r(ld_u32(a), ld_u32(a + 4), 8u * (t & 3u));
+        prev[k] = __shfl_up_sync(0xffffffffu, last[k], 1);
+    }
+    if (C == 2) {
+        // chain (lane 0, B) follows chain (lane 31, A)
+        const uint32_t x = __shfl_sync(0xffffffffu, last[0], 31);
+        if (lane == 0)
+            prev[1] = x;
+    }
+    uint32_t dst[2] = {0u, 0u}, sa[2] = {0u, 0u}, nw[2] = {0u, 0u}, sh[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+        const uint32_t e = s[k] + cnt[k];
+        const bool final_chain = lane == 31 && k == C - 1;
+        dst[k] = exp_base + (s[k] & ~3u);
+        sa[k] = src[k];
+        nw[k] = (final_chain ? (e + 3u) >> 2 : e >> 2) - (s[k] >> 2);
+        sh[k] = 8u * (s[k] & 3u);
+    }
+    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
+    for (uint32_t w = 0; w < nmax; w++) {
+#pragma unroll
+        for (int k = 0; k < C; k++) {
+            if (w < nw[k]) {
+                const uint32_t cur = ld_u32(sa[k] + 4 * w);
+                st_u32(dst[k] + 4 * w, __funnelshift_l(prev[k], cur, sh[k]));
+                prev[k] = cur;
+            }
+        }
     }
 }
 
@@ -444,79 +495,57 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             h[k] = bswap32(cur.s01[k].x);
             m[k] = bswap32(cur.s01[k].y);
             l[k] = bswap32(cur.s2[k]);
+            // bits from pend on belong to the next chain: zeros instead
+            const uint32_t pe = (uint32_t)pend[k];
+            h[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe);
+            m[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 32u ? pe - 32u : 0u);
+            l[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 64u ? pe - 64u : 0u);
             shift_window(h[k], m[k], l[k], (uint32_t)pos0[k]);
         }
 
-        // ---- decode each chain once into its staging slot
+        // ---- decode each chain once into its staging slot.  Past pend the
+        // window reads zeros, which decode as the all-zero code (the
+        // canonical first code, of length lmin); the last lookup of a chain
+        // starts on one of its own codes, so at most its two further codes
+        // are such zero codes: pos overshoots pend by a multiple of lmin
+        // (< 12) and the count by overshoot / lmin.
         uint32_t cnt[2];
         {
-            uint32_t q[2], q0[2];
-            int pos[2], bend[2];
+            uint32_t q[2], q0[2], e[2] = {1u, 1u};
+            int pos[2];
 #pragma unroll
             for (int k = 0; k < 2; k++) {
                 q0[k] = slot_base + k * (32 * kSlotStride);
                 q[k] = q0[k];
                 pos[k] = pos0[k];
-                bend[k] = pend[k] - kIdxBits;
             }
-            for (;;) {  // each pass resolves >= 1 code or ends both bulk loops
-                decode_bulk2(h[0], m[0], l[0], q[0], pos[0], h[1], m[1], l[1], q[1], pos[1], bend[0], bend[1],
-                             sym_base);
+            for (;;) {  // each pass resolves >= 1 code or ends both chains
+                decode_bulk2(h[0], m[0], l[0], q[0], pos[0], e[0], h[1], m[1], l[1], q[1], pos[1], e[1], pend[0],
+                             pend[1], sym_base);
                 bool any_long = false;
 #pragma unroll
                 for (int k = 0; k < 2; k++) {
-                    if (pos[k] < bend[k] && sym_tab[h[k] >> (32 - kIdxBits)] == 0) {
-                        // a code longer than 12 bits: the page's LUTs
+                    if (pos[k] < pend[k]) {
+                        // stopped on a code longer than 12 bits: the page's LUTs
                         const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
                         const uint32_t len = (d >> 8) ? (d >> 8) : 1u;
                         st_u8(q[k], ror8(d & 0xFFu));
                         q[k] += 1;
                         pos[k] += (int)len;
                         shift_window(h[k], m[k], l[k], len);
+                        e[k] = 1u;
                         any_long = true;
                     }
                 }
                 if (!any_long)
                     break;
             }
-            // the last <= 12 bits of each chain: lookups on the masked window,
-            // both chains per pass
-            for (int it = 0; it < kIdxBits; it++) {
-                bool any = false;
-#pragma unroll
-                for (int k = 0; k < 2; k++) {
-                    if (pos[k] >= pend[k])
-                        continue;
-                    any = true;
-                    const int r0 = pend[k] - pos[k];  // 1..12 for consistent data
-                    const int r = r0 < kIdxBits ? r0 : kIdxBits;
-                    const uint32_t idx = (h[k] >> (32 - kIdxBits)) & ((0xFFFu << (kIdxBits - r)) & 0xFFFu);
-                    const uint32_t e = sym_tab[idx];
-                    uint32_t n = e >> 29, c = (e >> 24) & 31u;
-                    if (c > (uint32_t)r) {  // the entry read into the zero fill
-                        const uint32_t z = zq[(c - r) & 15u];
-                        const uint32_t zn = z & 0x7Fu;
-                        bad |= !(z & 0x80u) || zn >= n;
-                        n = zn < n ? n - zn : 1u;
-                        c = (uint32_t)r;
-                    }
-                    bad |= n == 0 || r0 > kIdxBits;
-                    n = n ? n : 1u;
-                    c = c ? c : 1u;
-                    st_u8(q[k], e);
-                    st_u8(q[k] + 1, e >> 8);
-                    st_u8(q[k] + 2, e >> 16);
-                    q[k] += n;
-                    pos[k] += (int)c;
-                    shift_window(h[k], m[k], l[k], c);
-                }
-                if (!any)
-                    break;
-            }
 #pragma unroll
             for (int k = 0; k < 2; k++) {
-                bad |= pos[k] != pend[k];
-                cnt[k] = q[k] - q0[k];
+                const uint32_t d = (uint32_t)(pos[k] - pend[k]);  // >= 0
+                const uint32_t z = zq[d & 15u];
+                bad |= d > 15u || !(z & 0x80u);
+                cnt[k] = q[k] - q0[k] - (z & 0x7Fu);
             }
         }
 
@@ -549,11 +578,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
         } else {
-            // ---- place: each chain's slot into the write buffer
+            // ---- place: each chain's slot into the write buffer; whole words
+            // when every chain holds >= 3 codes (the normal case), else
+            // with single bytes at the chains' edges
             {
-                const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
                 const uint32_t srcs[2] = {slot_base, slot_base + 32 * kSlotStride};
-                copy_slots2(dsts, srcs, cnt);
+                bool short_chain = cnt[0] < 3u;
+                if (C == 2)
+                    short_chain |= cnt[1] < 3u;
+                if (!__any_sync(0xffffffffu, short_chain)) {
+                    const uint32_t offs2[2] = {lo_off + first[0], lo_off + first[1]};
+                    place_words<C>(exp_base, offs2, srcs, cnt, lane);
+                } else {
+                    const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
+                    copy_slots2(dsts, srcs, cnt);
+                }
             }
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
