@@ -47,8 +47,10 @@
 //     funnel shifts and compares;
 //   * the next block's stream words, Gaps words and offsets are loaded into
 //     registers while the current block is decoded; the current block's
-//     sign/mantissa bytes arrive in shared memory by asynchronous copies
-//     (cp.async) during decoding.
+//     sign/mantissa bytes are prefetched into L2 (one bulk prefetch by the
+//     TMA unit) when its decoding starts and read from there by the merge,
+//     which keeps shared memory for 32 warps per SM: their number, not a
+//     staging copy, hides the load latency.
 // Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
 
@@ -89,14 +91,14 @@ struct Params {
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
 // Shared memory: tables at fixed offsets, then per warp: the exponent write
-// buffer, the block's sign/mantissa bytes and the chains' staging slots.
+// buffer and the chains' staging slots.
 struct Smem {
     static constexpr uint32_t sym = 0;                       // uint32[4096]
     static constexpr uint32_t luts = sym + kIdxEntries * 4;  // 17 * 256
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
     static constexpr uint32_t zq = cl + 256;                 // uint8[16]
     static constexpr uint32_t bufs = zq + 16;
-    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap) { return 2 * cap + kSlotBytes; }
+    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap) { return cap + kSlotBytes; }
     __host__ __device__ static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * per_warp(cap); }
 };
 static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
@@ -153,12 +155,6 @@ __device__ __forceinline__ void merge4(uint32_t S, uint32_t E, uint32_t &lo2, ui
 __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
 {
     return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
-}
-
-__device__ __forceinline__ void cp_async16(uint8_t *dst_smem, const void *src)
-{
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
 }
 
 // Shared-memory accesses by 32-bit address.  They are volatile (kept in
@@ -398,8 +394,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     uint8_t *zq = smem + Smem::zq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
-    uint8_t *sm_s = exp_s + p.cap;
-    uint8_t *slots = sm_s + p.cap;
+    uint8_t *slots = exp_s + p.cap;
 
     // the first block's registers load while the tables are built
     const uint32_t stride = gridDim.x * kWarps;
@@ -460,6 +455,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * kSlotStride;
 
+
     // ---- each warp walks its own blocks; no block-wide barrier from here on
     for (; b < p.nblocks; b += stride) {
         if (b + stride < p.nblocks)
@@ -469,14 +465,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         const uint64_t g0 = (uint64_t)o0 - lo_off;  // multiple of 16
         const bool offs_ok = o1 >= o0 && (uint64_t)o1 <= p.n && (uint64_t)lo_off + (o1 - o0) + 16u <= p.cap;
 
-        // ---- the block's sign/mantissa bytes: asynchronous copy, waited for
-        // just before the merge
-        if (offs_ok) {
-            const uint32_t nbytes = align16(lo_off + (o1 - o0));
-            for (uint32_t off = 16 * lane; off < nbytes; off += 16 * 32)
-                cp_async16(sm_s + off, p.sm + g0 + off);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        // ---- the block's sign/mantissa bytes: into L2 now, read by the merge
+        const uint32_t nbytes = offs_ok ? align16(lo_off + (o1 - o0)) : 0u;
+        if (nbytes && lane == 0)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + g0), "r"(nbytes) : "memory");
 
         // ---- locate: chain k's codes start in [pos0, pend) of its window
         bool bad = false;
@@ -575,7 +567,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         if (block_bad) {
             if (lane == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
         } else {
             // ---- place: each chain's slot into the write buffer; whole words
@@ -594,33 +585,32 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
                     copy_slots2(dsts, srcs, cnt);
                 }
             }
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
             __syncwarp();
 
-            // ---- merge with sign/mantissa, coalesced 16-byte stores
+            // ---- merge with sign/mantissa (from L2): 8 elements per lane and
+            // step, so that a warp's 16-byte stores cover 512 contiguous bytes
             const uint32_t hi = lo_off + total;
-            const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
-            for (uint32_t c = c_first + lane; c < c_end; c += 32) {
-                const uint32_t l0 = 16 * c;
-                const uint4 s = *reinterpret_cast<const uint4 *>(sm_s + l0);
-                const uint4 e = *reinterpret_cast<const uint4 *>(exp_s + l0);
-                uint4 r0, r1;
-                merge4(s.x, e.x, r0.x, r0.y);
-                merge4(s.y, e.y, r0.z, r0.w);
-                merge4(s.z, e.z, r1.x, r1.y);
-                merge4(s.w, e.w, r1.z, r1.w);
-                uint4 *d = reinterpret_cast<uint4 *>(p.dst + g0 + l0);
-                d[0] = r0;
-                d[1] = r1;
+            const uint32_t u_first = (lo_off + 7u) >> 3, u_end = hi >> 3;  // full units [u_first, u_end)
+            const uint8_t *smg = p.sm + g0;
+#pragma unroll 4
+            for (uint32_t u = u_first + lane; u < u_end; u += 32) {
+                const uint32_t l0 = 8 * u;
+                const uint2 s2 = __ldg(reinterpret_cast<const uint2 *>(smg + l0));
+                const uint2 e2 = *reinterpret_cast<const uint2 *>(exp_s + l0);
+                uint4 r;
+                merge4(s2.x, e2.x, r.x, r.y);
+                merge4(s2.y, e2.y, r.z, r.w);
+                *reinterpret_cast<uint4 *>(p.dst + g0 + l0) = r;
             }
-            // partial first chunk (lanes 0..15) and partial last chunk
-            // (lanes 16..31): one element per lane
+            // the partial units before u_first (lanes 0..15) and from u_end
+            // on (lanes 16..31): one element per lane
             {
-                const bool head = lane < 16;
-                const uint32_t l = head ? lane : 16 * c_end + (lane - 16);
-                const bool want = head ? (lo_off != 0 || hi < 16) : (c_end > 0 && (hi & 15u) != 0);
-                if (want && l >= lo_off && l < hi)
-                    p.dst[g0 + l] = merge1(sm_s[l], exp_s[l]);
+                const uint32_t head_end = 8 * u_first < hi ? 8 * u_first : hi;
+                const uint32_t tail0 = 8 * (u_end > u_first ? u_end : u_first);
+                const uint32_t l = lane < 16 ? (uint32_t)lane : tail0 + (lane - 16);
+                const bool want = lane < 16 ? (l >= lo_off && l < head_end) : (lane < 24 && l < hi);
+                if (want)
+                    p.dst[g0 + l] = merge1(__ldg(smg + l), exp_s[l]);
             }
             __syncwarp();
         }
