@@ -86,6 +86,7 @@ struct Params {
     uint32_t nblocks;
     uint32_t num_luts;
     uint32_t cap;  // bytes of one warp's exponent (and sign/mantissa) buffer
+    uint32_t wide;  // dst is 32-byte aligned: the merge uses 32-byte stores
 };
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -587,24 +588,51 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             }
             __syncwarp();
 
-            // ---- merge with sign/mantissa (from L2): 8 elements per lane and
-            // step, so that a warp's 16-byte stores cover 512 contiguous bytes
+            // ---- merge with sign/mantissa (from L2)
             const uint32_t hi = lo_off + total;
-            const uint32_t u_first = (lo_off + 7u) >> 3, u_end = hi >> 3;  // full units [u_first, u_end)
             const uint8_t *smg = p.sm + g0;
+            if (p.wide) {
+                // 16 elements per lane and step, one 32-byte store: a warp's
+                // stores cover 1 KB contiguous
+                const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
+#pragma unroll 2
+                for (uint32_t c = c_first + lane; c < c_end; c += 32) {
+                    const uint32_t l0 = 16 * c;
+                    const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(smg + l0));
+                    const uint4 e4 = *reinterpret_cast<const uint4 *>(exp_s + l0);
+                    uint32_t r[8];
+                    merge4(s4.x, e4.x, r[0], r[1]);
+                    merge4(s4.y, e4.y, r[2], r[3]);
+                    merge4(s4.z, e4.z, r[4], r[5]);
+                    merge4(s4.w, e4.w, r[6], r[7]);
+                    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p.dst + g0 + l0),
+                                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                                 "r"(r[7])
+                                 : "memory");
+                }
+                // partial first chunk (lanes 0..15) and partial last chunk
+                // (lanes 16..31): one element per lane
+                const bool head = lane < 16;
+                const uint32_t l = head ? lane : 16 * c_end + (lane - 16);
+                const bool want = head ? (lo_off != 0 || hi < 16) : (c_end > 0 && (hi & 15u) != 0);
+                if (want && l >= lo_off && l < hi)
+                    p.dst[g0 + l] = merge1(__ldg(smg + l), exp_s[l]);
+            } else {
+                // 8 elements per lane and step, one 16-byte store: a warp's
+                // stores cover 512 contiguous bytes
+                const uint32_t u_first = (lo_off + 7u) >> 3, u_end = hi >> 3;  // full units [u_first, u_end)
 #pragma unroll 4
-            for (uint32_t u = u_first + lane; u < u_end; u += 32) {
-                const uint32_t l0 = 8 * u;
-                const uint2 s2 = __ldg(reinterpret_cast<const uint2 *>(smg + l0));
-                const uint2 e2 = *reinterpret_cast<const uint2 *>(exp_s + l0);
-                uint4 r;
-                merge4(s2.x, e2.x, r.x, r.y);
-                merge4(s2.y, e2.y, r.z, r.w);
-                *reinterpret_cast<uint4 *>(p.dst + g0 + l0) = r;
-            }
-            // the partial units before u_first (lanes 0..15) and from u_end
-            // on (lanes 16..31): one element per lane
-            {
+                for (uint32_t u = u_first + lane; u < u_end; u += 32) {
+                    const uint32_t l0 = 8 * u;
+                    const uint2 s2 = __ldg(reinterpret_cast<const uint2 *>(smg + l0));
+                    const uint2 e2 = *reinterpret_cast<const uint2 *>(exp_s + l0);
+                    uint4 r;
+                    merge4(s2.x, e2.x, r.x, r.y);
+                    merge4(s2.y, e2.y, r.z, r.w);
+                    *reinterpret_cast<uint4 *>(p.dst + g0 + l0) = r;
+                }
+                // the partial units before u_first (lanes 0..15) and from
+                // u_end on (lanes 16..31): one element per lane
                 const uint32_t head_end = 8 * u_first < hi ? 8 * u_first : hi;
                 const uint32_t tail0 = 8 * (u_end > u_first ? u_end : u_first);
                 const uint32_t l = lane < 16 ? (uint32_t)lane : tail0 + (lane - 16);
@@ -738,6 +766,7 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     prm.num_luts = a->num_luts;
     // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
     prm.cap = align16(a->max_block_elems + 32);
+    prm.wide = aligned(dst, 32) ? 1u : 0u;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
 }

@@ -128,19 +128,22 @@ def test_multi_matrix(oracle_mod):
     assert np.array_equal(got, ref)
 
 
-def test_output_alignment_and_neighbours():
-    # decoding into the middle of a larger buffer writes exactly n elements
+@pytest.mark.parametrize("offset", [8, 16])
+def test_output_alignment_and_neighbours(offset):
+    # decoding into the middle of a larger buffer writes exactly n elements;
+    # offset 8 leaves the output 16-byte aligned only (16-byte stores),
+    # offset 16 makes it 32-byte aligned (32-byte stores)
     torch = torch_cuda()
     w = inputs.gaussian(12_345, [24])
     fmt = df11.build_format(w)
     dev = df11.DeviceFormat(fmt, "cuda")
     buf = torch.full((12_345 + 64,), 7, dtype=torch.int16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    df11.decompress(dev, buf[8:].view(torch.bfloat16), status)
+    df11.decompress(dev, buf[offset:].view(torch.bfloat16), status)
     assert df11.read_status(status) == 0
     h = buf.cpu().numpy().view(np.uint16)
-    assert np.all(h[:8] == 7) and np.all(h[8 + 12_345:] == 7)
-    assert np.array_equal(h[8:8 + 12_345], w)
+    assert np.all(h[:offset] == 7) and np.all(h[offset + 12_345:] == 7)
+    assert np.array_equal(h[offset:offset + 12_345], w)
 
 
 def test_repeated_launches_are_identical():
