@@ -76,7 +76,8 @@ class df11_info(ctypes.Structure):
 
 EXPORTS = (
     "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
-    "df11_strerror", "df11_decompress", "df11_decompress_host", "df11_read_status",
+    "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_host",
+    "df11_read_status",
 )
 
 _lib = None
@@ -105,6 +106,8 @@ def load_library(path: str | None = None):
     lib.df11_strerror.restype = ctypes.c_char_p
     lib.df11_decompress.argtypes = [ctypes.POINTER(df11_arrays), P, P, P]
     lib.df11_decompress.restype = ctypes.c_int
+    lib.df11_decompress_sms.argtypes = [ctypes.POINTER(df11_arrays), P, P, P, ctypes.c_uint32]
+    lib.df11_decompress_sms.restype = ctypes.c_int
     lib.df11_decompress_host.argtypes = [
         ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_arrays), P, P, P, P]
     lib.df11_decompress_host.restype = ctypes.c_int
@@ -264,9 +267,10 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def decompress(dev: DeviceFormat, out=None, status=None, stream=None):
+def decompress(dev: DeviceFormat, out=None, status=None, stream=None, max_sms: int = 0):
     """Rebuilds the BF16 stream on the GPU (asynchronous, stream-ordered).
-    Returns ``out`` (a torch.bfloat16 tensor of n elements, allocated if None)."""
+    Returns ``out`` (a torch.bfloat16 tensor of n elements, allocated if None).
+    ``max_sms`` > 0 caps the SMs the decoder occupies (df11_decompress_sms)."""
     import torch
 
     if out is None:
@@ -274,9 +278,12 @@ def decompress(dev: DeviceFormat, out=None, status=None, stream=None):
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev.device)
     assert out.is_cuda and out.is_contiguous() and out.numel() >= dev.n and out.element_size() == 2
-    _check(load_library().df11_decompress(ctypes.byref(dev.c_arrays), ctypes.c_void_p(out.data_ptr()),
-                                          ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
-           "df11_decompress")
+    args = (ctypes.byref(dev.c_arrays), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(status.data_ptr()),
+            _stream_ptr(stream))
+    if max_sms:
+        _check(load_library().df11_decompress_sms(*args, int(max_sms)), "df11_decompress_sms")
+    else:
+        _check(load_library().df11_decompress(*args), "df11_decompress")
     return out
 
 

@@ -87,6 +87,7 @@ struct Params {
     uint32_t num_luts;
     uint32_t cap;  // bytes of one warp's exponent (and sign/mantissa) buffer
     uint32_t wide;  // dst is 32-byte aligned: the merge uses 32-byte stores
+    uint32_t max_ctas;  // 0 = one CTA on every SM
 };
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -694,6 +695,8 @@ df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, 
     // one persistent CTA per SM: __launch_bounds__(WARPS * 32, 1) and the
     // shared-memory footprint allow no second one
     uint64_t grid = (uint64_t)f->sms;
+    if (prm.max_ctas && prm.max_ctas < grid)
+        grid = prm.max_ctas;
     const uint64_t need = (prm.nblocks + WARPS - 1) / WARPS;
     if (grid > need)
         grid = need;
@@ -724,7 +727,9 @@ df11_status launch(const Params &prm, cudaStream_t stream)
 
 }  // namespace
 
-extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream)
+namespace {
+df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream,
+                            uint32_t max_sms)
 {
     if (!a || !status_dev)
         return DF11_ERR_INVALID_ARG;
@@ -767,8 +772,21 @@ extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint
     // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
     prm.cap = align16(a->max_block_elems + 32);
     prm.wide = aligned(dst, 32) ? 1u : 0u;
+    prm.max_ctas = max_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
+}
+}  // namespace
+
+extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream)
+{
+    return decompress_impl(a, dst, status_dev, stream, 0);
+}
+
+extern "C" df11_status df11_decompress_sms(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream,
+                                           uint32_t max_sms)
+{
+    return decompress_impl(a, dst, status_dev, stream, max_sms);
 }
 
 extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arrays *d, uint16_t *dst_dev,

@@ -168,6 +168,17 @@ df11_status df11_decompress(const df11_arrays *dev, uint16_t *dst,
                             uint32_t *status_dev, void *stream);
 
 /*
+ * df11_decompress_sms -- df11_decompress on at most `max_sms` SMs
+ * ("Dekompresi per transformer block": decompressing the next block while
+ * the current one is used).  The decoder otherwise runs one persistent CTA
+ * on every SM, which leaves no SM to kernels on other streams until it ends;
+ * a cap leaves the remaining SMs to them.  max_sms = 0 means every SM (the
+ * same as df11_decompress); arguments, outputs and errors as there.
+ */
+df11_status df11_decompress_sms(const df11_arrays *dev, uint16_t *dst,
+                                uint32_t *status_dev, void *stream, uint32_t max_sms);
+
+/*
  * df11_decompress_host -- the same decode, starting and ending in host
  * memory: copies every array of *host (host pointers, ideally pinned) into
  * the device buffers named by *dev_buffers (device pointers with at least the

@@ -146,6 +146,18 @@ def test_output_alignment_and_neighbours(offset):
     assert np.array_equal(h[offset:offset + 12_345], w)
 
 
+@pytest.mark.parametrize("max_sms", [1, 3, 17, 1000])
+def test_sm_cap_gives_the_same_result(max_sms):
+    # df11_decompress_sms: fewer persistent CTAs walk more blocks each
+    torch = torch_cuda()
+    w = inputs.gaussian(3_000_017, [26])
+    dev = df11.DeviceFormat(df11.build_format(w), "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = df11.decompress(dev, None, status, max_sms=max_sms)
+    assert df11.read_status(status) == 0
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), w)
+
+
 def test_repeated_launches_are_identical():
     torch = torch_cuda()
     w = inputs.gaussian(1 << 20, [25])
