@@ -34,10 +34,11 @@
 //     turns the final BF16 merge into two bit-selects and two byte permutes
 //     per 4 elements.  Codes longer than 12 bits fall back to the page's
 //     pointer-chasing LUTs;
-//   * a chain stops exactly at its last code: the next segment's Gap gives the
-//     bit where the next chain starts; the lookups of the last <= 12 bits
-//     mask the bits past that point to zeros, and the codes the zeros form
-//     (the all-zero code is the canonical first code) are discounted;
+//   * a chain ends exactly at its last code: the next segment's Gap gives the
+//     bit where the next chain starts; the chain's window reads zeros past
+//     that bit, the decode loop runs until the position passes it, and the
+//     codes the zeros form (the all-zero code is the canonical first code;
+//     at most two per chain) are discounted;
 //   * each chain's 64 + 32 bits live in a three-register shift window: the
 //     table index is the top 12 bits, a step is three funnel shifts;
 //   * the decode loop is hand-written PTX: both chains of a lane step in one
@@ -50,7 +51,12 @@
 //     sign/mantissa bytes are prefetched into L2 (one bulk prefetch by the
 //     TMA unit) when its decoding starts and read from there by the merge,
 //     which keeps shared memory for 32 warps per SM: their number, not a
-//     staging copy, hides the load latency.
+//     staging copy, hides the load latency;
+//   * the merge writes 16 outputs per lane with one 32-byte store when the
+//     output is 32-byte aligned (a warp's stores then cover 1 KB contiguous);
+//   * df11_decompress_sms caps the persistent grid below one CTA per SM, so
+//     that kernels on other streams (the use of the previous transformer
+//     block) can run beside the decode.
 // Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
 
@@ -456,7 +462,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(sym_tab));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * kSlotStride;
-
 
     // ---- each warp walks its own blocks; no block-wide barrier from here on
     for (; b < p.nblocks; b += stride) {
