@@ -77,7 +77,8 @@ class df11_info(ctypes.Structure):
 EXPORTS = (
     "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
     "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_host",
-    "df11_read_status",
+    "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
+    "df11_device_encode_scratch_words", "df11_device_encode",
 )
 
 _lib = None
@@ -113,6 +114,14 @@ def load_library(path: str | None = None):
     lib.df11_decompress_host.restype = ctypes.c_int
     lib.df11_read_status.argtypes = [P, P]
     lib.df11_read_status.restype = ctypes.c_int
+    lib.df11_device_histogram.argtypes = [P, ctypes.c_uint64, P, P]
+    lib.df11_device_histogram.restype = ctypes.c_int
+    lib.df11_plan_from_histogram.argtypes = [P, ctypes.c_uint32, ctypes.POINTER(P)]
+    lib.df11_plan_from_histogram.restype = ctypes.c_int
+    lib.df11_device_encode_scratch_words.argtypes = [ctypes.c_uint64]
+    lib.df11_device_encode_scratch_words.restype = ctypes.c_uint64
+    lib.df11_device_encode.argtypes = [P, P, ctypes.POINTER(df11_arrays), P, ctypes.c_uint64, P, P, P]
+    lib.df11_device_encode.restype = ctypes.c_int
     if path == _build.LIB_PATH:
         _lib = lib
     return lib
@@ -236,6 +245,21 @@ class DeviceFormat:
         self.c_arrays = self._struct(self.tensors)
         self.c_host_arrays = self._struct(self.host_tensors) if pin_host else None
 
+    @classmethod
+    def from_tensors(cls, scalars: dict, tensors: dict, device) -> "DeviceFormat":
+        """A stream whose arrays are already device tensors (uint8, named as in
+        ``Format.arrays()``), e.g. the output of ``encode_device``."""
+        import torch
+
+        self = cls.__new__(cls)
+        self.device = torch.device(device)
+        self.scalars = dict(scalars)
+        self.tensors = dict(tensors)
+        self.host_tensors = {}
+        self.c_arrays = self._struct(self.tensors)
+        self.c_host_arrays = None
+        return self
+
     def _struct(self, ts) -> df11_arrays:
         a = df11_arrays()
         for k, v in self.scalars.items():
@@ -296,6 +320,73 @@ def decompress_host(dev: DeviceFormat, out_dev, out_host, status, stream=None):
         ctypes.c_void_p(out_host.data_ptr()), ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
         "df11_decompress_host")
     return out_host
+
+
+def encode_device(w, threads_per_block: int = 64, stream=None):
+    """Compresses BF16 weights that are already on the GPU: exponent histogram
+    on the device (df11_device_histogram), the code from the 256 counts on the
+    host (df11_plan_from_histogram), every array on the device
+    (df11_device_encode).  ``w``: a contiguous CUDA tensor of bfloat16 (or
+    16-bit integer) patterns, any shape, read in memory order.  Returns
+    ``(DeviceFormat, Format)``: the stream, whose arrays never left the device,
+    and its plan (code, LUTs, statistics).  Synchronises ``stream`` twice: the
+    counts and the largest block size come back to the host."""
+    import torch
+
+    lib = load_library()
+    flat = w.detach().reshape(-1)
+    if flat.dtype == torch.bfloat16:
+        flat = flat.view(torch.int16)
+    if not (flat.is_cuda and flat.element_size() == 2 and flat.is_contiguous()):
+        raise ValueError("encode_device needs a contiguous CUDA tensor of 16-bit patterns")
+    dev = flat.device
+    n = flat.numel()
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(s.cuda_stream)
+    wp = ctypes.c_void_p(flat.data_ptr() if n else None)
+    hist = torch.empty(256, dtype=torch.int64, device=dev)
+    _check(lib.df11_device_histogram(wp, n, ctypes.c_void_p(hist.data_ptr()), sp), "df11_device_histogram")
+    s.synchronize()
+    hist_host = hist.cpu().numpy()
+    h = ctypes.c_void_p()
+    _check(lib.df11_plan_from_histogram(hist_host.ctypes.data, int(threads_per_block), ctypes.byref(h)),
+           "df11_plan_from_histogram")
+    plan = Format(h.value, lib)
+    a = plan.c_arrays
+    sizes = {
+        "encoded_exponent": int(a.encoded_exponent_bytes),
+        "packed_sign_mantissa": int(a.packed_sign_mantissa_bytes),
+        "gaps": 8 * int(a.gaps_words),
+        "block_offset": 4 * (int(a.num_blocks) + 1),
+        "luts": 256 * int(a.num_luts),
+        "code_lengths": 256,
+    }
+    with torch.cuda.stream(s):
+        tensors = {k: torch.empty(v, dtype=torch.uint8, device=dev) for k, v in sizes.items()}
+        words = int(lib.df11_device_encode_scratch_words(n))
+        scratch = torch.empty(max(words, 1), dtype=torch.int64, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        maxb = torch.zeros(1, dtype=torch.int32, device=dev)
+    dst = df11_arrays()
+    dst.encoded_exponent = tensors["encoded_exponent"].data_ptr()
+    dst.encoded_exponent_bytes = sizes["encoded_exponent"]
+    dst.packed_sign_mantissa = tensors["packed_sign_mantissa"].data_ptr()
+    dst.packed_sign_mantissa_bytes = sizes["packed_sign_mantissa"]
+    dst.gaps = tensors["gaps"].data_ptr()
+    dst.gaps_words = int(a.gaps_words)
+    dst.block_offset = tensors["block_offset"].data_ptr()
+    dst.luts = tensors["luts"].data_ptr()
+    dst.code_lengths = tensors["code_lengths"].data_ptr()
+    _check(lib.df11_device_encode(plan._h, wp, ctypes.byref(dst), ctypes.c_void_p(scratch.data_ptr()), words,
+                                  ctypes.c_void_p(maxb.data_ptr()), ctypes.c_void_p(status.data_ptr()), sp),
+           "df11_device_encode")
+    s.synchronize()
+    st = int(status.item())
+    if st:
+        raise Df11Error(6, f"df11_device_encode: the elements do not match their histogram (status word {st})")
+    scalars = plan.scalars()
+    scalars["max_block_elems"] = int(maxb.item())
+    return DeviceFormat.from_tensors(scalars, tensors, dev), plan
 
 
 def read_status(status, stream=None) -> int:

@@ -17,7 +17,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libdf11_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
-SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_format.cpp")]
+SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_encode.cu"),
+           os.path.join(CSRC, "df11_format.cpp")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

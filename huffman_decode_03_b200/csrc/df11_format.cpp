@@ -273,6 +273,7 @@ struct df11_format {
     uint8_t code_lengths[kSymbols];
     uint32_t codes[kSymbols];
     uint64_t hist[kSymbols];
+    bool plan_only = false;  // made by df11_plan_from_histogram: no host arrays
 };
 
 extern "C" df11_status df11_build_format(const uint16_t *const *mats, const uint64_t *counts,
@@ -488,6 +489,94 @@ extern "C" df11_status df11_build_format(const uint16_t *const *mats, const uint
         return DF11_ERR_NO_MEMORY;
     }
     *out = f;
+    return DF11_OK;
+}
+
+// A code without its arrays: the output of df11_plan_from_histogram.  Same
+// steps 2, 3a and 5 as df11_build_format, from a histogram instead of the
+// elements; the array sizes follow from sum(hist * length).
+extern "C" df11_status df11_plan_from_histogram(const uint64_t *hist, uint32_t T, df11_format **out)
+{
+    if (!out || !hist)
+        return DF11_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (T == 0)
+        T = DF11_DEFAULT_THREADS;
+    if (T < 32 || T > 1024 || T % 32)
+        return DF11_ERR_INVALID_ARG;
+    uint64_t n = 0;
+    for (int s = 0; s < kSymbols; s++) {
+        if (hist[s] && s >= kFirstPointer)
+            return DF11_ERR_UNSUPPORTED_EXPONENT;
+        n += hist[s];
+        if (n >= (1ull << 32))
+            return DF11_ERR_TOO_LARGE;
+    }
+    df11_format *f = new (std::nothrow) df11_format();
+    if (!f)
+        return DF11_ERR_NO_MEMORY;
+    try {
+        std::memcpy(f->hist, hist, sizeof(f->hist));
+        int longest = huffman_lengths(f->hist, f->code_lengths);
+        if (longest > DF11_MAX_CODE_LEN) {
+            if (!package_merge(f->hist, DF11_MAX_CODE_LEN, f->code_lengths)) {
+                delete f;
+                return DF11_ERR_INVALID_ARG;
+            }
+            longest = 0;
+            for (int s = 0; s < kSymbols; s++)
+                longest = std::max(longest, (int)f->code_lengths[s]);
+        }
+        canonical_codes(f->code_lengths, f->codes);
+        uint64_t total_bits = 0;
+        for (int s = 0; s < kSymbols; s++)
+            total_bits += f->hist[s] * f->code_lengths[s];
+        const uint64_t nseg = (total_bits + 63) / 64;
+        const uint64_t nblocks = (nseg + T - 1) / T;
+        if (nblocks >= (1ull << 31)) {
+            delete f;
+            return DF11_ERR_TOO_LARGE;
+        }
+        df11_status st = build_luts(f->code_lengths, f->codes, f->luts, &f->a.num_luts);
+        if (st != DF11_OK) {
+            delete f;
+            return st;
+        }
+        df11_arrays &a = f->a;
+        a.n = n;
+        a.total_bits = total_bits;
+        a.num_segments = nseg;
+        a.threads_per_block = T;
+        a.num_blocks = (uint32_t)nblocks;
+        a.max_code_len = (uint32_t)longest;
+        a.max_block_elems = 0;  // known once the elements are encoded
+        a.reserved = 0;
+        a.encoded_exponent = nullptr;
+        a.encoded_exponent_bytes = nblocks * T * 8 + 16;
+        a.packed_sign_mantissa = nullptr;
+        a.packed_sign_mantissa_bytes = ((n + 15) / 16) * 16 + 16;
+        a.gaps = nullptr;
+        a.gaps_words = (5 * nblocks * T + 63) / 64 + 2;
+        a.block_offset = nullptr;
+        a.luts = f->luts.data();
+        a.code_lengths = f->code_lengths;
+        f->plan_only = true;
+    } catch (const std::bad_alloc &) {
+        delete f;
+        return DF11_ERR_NO_MEMORY;
+    }
+    *out = f;
+    return DF11_OK;
+}
+
+// Read by the device encoder (df11_encode.cu): a plan's canonical codes.
+// Library-internal: not exported.
+__attribute__((visibility("hidden"))) df11_status df11_internal_plan_codes(const df11_format *f,
+                                                                           uint32_t *codes256)
+{
+    if (!f || !codes256)
+        return DF11_ERR_INVALID_ARG;
+    std::memcpy(codes256, f->codes, sizeof(f->codes));
     return DF11_OK;
 }
 

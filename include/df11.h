@@ -197,6 +197,73 @@ df11_status df11_decompress_host(const df11_arrays *host, const df11_arrays *dev
  */
 df11_status df11_read_status(const uint32_t *status_dev, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Compression of weights already in device memory.  The page compresses
+ * offline ("Format DFloat11"); these entry points run the same steps on the
+ * GPU and produce exactly the arrays df11_build_format builds on the host
+ * (the same code, the same bytes).  Three calls:
+ *   1. df11_device_histogram   exponent counts, on the device;
+ *   2. df11_plan_from_histogram the code, LUTs and array sizes, on the host;
+ *   3. df11_device_encode       every array, on the device, into buffers
+ *                               the caller allocated with the plan's sizes.
+ * ---------------------------------------------------------------------- */
+
+/*
+ * df11_device_histogram -- exponent histogram of n BF16 patterns.
+ *   w_dev     device pointer, 16-byte aligned, n uint16 (only read).
+ *   hist_dev  device pointer to 256 uint64, overwritten with the counts of
+ *             exponents 0..255 ("Ruang kompresi": the exponent is bits 7..14).
+ * Asynchronous on `stream`.  DF11_ERR_INVALID_ARG for NULL / misaligned
+ * pointers, DF11_ERR_CUDA if a launch fails.
+ */
+df11_status df11_device_histogram(const uint16_t *w_dev, uint64_t n, uint64_t *hist_dev, void *stream);
+
+/*
+ * df11_plan_from_histogram -- the code of a stream from its exponent counts
+ * ("Format DFloat11"; LUTs per "Decoding berbasis LUT hierarkis"): Huffman
+ * lengths (package-merge when deeper than 32), canonical codes, LUTs and
+ * CodeLengths, and the sizes of every array (total_bits = sum hist * length).
+ *   hist      host pointer to 256 counts (only read).
+ *   out       receives a handle owned by the caller (df11_free).  Its
+ *             df11_format_arrays view has the sizes, host pointers for luts
+ *             and code_lengths, NULL for the other arrays, and
+ *             max_block_elems = 0 (known once the elements are encoded).
+ * Errors as df11_build_format (exponents 240..255, n >= 2^32, > 16 child
+ * LUTs).
+ */
+df11_status df11_plan_from_histogram(const uint64_t *hist, uint32_t threads_per_block, df11_format **out);
+
+/* Scratch words df11_device_encode needs for n elements (one per chunk of
+ * 8192 elements, plus one). */
+uint64_t df11_device_encode_scratch_words(uint64_t n);
+
+/*
+ * df11_device_encode -- every array of the stream, on the device
+ * ("Format DFloat11"; Gaps and BlockOffset per "Kernel GPU 2 tahap dan
+ * metadata bantu").
+ *   plan      from df11_plan_from_histogram of these elements' histogram.
+ *   w_dev     device pointer, 16-byte aligned, plan's n uint16 (only read).
+ *   dst_dev   device pointers with at least the plan's sizes (alignment as
+ *             df11_decompress requires); all six arrays are written, the
+ *             LUTs and CodeLengths copied from the plan.  Its scalar fields
+ *             are not read.
+ *   scratch_dev  device pointer to scratch_words uint64 (at least
+ *             df11_device_encode_scratch_words(n)); contents need not start
+ *             at zero and are meaningless afterwards.
+ *   max_block_elems_dev  device pointer to one uint32: the largest block's
+ *             element count (the df11_arrays field of the same name).
+ *   status_dev  device pointer to one uint32, OR-accumulated with
+ *             DF11_ERR_CORRUPT when the elements do not match the plan (an
+ *             exponent without a code, or another total bit count); the
+ *             arrays are then not a valid stream.  Zero it first.
+ * Asynchronous on `stream`; every write stays inside the given sizes.
+ * DF11_ERR_INVALID_ARG for bad pointers, sizes or alignment, DF11_ERR_CUDA
+ * if a CUDA call fails.
+ */
+df11_status df11_device_encode(const df11_format *plan, const uint16_t *w_dev, const df11_arrays *dst_dev,
+                               uint64_t *scratch_dev, uint64_t scratch_words, uint32_t *max_block_elems_dev,
+                               uint32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
