@@ -78,7 +78,7 @@ EXPORTS = (
     "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
     "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_host",
     "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
-    "df11_device_encode_scratch_words", "df11_device_encode",
+    "df11_device_encode_scratch_words", "df11_device_encode", "df11_device_encode_static",
 )
 
 _lib = None
@@ -122,6 +122,8 @@ def load_library(path: str | None = None):
     lib.df11_device_encode_scratch_words.restype = ctypes.c_uint64
     lib.df11_device_encode.argtypes = [P, P, ctypes.POINTER(df11_arrays), P, ctypes.c_uint64, P, P, P]
     lib.df11_device_encode.restype = ctypes.c_int
+    lib.df11_device_encode_static.argtypes = [P, P, ctypes.POINTER(df11_arrays), P, P, P]
+    lib.df11_device_encode_static.restype = ctypes.c_int
     if path == _build.LIB_PATH:
         _lib = lib
     return lib
@@ -322,7 +324,7 @@ def decompress_host(dev: DeviceFormat, out_dev, out_host, status, stream=None):
     return out_host
 
 
-def encode_device(w, threads_per_block: int = 64, stream=None):
+def encode_device(w, threads_per_block: int = 64, stream=None, static_scratch: bool = False):
     """Compresses BF16 weights that are already on the GPU: exponent histogram
     on the device (df11_device_histogram), the code from the 256 counts on the
     host (df11_plan_from_histogram), every array on the device
@@ -330,7 +332,9 @@ def encode_device(w, threads_per_block: int = 64, stream=None):
     16-bit integer) patterns, any shape, read in memory order.  Returns
     ``(DeviceFormat, Format)``: the stream, whose arrays never left the device,
     and its plan (code, LUTs, statistics).  Synchronises ``stream`` twice: the
-    counts and the largest block size come back to the host."""
+    counts and the largest block size come back to the host.  With
+    ``static_scratch`` the encode step runs through df11_device_encode_static
+    (scratch inside the library; streams of at most 2^29 elements)."""
     import torch
 
     lib = load_library()
@@ -364,7 +368,7 @@ def encode_device(w, threads_per_block: int = 64, stream=None):
     with torch.cuda.stream(s):
         tensors = {k: torch.empty(v, dtype=torch.uint8, device=dev) for k, v in sizes.items()}
         words = int(lib.df11_device_encode_scratch_words(n))
-        scratch = torch.empty(max(words, 1), dtype=torch.int64, device=dev)
+        scratch = None if static_scratch else torch.empty(max(words, 1), dtype=torch.int64, device=dev)
         status = torch.zeros(1, dtype=torch.int32, device=dev)
         maxb = torch.zeros(1, dtype=torch.int32, device=dev)
     dst = df11_arrays()
@@ -377,9 +381,14 @@ def encode_device(w, threads_per_block: int = 64, stream=None):
     dst.block_offset = tensors["block_offset"].data_ptr()
     dst.luts = tensors["luts"].data_ptr()
     dst.code_lengths = tensors["code_lengths"].data_ptr()
-    _check(lib.df11_device_encode(plan._h, wp, ctypes.byref(dst), ctypes.c_void_p(scratch.data_ptr()), words,
-                                  ctypes.c_void_p(maxb.data_ptr()), ctypes.c_void_p(status.data_ptr()), sp),
-           "df11_device_encode")
+    if static_scratch:
+        _check(lib.df11_device_encode_static(plan._h, wp, ctypes.byref(dst), ctypes.c_void_p(maxb.data_ptr()),
+                                             ctypes.c_void_p(status.data_ptr()), sp),
+               "df11_device_encode_static")
+    else:
+        _check(lib.df11_device_encode(plan._h, wp, ctypes.byref(dst), ctypes.c_void_p(scratch.data_ptr()), words,
+                                      ctypes.c_void_p(maxb.data_ptr()), ctypes.c_void_p(status.data_ptr()), sp),
+               "df11_device_encode")
     s.synchronize()
     st = int(status.item())
     if st:

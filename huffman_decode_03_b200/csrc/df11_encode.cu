@@ -30,6 +30,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 df11_status df11_internal_plan_codes(const df11_format *f, uint32_t *codes256);  // df11_format.cpp
 
@@ -381,6 +382,32 @@ int sm_count()
     return sms;
 }
 
+// Scratch of df11_device_encode_static: one word per 8192-element chunk plus
+// one, for streams of up to 2^16 chunks = 2^29 elements (512 KiB).  Every
+// call writes each entry it reads before reading it, so nothing in it has to
+// start at zero.  One array per device, shared by every call.
+constexpr uint64_t kStaticMaxChunks = 1ull << 16;
+static __device__ __align__(256) uint64_t g_static_scratch[kStaticMaxChunks + 1];
+
+std::mutex g_static_mu;
+uint64_t *g_static_addr[64] = {};  // per device, looked up once
+
+df11_status static_scratch(uint64_t **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return DF11_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || !addr)
+            return DF11_ERR_CUDA;
+        g_static_addr[dev] = static_cast<uint64_t *>(addr);
+    }
+    *out = g_static_addr[dev];
+    return DF11_OK;
+}
+
 }  // namespace
 
 extern "C" df11_status df11_device_histogram(const uint16_t *w_dev, uint64_t n, uint64_t *hist_dev, void *stream)
@@ -476,4 +503,20 @@ extern "C" df11_status df11_device_encode(const df11_format *plan, const uint16_
     const uint32_t mgrid = (a.num_blocks + 255) / 256;
     max_block_kernel<<<mgrid ? (mgrid < 1024 ? mgrid : 1024) : 1, 256, 0, s>>>(prm.offs, a.num_blocks, max_block_dev);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+extern "C" df11_status df11_device_encode_static(const df11_format *plan, const uint16_t *w_dev,
+                                                 const df11_arrays *dst, uint32_t *max_block_dev,
+                                                 uint32_t *status_dev, void *stream)
+{
+    df11_arrays a;
+    if (!plan || df11_format_arrays(plan, &a) != DF11_OK)
+        return DF11_ERR_INVALID_ARG;
+    if (df11_device_encode_scratch_words(a.n) > kStaticMaxChunks + 1)
+        return DF11_ERR_TOO_LARGE;  // more than 2^29 elements
+    uint64_t *scratch = nullptr;
+    const df11_status st = static_scratch(&scratch);
+    if (st != DF11_OK)
+        return st;
+    return df11_device_encode(plan, w_dev, dst, scratch, kStaticMaxChunks + 1, max_block_dev, status_dev, stream);
 }

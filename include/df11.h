@@ -264,6 +264,28 @@ df11_status df11_device_encode(const df11_format *plan, const uint16_t *w_dev, c
                                uint64_t *scratch_dev, uint64_t scratch_words, uint32_t *max_block_elems_dev,
                                uint32_t *status_dev, void *stream);
 
+/*
+ * df11_device_encode_static -- df11_device_encode with its scratch in a
+ * fixed device array inside the library instead of a caller's buffer: the
+ * call allocates nothing.  The DFloat11 page has no counterpart (it
+ * compresses offline on the host); this variant is for callers that may not
+ * allocate device memory at the point of the call.
+ *   Limit: streams of at most 2^29 elements (65,536 chunks of 8192; the
+ *   array is 512 KiB per device).  Larger plans return DF11_ERR_TOO_LARGE
+ *   and nothing is launched.
+ *   plan, w_dev, dst_dev, max_block_elems_dev, status_dev, stream: as
+ *   df11_device_encode (status_dev must be zeroed by the caller).
+ * The array is shared by every call on a device: calls that overlap in time
+ * (on other streams or from other threads) race on it and must be
+ * serialised by the caller.  No entry of it has to start at zero (a call
+ * writes every entry it reads before reading it), so it is never cleared.
+ * The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  DF11_ERR_CUDA if the lookup fails.
+ */
+df11_status df11_device_encode_static(const df11_format *plan, const uint16_t *w_dev, const df11_arrays *dst_dev,
+                                      uint32_t *max_block_elems_dev, uint32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
