@@ -29,6 +29,15 @@ DF11_OK = 0
 DF11_ERR_CORRUPT = 6
 
 
+class df11_gemv_matrix(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_uint32),
+        ("cols", ctypes.c_uint32),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
 class Df11Error(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = int(status)
@@ -76,7 +85,7 @@ class df11_info(ctypes.Structure):
 
 EXPORTS = (
     "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
-    "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_host",
+    "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_gemv", "df11_decompress_host",
     "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
     "df11_device_encode_scratch_words", "df11_device_encode", "df11_device_encode_static",
 )
@@ -109,6 +118,9 @@ def load_library(path: str | None = None):
     lib.df11_decompress.restype = ctypes.c_int
     lib.df11_decompress_sms.argtypes = [ctypes.POINTER(df11_arrays), P, P, P, ctypes.c_uint32]
     lib.df11_decompress_sms.restype = ctypes.c_int
+    lib.df11_decompress_gemv.argtypes = [ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_gemv_matrix),
+                                         ctypes.c_uint32, P, P]
+    lib.df11_decompress_gemv.restype = ctypes.c_int
     lib.df11_decompress_host.argtypes = [
         ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_arrays), P, P, P, P]
     lib.df11_decompress_host.restype = ctypes.c_int
@@ -311,6 +323,32 @@ def decompress(dev: DeviceFormat, out=None, status=None, stream=None, max_sms: i
     else:
         _check(load_library().df11_decompress(*args), "df11_decompress")
     return out
+
+
+def decompress_gemv(dev: DeviceFormat, shapes, xs, ys, status=None, stream=None):
+    """Decode and use in one pass (df11_decompress_gemv): ``ys[m] += W_m @ xs[m]``
+    for the stream's matrices, of ``shapes[m] = (rows, cols)`` in stream order;
+    the decoded weights never reach memory.  ``xs``: CUDA bfloat16 vectors of
+    length cols (16-byte aligned); ``ys``: CUDA float32 vectors of length rows,
+    accumulated (zero them for y = W x).  Asynchronous; returns ``ys``."""
+    import torch
+
+    k = len(shapes)
+    if not (len(xs) == len(ys) == k):
+        raise ValueError("one activation vector and one output vector per matrix")
+    mats = (df11_gemv_matrix * max(k, 1))()
+    for m, ((rows, cols), x, y) in enumerate(zip(shapes, xs, ys)):
+        if x.dtype != torch.bfloat16 or y.dtype != torch.float32 or not (x.is_cuda and y.is_cuda):
+            raise ValueError("x must be CUDA bfloat16 and y CUDA float32")
+        if x.numel() != cols or y.numel() != rows or not (x.is_contiguous() and y.is_contiguous()):
+            raise ValueError(f"matrix {m}: x needs {cols} and y {rows} contiguous elements")
+        mats[m].rows, mats[m].cols, mats[m].x, mats[m].y = rows, cols, x.data_ptr(), y.data_ptr()
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev.device)
+    _check(load_library().df11_decompress_gemv(ctypes.byref(dev.c_arrays), mats, k,
+                                               ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
+           "df11_decompress_gemv")
+    return ys
 
 
 def decompress_host(dev: DeviceFormat, out_dev, out_host, status, stream=None):

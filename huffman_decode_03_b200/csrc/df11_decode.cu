@@ -63,6 +63,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 namespace {
@@ -76,6 +77,16 @@ constexpr uint32_t kSlotStride = 68;  // bytes per lane's staging slot (64 codes
 // inconsistent data (up to 95 one-bit codes + 2 spill bytes) stays inside the
 // warp's own slots; such a block is reported and writes nothing
 constexpr uint32_t kSlotBytes = 2 * 32 * kSlotStride + 32;
+
+// One matrix of a fused decode + matrix-vector product: rows x cols,
+// row-major, elements [off, end) of the stream; its rows are numbered
+// rowbase.. across the launch's matrices.
+struct GemvMat {
+    uint32_t end, off, cols, rowbase;
+    const uint16_t *x;  // cols BF16 activations
+    float *y;           // rows outputs, accumulated
+};
+constexpr uint32_t kMaxGemvMats = 16;
 
 struct Params {
     const uint8_t *stream;
@@ -94,6 +105,8 @@ struct Params {
     uint32_t cap;  // bytes of one warp's exponent (and sign/mantissa) buffer
     uint32_t wide;  // dst is 32-byte aligned: the merge uses 32-byte stores
     uint32_t max_ctas;  // 0 = one CTA on every SM
+    uint32_t num_mats;  // fused matrix-vector product (MODE 1) only
+    GemvMat mats[kMaxGemvMats];
 };
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -386,10 +399,125 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
     }
 }
 
+// Matrix of the fused product holding stream element g (matrices in order).
+__device__ __forceinline__ uint32_t gemv_matrix(const Params &p, uint32_t g)
+{
+    uint32_t m = 0;
+    while (m + 1 < p.num_mats && g >= p.mats[m].end)
+        m++;
+    return m;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(two & 0xFFFF0000u); }
+
+// Sums v over each run of lanes that hold the same key (a run's key is not
+// used by any other lane) and adds the sum to *y from the run's first lane
+// (y may be null: nothing to add).
+__device__ __forceinline__ void add_runs(float v, uint32_t key, float *y, int lane)
+{
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float o = __shfl_down_sync(0xffffffffu, v, d);
+        const uint32_t k = __shfl_down_sync(0xffffffffu, key, d);
+        if (lane + d < 32 && k == key)
+            v += o;
+    }
+    const uint32_t before = __shfl_up_sync(0xffffffffu, key, 1);
+    if ((lane == 0 || before != key) && y)
+        atomicAdd(y, v);
+}
+
+// Fused use of one decoded block (MODE 1): y += W x for the block's outputs
+// [g0 + lo_off, g0 + hi), instead of storing them.  16 elements per lane and
+// step (a 16-element chunk never crosses a row: columns and matrix sizes are
+// multiples of 16); products in fp32, summed per row over the warp, one
+// atomic add per row and step.  The ragged first and last chunks: one element
+// per lane.
+__device__ __forceinline__ void gemv_block(const Params &p, uint64_t g0, uint32_t lo_off, uint32_t hi,
+                                           const uint8_t *exp_s, int lane)
+{
+    const uint8_t *smg = p.sm + g0;
+    const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
+    // the lane's chunks are 512 elements apart: its matrix, row and column
+    // from one division, then advanced step by step
+    uint32_t m = 0, row = 0, col = 0;
+    {
+        const uint32_t g = (uint32_t)(g0 + 16 * (c_first + lane));
+        m = gemv_matrix(p, g);
+        const uint32_t rel = g - p.mats[m].off;
+        row = rel / p.mats[m].cols;
+        col = rel - row * p.mats[m].cols;
+    }
+    for (uint32_t base = c_first; base < c_end; base += 32) {
+        const uint32_t c = base + lane;
+        float v = 0.f;
+        uint32_t key = 0xFFFFFFFFu - lane;  // lanes without a chunk: runs of one, nothing to add
+        float *y = nullptr;
+        if (c < c_end) {
+            const uint32_t l0 = 16 * c;
+            const GemvMat &M = p.mats[m];
+            const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(smg + l0));
+            const uint4 e4 = *reinterpret_cast<const uint4 *>(exp_s + l0);
+            uint32_t w[8];
+            merge4(s4.x, e4.x, w[0], w[1]);
+            merge4(s4.y, e4.y, w[2], w[3]);
+            merge4(s4.z, e4.z, w[4], w[5]);
+            merge4(s4.w, e4.w, w[6], w[7]);
+            const uint4 *xp = reinterpret_cast<const uint4 *>(M.x + col);
+            const uint4 xa = __ldg(xp), xb = __ldg(xp + 1);
+            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                v = fmaf(bf16_lo(w[j]), bf16_lo(xw[j]), v);
+                v = fmaf(bf16_hi(w[j]), bf16_hi(xw[j]), v);
+            }
+            key = 2 * (M.rowbase + row);
+            y = M.y + row;
+            // next chunk of this lane: 512 elements on
+            const uint32_t g = (uint32_t)(g0 + l0) + 512u;
+            if (g < M.end) {
+                col += 512u;
+                while (col >= M.cols) {  // at most 512 / cols + 1 steps
+                    col -= M.cols;
+                    row++;
+                }
+            } else if (c + 32 < c_end) {
+                m = gemv_matrix(p, g);
+                const uint32_t rel = g - p.mats[m].off;
+                row = rel / p.mats[m].cols;
+                col = rel - row * p.mats[m].cols;
+            }
+        }
+        add_runs(v, key, y, lane);
+    }
+    // ragged chunks: lanes 0..15 the first, lanes 16..31 the last; the two
+    // halves get distinct keys even for the same row (runs must be unique)
+    {
+        const bool head = lane < 16;
+        const uint32_t l = head ? lane : 16 * c_end + (lane - 16);
+        const bool want = head ? (lo_off != 0 || hi < 16) : (c_end > 0 && (hi & 15u) != 0);
+        float v = 0.f;
+        uint32_t key = 0xFFFFFFFFu - lane;
+        float *y = nullptr;
+        if (want && l >= lo_off && l < hi) {
+            const uint32_t g = (uint32_t)(g0 + l);
+            const GemvMat &M = p.mats[gemv_matrix(p, g)];
+            const uint32_t rel = g - M.off, row = rel / M.cols, col = rel - row * M.cols;
+            const uint32_t wbits = merge1(smg[l], exp_s[l]);
+            v = bf16_lo(wbits) * bf16_lo(M.x[col]);
+            key = 2 * (M.rowbase + row) + (head ? 0u : 1u);
+            y = M.y + row;
+        }
+        add_runs(v, key, y, lane);
+    }
+}
+
 // C = segments per lane: the format block is 32 * C segments, one warp; lane
 // l decodes segments l, l + 32, ... as C independent chains.  WARPS warps per
 // CTA, one CTA per SM.
-template <int C, int WARPS>
+// MODE 0: store the BF16 outputs; MODE 1: fused matrix-vector product.
+template <int C, int WARPS, int MODE>
 __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params p)
 {
     static_assert(C == 1 || C == 2, "one or two chains per lane");
@@ -597,7 +725,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             // ---- merge with sign/mantissa (from L2)
             const uint32_t hi = lo_off + total;
             const uint8_t *smg = p.sm + g0;
-            if (p.wide) {
+            if (MODE == 1) {
+                gemv_block(p, g0, lo_off, hi, exp_s, lane);
+            } else if (p.wide) {
                 // 16 elements per lane and step, one 32-byte store: a warp's
                 // stores cover 1 KB contiguous
                 const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
@@ -659,7 +789,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 struct DeviceFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][4] = {};  // [C - 1][warps 32 / 24 / 16 / 8]
+    uint32_t granted[2][2][4] = {};  // [MODE][C - 1][warps 32 / 24 / 16 / 8]
 };
 std::mutex g_mu;
 DeviceFacts g_dev[64];
@@ -685,10 +815,10 @@ df11_status device_facts(DeviceFacts **out)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-template <int C, int WARPS>
+template <int C, int WARPS, int MODE>
 df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, DeviceFacts *f, uint32_t &granted)
 {
-    auto kern = df11_decode_kernel<C, WARPS>;
+    auto kern = df11_decode_kernel<C, WARPS, MODE>;
     if (smem > granted) {
         std::lock_guard<std::mutex> lock(g_mu);
         if (smem > granted) {
@@ -711,7 +841,7 @@ df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, 
 
 // As many warps per CTA (32, 24, 16 or 8) as the per-warp buffers allow in
 // shared memory; blocks of very short codes hold up to 64 outputs per segment.
-template <int C>
+template <int C, int MODE>
 df11_status launch(const Params &prm, cudaStream_t stream)
 {
     DeviceFacts *f = nullptr;
@@ -720,34 +850,33 @@ df11_status launch(const Params &prm, cudaStream_t stream)
         return st;
     const uint32_t optin = (uint32_t)f->smem_optin;
     if (Smem::bytes(prm.cap, 32) <= optin)
-        return launch_warps<C, 32>(prm, stream, Smem::bytes(prm.cap, 32), f, f->granted[C - 1][0]);
+        return launch_warps<C, 32, MODE>(prm, stream, Smem::bytes(prm.cap, 32), f, f->granted[MODE][C - 1][0]);
     if (Smem::bytes(prm.cap, 24) <= optin)
-        return launch_warps<C, 24>(prm, stream, Smem::bytes(prm.cap, 24), f, f->granted[C - 1][1]);
+        return launch_warps<C, 24, MODE>(prm, stream, Smem::bytes(prm.cap, 24), f, f->granted[MODE][C - 1][1]);
     if (Smem::bytes(prm.cap, 16) <= optin)
-        return launch_warps<C, 16>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[C - 1][2]);
+        return launch_warps<C, 16, MODE>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[MODE][C - 1][2]);
     if (Smem::bytes(prm.cap, 8) <= optin)
-        return launch_warps<C, 8>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[C - 1][3]);
+        return launch_warps<C, 8, MODE>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[MODE][C - 1][3]);
     return DF11_ERR_INVALID_ARG;
 }
 
 }  // namespace
 
 namespace {
-df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream,
-                            uint32_t max_sms)
+// Checks a stream's arrays (device pointers) and fills the launch fields they
+// determine.
+df11_status stream_params(const df11_arrays *a, uint32_t *status_dev, Params &prm)
 {
     if (!a || !status_dev)
         return DF11_ERR_INVALID_ARG;
-    if (a->n == 0)
-        return DF11_OK;
     const uint32_t T = a->threads_per_block;
     if (T != 32 && T != 64)
         return DF11_ERR_INVALID_ARG;
-    if (!dst || !a->encoded_exponent || !a->packed_sign_mantissa || !a->gaps || !a->block_offset || !a->luts ||
+    if (!a->encoded_exponent || !a->packed_sign_mantissa || !a->gaps || !a->block_offset || !a->luts ||
         !a->code_lengths)
         return DF11_ERR_INVALID_ARG;
-    if (!aligned(dst, 16) || !aligned(a->encoded_exponent, 16) || !aligned(a->packed_sign_mantissa, 16) ||
-        !aligned(a->gaps, 8) || !aligned(a->block_offset, 4))
+    if (!aligned(a->encoded_exponent, 16) || !aligned(a->packed_sign_mantissa, 16) || !aligned(a->gaps, 8) ||
+        !aligned(a->block_offset, 4))
         return DF11_ERR_INVALID_ARG;
     if (a->num_luts < 1 || a->num_luts > DF11_MAX_LUTS || a->n >= (1ull << 32))
         return DF11_ERR_INVALID_ARG;
@@ -759,15 +888,13 @@ df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *statu
         a->packed_sign_mantissa_bytes < ((a->n + 15) / 16) * 16 ||
         a->gaps_words < (5ull * a->num_blocks * T + 63) / 64 + 2 || a->max_block_elems > 64u * T)
         return DF11_ERR_INVALID_ARG;
-
-    Params prm;
+    std::memset(&prm, 0, sizeof(prm));
     prm.stream = a->encoded_exponent;
     prm.sm = a->packed_sign_mantissa;
     prm.gaps = reinterpret_cast<const uint32_t *>(a->gaps);
     prm.offs = a->block_offset;
     prm.luts = a->luts;
     prm.cl = a->code_lengths;
-    prm.dst = dst;
     prm.status = status_dev;
     prm.n = a->n;
     prm.total_bits = a->total_bits;
@@ -776,10 +903,27 @@ df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *statu
     prm.num_luts = a->num_luts;
     // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
     prm.cap = align16(a->max_block_elems + 32);
+    return DF11_OK;
+}
+
+df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream,
+                            uint32_t max_sms)
+{
+    if (!a || !status_dev)
+        return DF11_ERR_INVALID_ARG;
+    if (a->n == 0)
+        return DF11_OK;
+    if (!dst || !aligned(dst, 16))
+        return DF11_ERR_INVALID_ARG;
+    Params prm;
+    const df11_status st = stream_params(a, status_dev, prm);
+    if (st != DF11_OK)
+        return st;
+    prm.dst = dst;
     prm.wide = aligned(dst, 32) ? 1u : 0u;
     prm.max_ctas = max_sms;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return T == 32 ? launch<1>(prm, s) : launch<2>(prm, s);
+    return a->threads_per_block == 32 ? launch<1, 0>(prm, s) : launch<2, 0>(prm, s);
 }
 }  // namespace
 
@@ -847,4 +991,41 @@ extern "C" df11_status df11_read_status(const uint32_t *status_dev, void *stream
         cudaStreamSynchronize(s) != cudaSuccess)
         return DF11_ERR_CUDA;
     return v ? DF11_ERR_CORRUPT : DF11_OK;
+}
+
+extern "C" df11_status df11_decompress_gemv(const df11_arrays *a, const df11_gemv_matrix *mats, uint32_t num_mats,
+                                            uint32_t *status_dev, void *stream)
+{
+    if (!a || !status_dev || !mats || num_mats < 1 || num_mats > kMaxGemvMats)
+        return DF11_ERR_INVALID_ARG;
+    Params prm;
+    if (a->n == 0)
+        return DF11_ERR_INVALID_ARG;  // no matrix has zero elements
+    const df11_status st = stream_params(a, status_dev, prm);
+    if (st != DF11_OK)
+        return st;
+    uint64_t off = 0, rows = 0;
+    for (uint32_t m = 0; m < num_mats; m++) {
+        const df11_gemv_matrix &M = mats[m];
+        if (M.rows == 0 || M.cols == 0 || M.cols % 16 || !M.x || !M.y || !aligned(M.x, 16) || !aligned(M.y, 4))
+            return DF11_ERR_INVALID_ARG;
+        const uint64_t size = (uint64_t)M.rows * M.cols;
+        prm.mats[m].off = (uint32_t)off;
+        off += size;
+        if (off > a->n)
+            return DF11_ERR_INVALID_ARG;
+        prm.mats[m].end = (uint32_t)off;
+        prm.mats[m].cols = M.cols;
+        prm.mats[m].rowbase = (uint32_t)rows;
+        rows += M.rows;
+        if (rows >= (1ull << 30))
+            return DF11_ERR_INVALID_ARG;
+        prm.mats[m].x = M.x;
+        prm.mats[m].y = M.y;
+    }
+    if (off != a->n)
+        return DF11_ERR_INVALID_ARG;  // the matrices must cover the stream exactly
+    prm.num_mats = num_mats;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return a->threads_per_block == 32 ? launch<1, 1>(prm, s) : launch<2, 1>(prm, s);
 }

@@ -17,7 +17,9 @@ block) and orders the two streams with events:
 Every decode goes through ``df11_decompress`` (the CUDA kernel); this module
 only orders launches.  Run as a module it times one such pass with a
 stand-in consumer (the block's seven GEMMs against a batch of activations):
-``python -m huffman_decode_03_b200.pipeline --blocks 8 --batch 64``.
+``python -m huffman_decode_03_b200.pipeline --blocks 8 --batch 64``; with
+``--gemv`` it compares, at batch 1, decompress + cuBLAS matrix-vector
+products against the fused ``df11_decompress_gemv``.
 """
 from __future__ import annotations
 
@@ -168,6 +170,76 @@ def _bench(args):
     print(json.dumps(res))
 
 
+def _bench_gemv(args):
+    """Batch-1 use of each block: decompress, then the seven matrix-vector
+    products with cuBLAS, against df11_decompress_gemv (decode and product
+    in one pass, no BF16 weights written)."""
+    import numpy as np
+    import torch
+
+    from . import decompress_gemv
+
+    dev = torch.device("cuda")
+    shapes = [s for _, s in inputs.LLAMA3_8B]
+    fmts, dense = [], []
+    for b in range(args.blocks):
+        mats = [m for _, _, m in inputs.block(5, b)]
+        fmts.append(DeviceFormat(build_format(mats), dev))
+        dense.append(torch.from_numpy(np.concatenate(mats).view(np.int16)).to(dev).view(torch.bfloat16))
+    g = torch.Generator(device="cpu").manual_seed(11)
+    xs = [(torch.randn(c, generator=g)).to(torch.bfloat16).to(dev) for _, c in shapes]
+    ys = [torch.zeros(r, dtype=torch.float32, device=dev) for r, _ in shapes]
+    buf = torch.empty(max(f.n for f in fmts), dtype=torch.bfloat16, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def gemvs(w):
+        off, outs = 0, []
+        for (r, c), x in zip(shapes, xs):
+            outs.append(w[off:off + r * c].view(r, c) @ x)
+            off += r * c
+        return outs
+
+    def separate():
+        for f in fmts:
+            decompress(f, buf[:f.n], st)
+            gemvs(buf[:f.n])
+
+    def fused():
+        for y in ys:
+            y.zero_()
+        for f in fmts:
+            decompress_gemv(f, shapes, xs, ys, st)
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
+    nb = args.blocks
+    res = {"blocks": nb, "batch": 1, "block": "llama3_8b (q,k,v,o,gate,up,down)",
+           "decode_then_cublas_gemv_ms": timed(separate, args.reps),
+           "fused_decode_gemv_ms": timed(fused, args.reps),
+           "cublas_gemv_dense_ms": timed(lambda: [gemvs(w) for w in dense], args.reps)}
+    # the fused result of the last block against cuBLAS on the original weights
+    for y in ys:
+        y.zero_()
+    decompress_gemv(fmts[-1], shapes, xs, ys, st)
+    ref = gemvs(dense[-1])
+    torch.cuda.synchronize()
+    rel = max(float(((y - r.float()).abs().max() / r.float().abs().max()).item()) for y, r in zip(ys, ref))
+    res["max_rel_diff_vs_cublas_bf16_out"] = rel
+    res["per_block_us"] = {k[:-3]: round(1000 * v / nb, 1) for k, v in res.items() if k.endswith("_ms")}
+    print(json.dumps(res))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--blocks", type=int, default=8)
@@ -178,7 +250,12 @@ def main(argv=None):
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the uncompressed-weights GEMM baseline (saves device memory)")
     ap.add_argument("--no-check", dest="check", action="store_false")
+    ap.add_argument("--gemv", action="store_true",
+                    help="batch-1 comparison: decompress + cuBLAS matrix-vector products vs df11_decompress_gemv")
     args = ap.parse_args(argv)
+    if args.gemv:
+        _bench_gemv(args)
+        return
     if args.check and not args.dense:
         ap.error("--check needs the dense baseline")
     _bench(args)

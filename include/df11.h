@@ -178,6 +178,36 @@ df11_status df11_decompress(const df11_arrays *dev, uint16_t *dst,
 df11_status df11_decompress_sms(const df11_arrays *dev, uint16_t *dst,
                                 uint32_t *status_dev, void *stream, uint32_t max_sms);
 
+/* One matrix of df11_decompress_gemv: `rows` x `cols` BF16 weights, row-major,
+ * the next rows*cols elements of the stream (matrices in stream order). */
+typedef struct df11_gemv_matrix {
+    uint32_t rows;
+    uint32_t cols;       /* a multiple of 16 */
+    const uint16_t *x;   /* device: cols BF16 activations, 16-byte aligned */
+    float *y;            /* device: rows float32 outputs, 4-byte aligned */
+} df11_gemv_matrix;
+
+/*
+ * df11_decompress_gemv -- decode and use in one pass: y_m += W_m x_m for
+ * every matrix m of the stream, the BF16 weights W_m decoded on chip and
+ * never written to memory ("Dekompresi yang disesuaikan untuk inferensi
+ * GPU": weights are decompressed only to be multiplied, then discarded).
+ * The same decode as df11_decompress; each decoded weight is multiplied by
+ * its activation in float32 and the products of a row are summed per warp
+ * and added to y by atomic adds (so the summation order, and the last bits
+ * of y, vary between runs; the error is that of a float32 sum of the row's
+ * cols products).
+ *   dev       the stream's arrays (device pointers), as df11_decompress.
+ *   mats      host array of num_mats (1..16) matrices whose rows*cols add
+ *             up to dev->n; y is accumulated, not overwritten: zero it for
+ *             y = W x.
+ *   status_dev, stream: as df11_decompress.
+ * Asynchronous; DF11_ERR_INVALID_ARG for bad arguments (nothing launched),
+ * DF11_ERR_CUDA if the launch fails.
+ */
+df11_status df11_decompress_gemv(const df11_arrays *dev, const df11_gemv_matrix *mats, uint32_t num_mats,
+                                 uint32_t *status_dev, void *stream);
+
 /*
  * df11_decompress_host -- the same decode, starting and ending in host
  * memory: copies every array of *host (host pointers, ideally pinned) into

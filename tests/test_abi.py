@@ -41,8 +41,9 @@ def test_struct_sizes_match_c():
 #include <stddef.h>
 #include "df11.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu\n", sizeof(df11_arrays), offsetof(df11_arrays, encoded_exponent),
-         offsetof(df11_arrays, code_lengths), sizeof(df11_info), offsetof(df11_info, histogram));
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(df11_arrays), offsetof(df11_arrays, encoded_exponent),
+         offsetof(df11_arrays, code_lengths), sizeof(df11_info), offsetof(df11_info, histogram),
+         sizeof(df11_gemv_matrix), offsetof(df11_gemv_matrix, x), offsetof(df11_gemv_matrix, y));
   return 0;
 }
 '''
@@ -53,9 +54,9 @@ int main(void) {
         open(c, "w").write(src)
         subprocess.run(["gcc", "-I", HEADER_DIR, c, "-o", exe], check=True)
         got = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
-    A, I = df11.df11_arrays, df11.df11_info
+    A, I, G = df11.df11_arrays, df11.df11_info, df11.df11_gemv_matrix
     assert got == [ctypes.sizeof(A), A.encoded_exponent.offset, A.code_lengths.offset,
-                   ctypes.sizeof(I), I.histogram.offset]
+                   ctypes.sizeof(I), I.histogram.offset, ctypes.sizeof(G), G.x.offset, G.y.offset]
 
 
 def test_strerror_covers_all_codes():
