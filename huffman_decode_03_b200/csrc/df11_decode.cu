@@ -62,9 +62,11 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 namespace {
 
@@ -790,6 +792,7 @@ struct DeviceFacts {
     int sms = 0;
     int smem_optin = 0;
     uint32_t granted[2][2][4] = {};  // [MODE][C - 1][warps 32 / 24 / 16 / 8]
+    cudaStream_t up = nullptr, down = nullptr;  // copy streams of the host path, made on first use
 };
 std::mutex g_mu;
 DeviceFacts g_dev[64];
@@ -925,6 +928,36 @@ df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *statu
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return a->threads_per_block == 32 ? launch<1, 0>(prm, s) : launch<2, 0>(prm, s);
 }
+
+// Decodes format blocks [b0, b1) only: the stream, Gaps and BlockOffset
+// pointers move to block b0 (its Gap fields start on a 32-bit boundary: 5 * 32
+// and 5 * 64 bits per block); BlockOffset values, output and sign/mantissa
+// stay absolute.  A range that ends before the stream's last block counts one
+// segment more, so that its last chain ends at the next block's first Gap.
+df11_status decompress_blocks(const df11_arrays *a, uint32_t b0, uint32_t b1, uint16_t *dst, uint32_t *status_dev,
+                              cudaStream_t s)
+{
+    Params prm;
+    const df11_status st = stream_params(a, status_dev, prm);
+    if (st != DF11_OK)
+        return st;
+    if (b0 >= b1 || b1 > a->num_blocks)
+        return DF11_ERR_INVALID_ARG;
+    const uint64_t T = a->threads_per_block;
+    prm.stream += b0 * T * 8;
+    prm.gaps += (5 * T * b0) / 32;
+    prm.offs += b0;
+    prm.nblocks = b1 - b0;
+    if (b1 < a->num_blocks) {
+        prm.nseg = (uint64_t)(b1 - b0) * T + 1;
+    } else {
+        prm.nseg -= b0 * T;
+        prm.total_bits -= 64 * b0 * T;
+    }
+    prm.dst = dst;
+    prm.wide = aligned(dst, 32) ? 1u : 0u;
+    return T == 32 ? launch<1, 0>(prm, s) : launch<2, 0>(prm, s);
+}
 }  // namespace
 
 extern "C" df11_status df11_decompress(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream)
@@ -946,26 +979,12 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
     if (d->encoded_exponent_bytes < h->encoded_exponent_bytes ||
         d->packed_sign_mantissa_bytes < h->packed_sign_mantissa_bytes || d->gaps_words < h->gaps_words)
         return DF11_ERR_INVALID_ARG;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const cudaMemcpyKind k = cudaMemcpyHostToDevice;
-    struct Copy {
-        const void *src;
-        const void *dst;
-        size_t bytes;
-    } copies[] = {
-        {h->encoded_exponent, d->encoded_exponent, h->encoded_exponent_bytes},
-        {h->packed_sign_mantissa, d->packed_sign_mantissa, h->packed_sign_mantissa_bytes},
-        {h->gaps, d->gaps, h->gaps_words * 8},
-        {h->block_offset, d->block_offset, (h->num_blocks + 1) * 4ull},
-        {h->luts, d->luts, h->num_luts * 256ull},
-        {h->code_lengths, d->code_lengths, 256},
-    };
-    for (const Copy &c : copies) {
-        if (!c.src || !c.dst)
-            return DF11_ERR_INVALID_ARG;
-        if (cudaMemcpyAsync(const_cast<void *>(c.dst), c.src, c.bytes, k, s) != cudaSuccess)
-            return DF11_ERR_CUDA;
-    }
+    if (!h->encoded_exponent || !h->packed_sign_mantissa || !h->gaps || !h->block_offset || !h->luts ||
+        !h->code_lengths || !d->encoded_exponent || !d->packed_sign_mantissa || !d->gaps || !d->block_offset ||
+        !d->luts || !d->code_lengths)
+        return DF11_ERR_INVALID_ARG;
+    if (h->n == 0)
+        return DF11_OK;
     df11_arrays dev = *h;  // same sizes, device pointers
     dev.encoded_exponent = d->encoded_exponent;
     dev.packed_sign_mantissa = d->packed_sign_mantissa;
@@ -973,12 +992,97 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
     dev.block_offset = d->block_offset;
     dev.luts = d->luts;
     dev.code_lengths = d->code_lengths;
-    df11_status st = df11_decompress(&dev, dst_dev, status_dev, stream);
-    if (st != DF11_OK)
-        return st;
-    if (h->n && cudaMemcpyAsync(dst_host, dst_dev, h->n * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    {
+        Params check;  // the whole stream's arguments, before anything is queued
+        const df11_status st = stream_params(&dev, status_dev, check);
+        if (st != DF11_OK)
+            return st;
+        if (!aligned(dst_dev, 16))
+            return DF11_ERR_INVALID_ARG;
+    }
+    DeviceFacts *f = nullptr;
+    if (device_facts(&f) != DF11_OK)
         return DF11_ERR_CUDA;
-    return DF11_OK;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!f->up && cudaStreamCreateWithFlags(&f->up, cudaStreamNonBlocking) != cudaSuccess)
+            return DF11_ERR_CUDA;
+        if (!f->down && cudaStreamCreateWithFlags(&f->down, cudaStreamNonBlocking) != cudaSuccess)
+            return DF11_ERR_CUDA;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream), up = f->up, down = f->down;
+
+    // Pieces of whole format blocks, ~8 Mi outputs each: piece k's arrays go
+    // up on `up`, it decodes on `s`, its outputs come down on `down`, so the
+    // copies of one piece overlap the decode of its neighbours.
+    const uint32_t nb = h->num_blocks;
+    const uint64_t per_piece = 8ull << 20;
+    uint32_t pieces = (uint32_t)((h->n + per_piece - 1) / per_piece);
+    pieces = pieces < 1 ? 1 : pieces;
+    pieces = pieces > nb ? nb : pieces;
+    const uint32_t *offs = h->block_offset;
+    const uint64_t T = h->threads_per_block;
+    cudaEvent_t start, done;
+    std::vector<cudaEvent_t> evs;
+    auto event = [&](cudaEvent_t *e) {
+        if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess)
+            return false;
+        evs.push_back(*e);
+        return true;
+    };
+    auto cleanup = [&](df11_status st) {
+        for (cudaEvent_t e : evs)
+            cudaEventDestroy(e);  // released once their work completes
+        return st;
+    };
+    if (!event(&start) || !event(&done))
+        return cleanup(DF11_ERR_CUDA);
+    bool ok = cudaEventRecord(start, s) == cudaSuccess && cudaStreamWaitEvent(up, start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(down, start, 0) == cudaSuccess;
+    // the small arrays whole, first
+    ok = ok && cudaMemcpyAsync(const_cast<uint64_t *>(d->gaps), h->gaps, h->gaps_words * 8, cudaMemcpyHostToDevice,
+                               up) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(const_cast<uint32_t *>(d->block_offset), offs, (nb + 1) * 4ull,
+                               cudaMemcpyHostToDevice, up) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(const_cast<uint8_t *>(d->luts), h->luts, h->num_luts * 256ull, cudaMemcpyHostToDevice,
+                               up) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(const_cast<uint8_t *>(d->code_lengths), h->code_lengths, 256, cudaMemcpyHostToDevice,
+                               up) == cudaSuccess;
+    if (!ok)
+        return cleanup(DF11_ERR_CUDA);
+    for (uint32_t k = 0; k < pieces; k++) {
+        uint32_t b0 = (uint32_t)((uint64_t)nb * k / pieces), b1 = (uint32_t)((uint64_t)nb * (k + 1) / pieces);
+        if (b0 == b1)
+            continue;
+        // stream bytes of the blocks plus the 16 the last chain reads beyond
+        const uint64_t s0 = b0 * T * 8, s1 = std::min<uint64_t>(b1 * T * 8 + 16, h->encoded_exponent_bytes);
+        // sign/mantissa bytes of the outputs, in whole 16-byte units
+        const uint64_t m0 = offs[b0] & ~15ull;
+        const uint64_t m1 = std::min<uint64_t>((offs[b1] + 15ull) & ~15ull, h->packed_sign_mantissa_bytes);
+        cudaEvent_t in, dec;
+        if (!event(&in) || !event(&dec))
+            return cleanup(DF11_ERR_CUDA);
+        ok = cudaMemcpyAsync(const_cast<uint8_t *>(d->encoded_exponent) + s0, h->encoded_exponent + s0, s1 - s0,
+                             cudaMemcpyHostToDevice, up) == cudaSuccess;
+        ok = ok && (m1 <= m0 || cudaMemcpyAsync(const_cast<uint8_t *>(d->packed_sign_mantissa) + m0,
+                                                h->packed_sign_mantissa + m0, m1 - m0, cudaMemcpyHostToDevice,
+                                                up) == cudaSuccess);
+        ok = ok && cudaEventRecord(in, up) == cudaSuccess && cudaStreamWaitEvent(s, in, 0) == cudaSuccess;
+        if (!ok)
+            return cleanup(DF11_ERR_CUDA);
+        const df11_status st = decompress_blocks(&dev, b0, b1, dst_dev, status_dev, s);
+        if (st != DF11_OK)
+            return cleanup(st);
+        ok = cudaEventRecord(dec, s) == cudaSuccess && cudaStreamWaitEvent(down, dec, 0) == cudaSuccess;
+        const uint64_t e0 = offs[b0], e1 = offs[b1];
+        ok = ok && (e1 <= e0 || cudaMemcpyAsync(dst_host + e0, dst_dev + e0, (e1 - e0) * 2, cudaMemcpyDeviceToHost,
+                                                down) == cudaSuccess);
+        if (!ok)
+            return cleanup(DF11_ERR_CUDA);
+    }
+    // the caller's stream resumes after the last outputs have come down
+    ok = cudaEventRecord(done, down) == cudaSuccess && cudaStreamWaitEvent(s, done, 0) == cudaSuccess;
+    return cleanup(ok ? DF11_OK : DF11_ERR_CUDA);
 }
 
 extern "C" df11_status df11_read_status(const uint32_t *status_dev, void *stream)

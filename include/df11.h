@@ -214,7 +214,13 @@ df11_status df11_decompress_gemv(const df11_arrays *dev, const df11_gemv_matrix 
  * the device buffers named by *dev_buffers (device pointers with at least the
  * host sizes; they are overwritten although the struct's pointers are const),
  * runs df11_decompress into dst_dev, then copies the n outputs to dst_host.
- * All copies are cudaMemcpyAsync on `stream`; the call does not synchronise.
+ * The work goes in pieces of whole format blocks (about 8 Mi outputs each):
+ * a piece's arrays are copied up on one internal stream, it is decoded on
+ * `stream`, its outputs are copied down on a second internal stream, so that
+ * with pinned host memory the two copy directions and the decode overlap.
+ * The internal streams first wait for the work already queued on `stream`,
+ * and `stream` waits for the last copy: the call is stream-ordered on
+ * `stream` and does not synchronise.  BlockOffset is read on the host.
  */
 df11_status df11_decompress_host(const df11_arrays *host, const df11_arrays *dev_buffers,
                                  uint16_t *dst_dev, uint16_t *dst_host,

@@ -158,6 +158,27 @@ def test_sm_cap_gives_the_same_result(max_sms):
     assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), w)
 
 
+@pytest.mark.parametrize("n,T,kind", [(1, 64, "g"), (100_003, 64, "g"), (20_000_011, 64, "g"),
+                                      (20_000_011, 32, "g"), (9_000_001, 32, "stress")])
+def test_host_buffers_round_trip(n, T, kind):
+    # df11_decompress_host: pieces of whole blocks copied up, decoded and
+    # copied down on separate streams (one piece below 8 Mi outputs, three
+    # above 16 Mi); the device arrays start as garbage, so every byte the
+    # decode reads must have been uploaded
+    torch = torch_cuda()
+    w = inputs.gaussian(n, [27, n, T]) if kind == "g" else inputs.stress(n, key=(27, n, T))
+    dev = df11.DeviceFormat(df11.build_format(w, T), "cuda", pin_host=True)
+    for t in dev.tensors.values():
+        t.fill_(0xA5)
+    out_dev = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    host_out = torch.empty(n, dtype=torch.int16).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress_host(dev, out_dev, host_out, status)
+    assert df11.read_status(status) == 0
+    assert np.array_equal(host_out.numpy().view(np.uint16), w)
+    assert np.array_equal(out_dev.view(torch.int16).cpu().numpy().view(np.uint16), w)
+
+
 def test_repeated_launches_are_identical():
     torch = torch_cuda()
     w = inputs.gaussian(1 << 20, [25])
