@@ -42,7 +42,7 @@ constexpr uint32_t kPerThread = kChunk / kThreads;     // 32 consecutive element
 constexpr uint32_t kMaxChunkBits = kChunk * 32;        // codes are <= 32 bits
 constexpr uint32_t kBitWords = kMaxChunkBits / 32 + 2;  // + partial words at both ends
 constexpr uint32_t kMaxSegs = kMaxChunkBits / 64 + 3;
-constexpr uint32_t kGapWords = (5 * kMaxSegs) / 64 + 3;
+constexpr uint32_t kGapWords = (5 * kMaxSegs) / 32 + 3;  // 32-bit staging words
 static_assert(kPerThread == 32, "one warp-sized run of elements per thread");
 
 struct EncParams {
@@ -58,6 +58,7 @@ struct EncParams {
     uint64_t total_bits;
     uint64_t nseg;
     uint32_t T;
+    uint32_t t32_magic;  // ceil(2^32 / (T / 32)): umulhi(x, magic) = x / (T / 32) exactly for x < 2^26
     uint32_t nblocks;
     uint32_t nchunks;
     uint32_t code[256];  // canonical code, right-aligned
@@ -223,22 +224,36 @@ __global__ void __launch_bounds__(1024) chunk_scan_kernel(const EncParams p)
 }
 
 // Gap field of segment s (5 bits at bit 5 s of the packed words, LSB first)
-// into the chunk's staging words, which start at global word gw0.
-__device__ __forceinline__ void put_gap(unsigned long long *gbuf, uint64_t gw0, uint64_t s, uint32_t g)
+// into the chunk's 32-bit staging words, which start at global 32-bit word
+// gw0 (the uint64 Gaps words read as little-endian halves).
+__device__ __forceinline__ void put_gap(uint32_t *gbuf, uint64_t gw0, uint64_t s, uint32_t g)
 {
     const uint64_t bit = 5 * s;
-    const uint64_t w = bit / 64 - gw0;
-    const uint32_t sh = (uint32_t)(bit % 64);
-    atomicOr(&gbuf[w], (unsigned long long)(g & 31u) << sh);
-    if (sh > 59)
-        atomicOr(&gbuf[w + 1], (unsigned long long)(g & 31u) >> (64 - sh));
+    const uint32_t w = (uint32_t)(bit / 32 - gw0);
+    const uint32_t sh = (uint32_t)(bit % 32);
+    atomicOr(&gbuf[w], (g & 31u) << sh);
+    if (sh > 27)
+        atomicOr(&gbuf[w + 1], (g & 31u) >> (32 - sh));
+}
+
+// Segment s (< 2^31) starts a format block: s % T == 0, with T a multiple of
+// 32; *b gets s / T.
+__device__ __forceinline__ bool block_start(const EncParams &p, uint64_t s, uint32_t *b)
+{
+    const uint32_t s32 = (uint32_t)s;
+    if (s32 & 31u)
+        return false;
+    const uint32_t x = s32 >> 5, t32 = p.T >> 5;
+    const uint32_t q = t32 == 1 ? x : __umulhi(x, p.t32_magic);
+    *b = q;
+    return x - q * t32 == 0;
 }
 
 __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *bits = reinterpret_cast<uint32_t *>(smem);                                  // kBitWords
-    unsigned long long *gbuf = reinterpret_cast<unsigned long long *>(smem + kBitWords * 4);  // kGapWords
+    uint32_t *gbuf = reinterpret_cast<uint32_t *>(smem + kBitWords * 4);  // kGapWords
     __shared__ uint32_t s_code[256];
     __shared__ uint8_t s_len[256];
     __shared__ uint32_t warp_tot[kThreads / 32];
@@ -265,8 +280,8 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
     const uint64_t s_lo = lo ? prev_start / 64 + 1 : 0;
     const uint64_t last_start = E - s_len[exponent(p.w[hi - 1])];
     const uint64_t s_hi1 = hi == p.n ? p.nseg : last_start / 64 + 1;  // exclusive
-    const uint64_t gw0 = 5 * s_lo / 64;
-    const uint32_t ngw = s_hi1 > s_lo ? (uint32_t)((5 * (s_hi1 - 1) + 4) / 64 + 1 - gw0) : 0u;
+    const uint64_t gw0 = 5 * s_lo / 32;
+    const uint32_t ngw = s_hi1 > s_lo ? (uint32_t)((5 * (s_hi1 - 1) + 4) / 32 + 1 - gw0) : 0u;
     if (ngw > kGapWords) {
         if (threadIdx.x == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
@@ -300,12 +315,15 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
         const uint32_t l = s_len[e];
         if (l == 0)
             continue;  // reported by chunk_bits_kernel
-        // segment boundaries in (prev, pos]: this code is the first to start
-        // at or after them (codes are <= 32 bits: at most one boundary)
-        for (uint64_t s = have_prev ? prev / 64 + 1 : 0; s <= pos / 64 && s < p.nseg; s++) {
-            put_gap(gbuf, gw0, s, (uint32_t)(pos - 64 * s));
-            if (s % p.T == 0)
-                p.offs[s / p.T] = (uint32_t)(i0 + k);
+        // a code of <= 32 bits after the previous start: at most one segment
+        // boundary lies in (prev, pos], and then this code is the first to
+        // start in segment pos / 64, at Gap pos % 64
+        const uint64_t seg = pos >> 6;
+        if (!have_prev || (prev >> 6) != seg) {
+            put_gap(gbuf, gw0, seg, (uint32_t)(pos & 63));
+            uint32_t blk;
+            if (block_start(p, seg, &blk))
+                p.offs[blk] = (uint32_t)(i0 + k);
         }
         // the code, MSB first, into the chunk's big-endian bit words
         const uint64_t q = pos - 32 * wb0;
@@ -320,10 +338,11 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
     }
     if (cnt && i0 + cnt == p.n) {
         // the stream's last code: the segments after it end at total_bits
-        for (uint64_t s = prev / 64 + 1; s < p.nseg; s++) {
+        for (uint64_t s = prev / 64 + 1; s < p.nseg; s++) {  // at most one
             put_gap(gbuf, gw0, s, (uint32_t)(p.total_bits - 64 * s));
-            if (s % p.T == 0)
-                p.offs[s / p.T] = (uint32_t)p.n;
+            uint32_t blk;
+            if (block_start(p, s, &blk))
+                p.offs[blk] = (uint32_t)p.n;
         }
         p.offs[p.nblocks] = (uint32_t)p.n;
     }
@@ -354,11 +373,12 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
         else
             stream32[wb0 + j] = val;
     }
+    uint32_t *gaps32 = reinterpret_cast<uint32_t *>(p.gaps);
     for (uint32_t j = threadIdx.x; j < ngw; j += kThreads) {
         if (j == 0 || j + 1 == ngw)
-            atomicOr(reinterpret_cast<unsigned long long *>(&p.gaps[gw0 + j]), gbuf[j]);
+            atomicOr(&gaps32[gw0 + j], gbuf[j]);
         else
-            p.gaps[gw0 + j] = gbuf[j];
+            gaps32[gw0 + j] = gbuf[j];
     }
 }
 
@@ -479,6 +499,8 @@ extern "C" df11_status df11_device_encode(const df11_format *plan, const uint16_
     prm.total_bits = a.total_bits;
     prm.nseg = a.num_segments;
     prm.T = a.threads_per_block;
+    // T / 32 in 1..32; unused for 1 (its reciprocal does not fit 32 bits)
+    prm.t32_magic = prm.T == 32 ? 0u : (uint32_t)(((1ull << 32) + (prm.T / 32) - 1) / (prm.T / 32));
     prm.nblocks = a.num_blocks;
     prm.nchunks = (uint32_t)nchunks;
 
@@ -496,7 +518,7 @@ extern "C" df11_status df11_device_encode(const df11_format *plan, const uint16_
     if (!n)
         return cudaMemsetAsync(prm.offs, 0, 4, s) == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 
-    const size_t smem = kBitWords * 4 + kGapWords * 8;
+    const size_t smem = kBitWords * 4 + kGapWords * 4;
     chunk_bits_kernel<<<(unsigned)nchunks, kThreads, 0, s>>>(prm);
     chunk_scan_kernel<<<1, 1024, 0, s>>>(prm);
     encode_kernel<<<(unsigned)nchunks, kThreads, smem, s>>>(prm);

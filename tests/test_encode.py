@@ -136,6 +136,14 @@ def test_device_encode_matches_host(name, T):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("T", [96, 128, 256, 1024])
+def test_device_encode_other_block_sizes(T):
+    # the format allows any multiple of 32 (the decoder takes 32 or 64): the
+    # BlockOffset of every T-th segment must still land where the host puts it
+    _device_vs_host(inputs.gaussian(1_000_003, [88, T]), T)
+
+
+@pytest.mark.gpu
 def test_device_encode_length_limited_code():
     _device_vs_host(_fibonacci_bits())
 
