@@ -307,34 +307,57 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncParams p)
     uint64_t pos = B + toff;
     uint64_t prev = i0 ? pos - s_len[exponent(p.w[i0 - 1])] : 0;
     bool have_prev = i0 != 0;
-#pragma unroll
-    for (uint32_t k = 0; k < 32; k++) {
-        if (k >= cnt)
+    // four passes over 8 elements each (reloaded from L1): a loop body of 8
+    // elements, not 32, keeps the code within the instruction cache
+    for (uint32_t grp = 0; grp < 4; grp++) {
+        if (8 * grp >= cnt)
             break;
-        const uint32_t e = exponent(element(v, k));
-        const uint32_t l = s_len[e];
-        if (l == 0)
-            continue;  // reported by chunk_bits_kernel
-        // a code of <= 32 bits after the previous start: at most one segment
-        // boundary lies in (prev, pos], and then this code is the first to
-        // start in segment pos / 64, at Gap pos % 64
-        const uint64_t seg = pos >> 6;
-        if (!have_prev || (prev >> 6) != seg) {
-            put_gap(gbuf, gw0, seg, (uint32_t)(pos & 63));
-            uint32_t blk;
-            if (block_start(p, seg, &blk))
-                p.offs[blk] = (uint32_t)(i0 + k);
+        uint32_t g4[4];
+        if (8 * grp + 8 <= cnt) {
+            const uint4 q4 = __ldg(reinterpret_cast<const uint4 *>(p.w + i0) + grp);
+            g4[0] = q4.x;
+            g4[1] = q4.y;
+            g4[2] = q4.z;
+            g4[3] = q4.w;
+        } else {
+#pragma unroll
+            for (uint32_t j = 0; j < 4; j++) {
+                const uint32_t k0 = 8 * grp + 2 * j;
+                const uint32_t a = k0 < cnt ? (uint32_t)p.w[i0 + k0] : 0u;
+                const uint32_t b = k0 + 1 < cnt ? (uint32_t)p.w[i0 + k0 + 1] : 0u;
+                g4[j] = a | (b << 16);
+            }
         }
-        // the code, MSB first, into the chunk's big-endian bit words
-        const uint64_t q = pos - 32 * wb0;
-        const uint32_t o = (uint32_t)(q & 31);
-        const unsigned long long val = (unsigned long long)s_code[e] << (64 - o - l);
-        atomicOr(&bits[q >> 5], (uint32_t)(val >> 32));
-        if ((uint32_t)val)
-            atomicOr(&bits[(q >> 5) + 1], (uint32_t)val);
-        prev = pos;
-        have_prev = true;
-        pos += l;
+#pragma unroll
+        for (uint32_t j = 0; j < 8; j++) {
+            const uint32_t k = 8 * grp + j;
+            if (k >= cnt)
+                break;
+            const uint32_t e = exponent((j & 1u) ? (g4[j >> 1] >> 16) : (g4[j >> 1] & 0xFFFFu));
+            const uint32_t l = s_len[e];
+            if (l == 0)
+                continue;  // reported by chunk_bits_kernel
+            // a code of <= 32 bits after the previous start: at most one segment
+            // boundary lies in (prev, pos], and then this code is the first to
+            // start in segment pos / 64, at Gap pos % 64
+            const uint64_t seg = pos >> 6;
+            if (!have_prev || (prev >> 6) != seg) {
+                put_gap(gbuf, gw0, seg, (uint32_t)(pos & 63));
+                uint32_t blk;
+                if (block_start(p, seg, &blk))
+                    p.offs[blk] = (uint32_t)(i0 + k);
+            }
+            // the code, MSB first, into the chunk's big-endian bit words
+            const uint64_t q = pos - 32 * wb0;
+            const uint32_t o = (uint32_t)(q & 31);
+            const unsigned long long val = (unsigned long long)s_code[e] << (64 - o - l);
+            atomicOr(&bits[q >> 5], (uint32_t)(val >> 32));
+            if ((uint32_t)val)
+                atomicOr(&bits[(q >> 5) + 1], (uint32_t)val);
+            prev = pos;
+            have_prev = true;
+            pos += l;
+        }
     }
     if (cnt && i0 + cnt == p.n) {
         // the stream's last code: the segments after it end at total_bits
