@@ -1056,9 +1056,13 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
             continue;
         // stream bytes of the blocks plus the 16 the last chain reads beyond
         const uint64_t s0 = b0 * T * 8, s1 = std::min<uint64_t>(b1 * T * 8 + 16, h->encoded_exponent_bytes);
-        // sign/mantissa bytes of the outputs, in whole 16-byte units
-        const uint64_t m0 = offs[b0] & ~15ull;
-        const uint64_t m1 = std::min<uint64_t>((offs[b1] + 15ull) & ~15ull, h->packed_sign_mantissa_bytes);
+        // the piece's outputs: BlockOffset entries clamped to n, so that a
+        // corrupt host copy (which the kernel reports) cannot move a copy
+        // outside the arrays
+        const uint64_t e0 = std::min<uint64_t>(offs[b0], h->n), e1 = std::min<uint64_t>(offs[b1], h->n);
+        // their sign/mantissa bytes, in whole 16-byte units
+        const uint64_t m0 = e0 & ~15ull;
+        const uint64_t m1 = std::min<uint64_t>((e1 + 15ull) & ~15ull, h->packed_sign_mantissa_bytes);
         cudaEvent_t in, dec;
         if (!event(&in) || !event(&dec))
             return cleanup(DF11_ERR_CUDA);
@@ -1074,7 +1078,6 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
         if (st != DF11_OK)
             return cleanup(st);
         ok = cudaEventRecord(dec, s) == cudaSuccess && cudaStreamWaitEvent(down, dec, 0) == cudaSuccess;
-        const uint64_t e0 = offs[b0], e1 = offs[b1];
         ok = ok && (e1 <= e0 || cudaMemcpyAsync(dst_host + e0, dst_dev + e0, (e1 - e0) * 2, cudaMemcpyDeviceToHost,
                                                 down) == cudaSuccess);
         if (!ok)

@@ -179,6 +179,25 @@ def test_host_buffers_round_trip(n, T, kind):
     assert np.array_equal(out_dev.view(torch.int16).cpu().numpy().view(np.uint16), w)
 
 
+def test_host_buffers_with_corrupt_offsets_stay_in_bounds():
+    # a host BlockOffset entry past n: the kernel reports the block, and the
+    # host-side copy ranges (taken from that array) stay inside the buffers
+    torch = torch_cuda()
+    n = 9_000_001
+    w = inputs.gaussian(n, [28])
+    dev = df11.DeviceFormat(df11.build_format(w), "cuda", pin_host=True)
+    offs = dev.host_tensors["block_offset"].view(torch.int32)
+    k = offs.numel() // 2
+    offs[k] = n + 12_345
+    guard = 64
+    out_dev = torch.empty(n + guard, dtype=torch.bfloat16, device="cuda")
+    host = torch.full((n + guard,), 0x5A5A, dtype=torch.int16).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress_host(dev, out_dev, host[:n], status)
+    assert df11.read_status(status) != 0
+    assert torch.all(host[n:] == 0x5A5A)  # nothing written past n
+
+
 def test_repeated_launches_are_identical():
     torch = torch_cuda()
     w = inputs.gaussian(1 << 20, [25])
