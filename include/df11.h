@@ -11,9 +11,21 @@
  * hierarkis") and per-thread / per-block metadata ("Kernel GPU 2 tahap dan
  * metadata bantu").
  *
- * The library has two halves:
- *   - host: df11_build_format compresses BF16 matrices into the format;
- *   - device: df11_decompress rebuilds the BF16 matrix on a CUDA stream.
+ * Entry points, by the side they run on:
+ *   - host: df11_build_format compresses BF16 matrices into the format
+ *     (df11_format_arrays / df11_format_info read it back, df11_free drops
+ *     it); df11_plan_from_histogram builds only the code and the sizes from
+ *     256 exponent counts;
+ *   - device decode: df11_decompress rebuilds the BF16 matrix on a CUDA
+ *     stream (df11_decompress_sms on at most a given number of SMs);
+ *     df11_decompress_gemv decodes and multiplies by vectors without storing
+ *     the weights; df11_decompress_host takes the arrays in host memory and
+ *     overlaps the copies with the decode; df11_read_status reads the
+ *     kernels' error word;
+ *   - device encode: df11_device_histogram counts exponents of a device
+ *     array; df11_device_encode (caller scratch) and
+ *     df11_device_encode_static (library scratch) write the compressed
+ *     arrays of a plan into device buffers.
  * No entry point takes or returns framework types; all pointers are plain
  * host or device addresses as stated per argument.
  *
