@@ -22,7 +22,8 @@ from . import build as _build
 
 __all__ = [
     "Df11Error", "Format", "DeviceFormat", "build_format", "decompress",
-    "decompress_host", "read_status", "load_library",
+    "decompress_gemv", "decompress_gemm", "decompress_host", "encode_device", "read_status",
+    "tile_major", "load_library",
 ]
 
 DF11_OK = 0
@@ -30,6 +31,15 @@ DF11_ERR_CORRUPT = 6
 
 
 class df11_gemv_matrix(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_uint32),
+        ("cols", ctypes.c_uint32),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+class df11_gemm_matrix(ctypes.Structure):
     _fields_ = [
         ("rows", ctypes.c_uint32),
         ("cols", ctypes.c_uint32),
@@ -85,8 +95,8 @@ class df11_info(ctypes.Structure):
 
 EXPORTS = (
     "df11_build_format", "df11_format_arrays", "df11_format_info", "df11_free",
-    "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_gemv", "df11_decompress_host",
-    "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
+    "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_gemv", "df11_decompress_gemm",
+    "df11_gemm_scratch_bytes", "df11_tile_major", "df11_decompress_host", "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
     "df11_device_encode_scratch_words", "df11_device_encode", "df11_device_encode_static",
 )
 
@@ -121,6 +131,13 @@ def load_library(path: str | None = None):
     lib.df11_decompress_gemv.argtypes = [ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_gemv_matrix),
                                          ctypes.c_uint32, P, P]
     lib.df11_decompress_gemv.restype = ctypes.c_int
+    lib.df11_decompress_gemm.argtypes = [ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_gemm_matrix),
+                                         ctypes.c_uint32, ctypes.c_uint32, P, ctypes.c_uint64, P, P]
+    lib.df11_decompress_gemm.restype = ctypes.c_int
+    lib.df11_gemm_scratch_bytes.argtypes = [ctypes.POINTER(df11_gemm_matrix), ctypes.c_uint32, ctypes.c_uint32]
+    lib.df11_gemm_scratch_bytes.restype = ctypes.c_uint64
+    lib.df11_tile_major.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32, P]
+    lib.df11_tile_major.restype = ctypes.c_int
     lib.df11_decompress_host.argtypes = [
         ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_arrays), P, P, P, P]
     lib.df11_decompress_host.restype = ctypes.c_int
@@ -349,6 +366,72 @@ def decompress_gemv(dev: DeviceFormat, shapes, xs, ys, status=None, stream=None)
                                                ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
            "df11_decompress_gemv")
     return ys
+
+
+def tile_major(w, rows: int, cols: int) -> np.ndarray:
+    """The rows x cols row-major BF16 matrix ``w`` (uint16 bit patterns) in
+    the tile-major order ``decompress_gemm`` reads (df11_tile_major): 128 x 64
+    tiles, row tiles in order, within one the column tiles in order, within a
+    tile its rows.  Compress the result with ``build_format``."""
+    src = np.ascontiguousarray(np.asarray(w).view(np.uint16).reshape(-1))
+    if src.size != rows * cols:
+        raise ValueError(f"{src.size} elements for a {rows} x {cols} matrix")
+    dst = np.empty_like(src)
+    _check(load_library().df11_tile_major(src.ctypes.data, rows, cols, dst.ctypes.data), "df11_tile_major")
+    return dst
+
+
+def _gemm_mats(shapes, xs, ys, batch):
+    import torch
+
+    k = len(shapes)
+    if not (len(xs) == len(ys) == k):
+        raise ValueError("one activation matrix and one output matrix per weight matrix")
+    mats = (df11_gemm_matrix * max(k, 1))()
+    for m, ((rows, cols), x, y) in enumerate(zip(shapes, xs, ys)):
+        if x.dtype != torch.bfloat16 or y.dtype != torch.float32 or not (x.is_cuda and y.is_cuda):
+            raise ValueError("x must be CUDA bfloat16 and y CUDA float32")
+        if tuple(x.shape) != (batch, cols) or tuple(y.shape) != (batch, rows) or not (
+                x.is_contiguous() and y.is_contiguous()):
+            raise ValueError(f"matrix {m}: x must be ({batch}, {cols}) and y ({batch}, {rows}), contiguous")
+        mats[m].rows, mats[m].cols, mats[m].x, mats[m].y = rows, cols, x.data_ptr(), y.data_ptr()
+    return mats
+
+
+def decompress_gemm(dev: DeviceFormat, shapes, xs, ys, status=None, stream=None, scratch=None):
+    """Decode and multiply on the tensor cores (df11_decompress_gemm):
+    ``ys[m] += xs[m] @ W_m.T`` for the stream's matrices, of ``shapes[m] =
+    (rows, cols)`` in stream order, each stored tile-major (``tile_major``);
+    the decoded weights never reach memory.  ``xs[m]``: CUDA bfloat16
+    (batch, cols); ``ys[m]``: CUDA float32 (batch, rows), accumulated; batch
+    a multiple of 16 up to 256.  ``scratch``: a CUDA uint8 tensor of at least
+    ``gemm_scratch_bytes`` bytes (allocated when None).  Asynchronous; returns
+    ``ys``."""
+    import torch
+
+    batch = int(xs[0].shape[0]) if len(xs) else 0
+    mats = _gemm_mats(shapes, xs, ys, batch)
+    lib = load_library()
+    need = int(lib.df11_gemm_scratch_bytes(mats, len(shapes), batch))
+    if need == 0:
+        raise Df11Error(1, "df11_gemm_scratch_bytes")
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device=dev.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev.device)
+    _check(lib.df11_decompress_gemm(ctypes.byref(dev.c_arrays), mats, len(shapes), batch,
+                                    ctypes.c_void_p(scratch.data_ptr()), scratch.numel(),
+                                    ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
+           "df11_decompress_gemm")
+    return ys
+
+
+def gemm_scratch_bytes(shapes, batch: int) -> int:
+    """Scratch bytes ``decompress_gemm`` needs (0: invalid shapes or batch)."""
+    mats = (df11_gemm_matrix * max(len(shapes), 1))()
+    for m, (rows, cols) in enumerate(shapes):
+        mats[m].rows, mats[m].cols = rows, cols
+    return int(load_library().df11_gemm_scratch_bytes(mats, len(shapes), int(batch)))
 
 
 def decompress_host(dev: DeviceFormat, out_dev, out_host, status, stream=None):

@@ -1,6 +1,6 @@
 """Builds the in-tree shared library ``libdf11_b200.so`` with nvcc (sm_100a).
 
-The library holds the host format builder (C++) and the CUDA decoder; the
+The library holds the host format builder (C++) and the CUDA kernels; the
 CUDA runtime is linked statically so the library loads on machines without a
 GPU (host-only entry points work there) and carries no runtime-version clash
 with other CUDA users in the process.
@@ -17,8 +17,9 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libdf11_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
-SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_encode.cu"),
-           os.path.join(CSRC, "df11_format.cpp")]
+SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_gemm.cu"),
+           os.path.join(CSRC, "df11_encode.cu"), os.path.join(CSRC, "df11_format.cpp")]
+HEADERS = [os.path.join(INCLUDE, "df11.h"), os.path.join(CSRC, "df11_block.cuh")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -33,7 +34,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB_PATH):
         return True
     t = os.path.getmtime(LIB_PATH)
-    deps = SOURCES + [os.path.join(INCLUDE, "df11.h")]
+    deps = SOURCES + HEADERS
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -59,6 +59,7 @@
 //     block) can run beside the decode.
 // Every loop is bounded; inconsistent data sets a status word, never traps.
 #include "df11.h"
+#include "df11_block.cuh"
 
 #include <cuda_runtime.h>
 
@@ -69,16 +70,6 @@
 #include <vector>
 
 namespace {
-
-constexpr int kIdxBits = 12;  // index width of the derived table
-constexpr int kIdxEntries = 1 << kIdxBits;
-constexpr int kLutBytes = DF11_MAX_LUTS * 256;
-constexpr uint32_t kPointerBase = 240;
-constexpr uint32_t kSlotStride = 68;  // bytes per lane's staging slot (64 codes + 2 spill + 2)
-// per warp: two chains x 32 lanes, plus 32 bytes so that a chain of
-// inconsistent data (up to 95 one-bit codes + 2 spill bytes) stays inside the
-// warp's own slots; such a block is reported and writes nothing
-constexpr uint32_t kSlotBytes = 2 * 32 * kSlotStride + 32;
 
 // One matrix of a fused decode + matrix-vector product: rows x cols,
 // row-major, elements [off, end) of the stream; its rows are numbered
@@ -110,296 +101,6 @@ struct Params {
     uint32_t num_mats;  // fused matrix-vector product (MODE 1) only
     GemvMat mats[kMaxGemvMats];
 };
-
-__host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
-
-// Shared memory: tables at fixed offsets, then per warp: the exponent write
-// buffer and the chains' staging slots.
-struct Smem {
-    static constexpr uint32_t sym = 0;                       // uint32[4096]
-    static constexpr uint32_t luts = sym + kIdxEntries * 4;  // 17 * 256
-    static constexpr uint32_t cl = luts + kLutBytes;         // 256
-    static constexpr uint32_t zq = cl + 256;                 // uint8[16]
-    static constexpr uint32_t bufs = zq + 16;
-    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap) { return cap + kSlotBytes; }
-    __host__ __device__ static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * per_warp(cap); }
-};
-static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
-static_assert(kSlotBytes % 16 == 0, "slots keep the buffers 16-byte aligned");
-
-__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
-
-__device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
-
-// The page's hierarchical lookup: LUT 0 on the first 8 bits of the window,
-// pointer value 256 - j continues in LUT j on the next 8 bits.  Returns
-// symbol | length << 8; *bad on a dangling pointer.
-__device__ __forceinline__ uint32_t lut_decode(uint32_t win, const uint8_t *luts, const uint8_t *cl,
-                                               uint32_t num_luts, bool *bad)
-{
-    uint32_t e = luts[win >> 24];
-#pragma unroll
-    for (int lvl = 1; lvl <= 3; lvl++) {
-        if (e < kPointerBase)
-            break;
-        uint32_t j = 256u - e;
-        if (j >= num_luts) {
-            *bad = true;
-            return 32u << 8;
-        }
-        e = luts[j * 256u + ((win >> (24 - 8 * lvl)) & 0xFFu)];
-    }
-    if (e >= kPointerBase) {
-        *bad = true;
-        return 32u << 8;
-    }
-    return e | ((uint32_t)cl[e] << 8);
-}
-
-// 96-bit window h:m:l shifted left by c bits (0 <= c <= 32).
-__device__ __forceinline__ void shift_window(uint32_t &h, uint32_t &m, uint32_t &l, uint32_t c)
-{
-    h = __funnelshift_lc(m, h, c);
-    m = __funnelshift_lc(l, m, c);
-    l = __funnelshift_lc(0u, l, c);
-}
-
-// Four BF16 values from four sign/mantissa bytes S and four rotated exponent
-// bytes E (ror8(e) = e >> 1 | (e & 1) << 7):
-//   high byte = sign | e >> 1,  low byte = (e & 1) << 7 | mantissa.
-__device__ __forceinline__ void merge4(uint32_t S, uint32_t E, uint32_t &lo2, uint32_t &hi2)
-{
-    const uint32_t HB = (S & 0x80808080u) | (E & 0x7F7F7F7Fu);
-    const uint32_t LB = (E & 0x80808080u) | (S & 0x7F7F7F7Fu);
-    lo2 = __byte_perm(LB, HB, 0x5140);
-    hi2 = __byte_perm(LB, HB, 0x7362);
-}
-
-__device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
-{
-    return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
-}
-
-// Shared-memory accesses by 32-bit address.  They are volatile (kept in
-// program order with each other and with the PTX loops); the staging slots
-// and write buffers they touch are not accessed through C++ pointers.
-__device__ __forceinline__ void st_u8(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v));
-}
-
-__device__ __forceinline__ uint32_t ld_u8(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ uint32_t ld_u32(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void st_u32(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
-}
-
-// Decode loop for two chains (A, B) of one lane, in PTX.  Symbol-table
-// entry: up to three rotated exponents in bytes 0..2, their total length in
-// bits 24..28, their number in bits 29..30 (0 = a code longer than 12 bits).
-// A chain is active while pos < pend and its last entry was not 0; the bits
-// of its window past pend are zeros.  Per lookup: the three exponent bytes go
-// to the chain's staging slot at q unconditionally (bytes past the codes
-// found are overwritten by the next lookup or never read), q advances by the
-// count, the window and pos by the length.  (entry >> 24) serves as the
-// funnel-shift amount directly: wrap mode reads only its low five bits.  An
-// entry of 0 changes nothing and stops its chain: the caller resolves that
-// long code, resets the chain's entry to non-zero and calls again.
-__device__ __forceinline__ void decode_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA, int &posA,
-                                             uint32_t &eA, uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
-                                             int &posB, uint32_t &eB, int pendA, int pendB, uint32_t sym_base)
-{
-    asm volatile(
-        "{\n\t"
-        ".reg .pred pa, pb, pz;\n\t"
-        ".reg .u32 ca, cb, t;\n\t"
-        "DB_TOP:\n\t"
-        "setp.lt.s32 pa, %4, %12;\n\t"
-        "setp.lt.s32 pb, %10, %13;\n\t"
-        "setp.ne.and.u32 pa, %5, 0, pa;\n\t"
-        "setp.ne.and.u32 pb, %11, 0, pb;\n\t"
-        "or.pred pz, pa, pb;\n\t"
-        "@!pz bra DB_END;\n\t"
-        "@pa shr.u32 %5, %0, 20;\n\t"
-        "@pb shr.u32 %11, %6, 20;\n\t"
-        "@pa mad.lo.u32 %5, %5, 4, %14;\n\t"
-        "@pb mad.lo.u32 %11, %11, 4, %14;\n\t"
-        "@pa ld.shared.u32 %5, [%5];\n\t"
-        "@pb ld.shared.u32 %11, [%11];\n\t"
-        // chain A
-        "@pa st.shared.u8 [%3], %5;\n\t"
-        "@pa mul.hi.u32 t, %5, 16777216;\n\t"
-        "@pa st.shared.u8 [%3+1], t;\n\t"
-        "@pa mul.hi.u32 t, %5, 65536;\n\t"
-        "@pa st.shared.u8 [%3+2], t;\n\t"
-        "@pa shr.u32 ca, %5, 24;\n\t"
-        "@pa mul.hi.u32 t, %5, 8;\n\t"
-        "@pa add.u32 %3, %3, t;\n\t"
-        "@pa and.b32 t, ca, 31;\n\t"
-        "@pa add.s32 %4, %4, t;\n\t"
-        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
-        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
-        "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
-        // chain B
-        "@pb st.shared.u8 [%9], %11;\n\t"
-        "@pb mul.hi.u32 t, %11, 16777216;\n\t"
-        "@pb st.shared.u8 [%9+1], t;\n\t"
-        "@pb mul.hi.u32 t, %11, 65536;\n\t"
-        "@pb st.shared.u8 [%9+2], t;\n\t"
-        "@pb shr.u32 cb, %11, 24;\n\t"
-        "@pb mul.hi.u32 t, %11, 8;\n\t"
-        "@pb add.u32 %9, %9, t;\n\t"
-        "@pb and.b32 t, cb, 31;\n\t"
-        "@pb add.s32 %10, %10, t;\n\t"
-        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
-        "@pb shf.l.wrap.b32 %7, %8, %7, cb;\n\t"
-        "@pb shf.l.wrap.b32 %8, 0, %8, cb;\n\t"
-        "bra DB_TOP;\n\t"
-        "DB_END:\n\t"
-        "}"
-        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(eA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB),
-          "+r"(posB), "+r"(eB)
-        : "r"(pendA), "r"(pendB), "r"(sym_base)
-        : "memory");
-}
-
-// Registers one lane holds for one block: per chain its 12 stream bytes and
-// the Gaps words holding its field and the next one; the block's offsets.
-template <int C>
-struct BlockRegs {
-    uint2 s01[C];
-    uint32_t s2[C];
-    uint32_t g0[C], g1[C];
-    uint32_t o0, o1;
-};
-
-template <int C>
-__device__ __forceinline__ void load_block(const Params &p, uint32_t b, int lane, BlockRegs<C> &r)
-{
-#pragma unroll
-    for (int k = 0; k < C; k++) {
-        const uint64_t seg = (uint64_t)b * (32 * C) + lane + 32 * k;
-        const uint8_t *s = p.stream + 8 * seg;
-        r.s01[k] = __ldg(reinterpret_cast<const uint2 *>(s));
-        r.s2[k] = __ldg(reinterpret_cast<const uint32_t *>(s + 8));
-        const uint64_t w = (5 * seg) >> 5;
-        r.g0[k] = __ldg(p.gaps + w);
-        r.g1[k] = __ldg(p.gaps + w + 1);
-    }
-    r.o0 = __ldg(p.offs + b);
-    r.o1 = __ldg(p.offs + b + 1);
-}
-
-// Copies each of two chains' staging slots (shared address src[k], 4-byte
-// aligned, len[k] bytes) to the write buffer at shared address dst[k]: the up
-// to three bytes before dst's first word boundary and after its last one
-// singly (those words are shared with neighbouring chains), the words in
-// between as 32-bit stores assembled by funnel shifts; both chains step
-// through one loop.
-__device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32_t src0[2], const uint32_t len0[2])
-{
-    uint32_t dst[2], src[2], nw[2], sh[2], sa[2], cur[2], tail[2];
-#pragma unroll
-    for (int k = 0; k < 2; k++) {
-        uint32_t head = (4u - (dst0[k] & 3u)) & 3u;
-        head = head < len0[k] ? head : len0[k];
-#pragma unroll
-        for (uint32_t i = 0; i < 3; i++)
-            if (i < head)
-                st_u8(dst0[k] + i, ld_u8(src0[k] + i));
-        dst[k] = dst0[k] + head;
-        src[k] = src0[k] + head;
-        const uint32_t len = len0[k] - head;
-        nw[k] = len >> 2;
-        tail[k] = len & 3u;
-        sh[k] = 8u * (src[k] & 3u);
-        sa[k] = src[k] & ~3u;
-        cur[k] = ld_u32(sa[k]);
-    }
-    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
-    for (uint32_t w = 0; w < nmax; w++) {
-#pragma unroll
-        for (int k = 0; k < 2; k++) {
-            if (w < nw[k]) {
-                const uint32_t nxt = ld_u32(sa[k] + 4 * w + 4);
-                st_u32(dst[k] + 4 * w, __funnelshift_r(cur[k], nxt, sh[k]));
-                cur[k] = nxt;
-            }
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < 2; k++) {
-        const uint32_t o = 4 * nw[k];
-#pragma unroll
-        for (uint32_t i = 0; i < 3; i++)
-            if (i < tail[k])
-                st_u8(dst[k] + o + i, ld_u8(src[k] + o + i));
-    }
-}
-
-// Places every chain's staging slot in the write buffer with 32-bit stores
-// only; valid when every chain of the block holds >= 3 codes.  Chain c covers
-// bytes [s_c, s_c + cnt_c) of the buffer.  It writes the words from the one
-// holding s_c up to, not including, the word that holds its own last byte
-// (the next chain writes that one); the block's last chain also writes its
-// final partial word.  The bytes of a chain's first word that precede s_c are
-// the previous chain's last bytes: each chain reads its last four slot bytes
-// as one word and passes it on by shuffle.  src[k]: the chain's slot (4-byte
-// aligned shared address); s[k]: its byte offset in the buffer at shared
-// address exp_base.
-template <int C>
-__device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[2], const uint32_t src[2],
-                                            const uint32_t cnt[2], int lane)
-{
-    uint32_t last[2] = {0u, 0u}, prev[2] = {0u, 0u};
-#pragma unroll
-    for (int k = 0; k < C; k++) {
-        const uint32_t t = src[k] + cnt[k] - 4u;  // >= src[k] - 1: inside the shared buffers
-        const uint32_t a = t & ~3u;
-        last[k] = __funnelshift_r(ld_u32(a), ld_u32(a + 4), 8u * (t & 3u));
-        prev[k] = __shfl_up_sync(0xffffffffu, last[k], 1);
-    }
-    if (C == 2) {
-        // chain (lane 0, B) follows chain (lane 31, A)
-        const uint32_t x = __shfl_sync(0xffffffffu, last[0], 31);
-        if (lane == 0)
-            prev[1] = x;
-    }
-    uint32_t dst[2] = {0u, 0u}, sa[2] = {0u, 0u}, nw[2] = {0u, 0u}, sh[2] = {0u, 0u};
-#pragma unroll
-    for (int k = 0; k < C; k++) {
-        const uint32_t e = s[k] + cnt[k];
-        const bool final_chain = lane == 31 && k == C - 1;
-        dst[k] = exp_base + (s[k] & ~3u);
-        sa[k] = src[k];
-        nw[k] = (final_chain ? (e + 3u) >> 2 : e >> 2) - (s[k] >> 2);
-        sh[k] = 8u * (s[k] & 3u);
-    }
-    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
-    for (uint32_t w = 0; w < nmax; w++) {
-#pragma unroll
-        for (int k = 0; k < C; k++) {
-            if (w < nw[k]) {
-                const uint32_t cur = ld_u32(sa[k] + 4 * w);
-                st_u32(dst[k] + 4 * w, __funnelshift_l(prev[k], cur, sh[k]));
-                prev[k] = cur;
-            }
-        }
-    }
-}
 
 // Matrix of the fused product holding stream element g (matrices in order).
 __device__ __forceinline__ uint32_t gemv_matrix(const Params &p, uint32_t g)
@@ -524,12 +225,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 {
     static_assert(C == 1 || C == 2, "one or two chains per lane");
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
-    constexpr uint32_t T = 32 * C;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
-    uint8_t *luts = smem + Smem::luts;
-    uint8_t *cl = smem + Smem::cl;
-    uint8_t *zq = smem + Smem::zq;
+    const uint8_t *luts = smem + Smem::luts;
+    const uint8_t *cl = smem + Smem::cl;
+    const uint8_t *zq = smem + Smem::zq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
     uint8_t *slots = exp_s + p.cap;
@@ -541,55 +240,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (b < p.nblocks)
         load_block<C>(p, b, lane, cur);
 
-    // ---- once per CTA: the page's LUTs and CodeLengths, derived tables
-    const uint32_t lut_bytes = p.num_luts * 256u;
-    for (uint32_t i = tid; i < lut_bytes; i += kThreads)
-        luts[i] = p.luts[i];
-    for (uint32_t i = tid; i < 256; i += kThreads)
-        cl[i] = p.cl[i];
-    __syncthreads();
-    // first_code[i]: the first code of the 12-bit window i (bits past 12 taken
-    // as zeros): symbol | length << 8, or 0 when that code is longer than 12
-    // bits.  A code found in a zero-filled window is genuine when it ends
-    // inside the window (prefix property).  Scratch in the per-warp buffers,
-    // which are free until the blocks start.
-    uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
-    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
-        bool bad = false;
-        const uint32_t e = lut_decode(i << (32 - kIdxBits), luts, cl, p.num_luts, &bad);
-        const uint32_t len = e >> 8;
-        first_code[i] = (!bad && len >= 1 && len <= kIdxBits) ? (uint16_t)e : (uint16_t)0;
-    }
-    __syncthreads();
-    // Symbol table: the first three codes of each window, by three dependent
-    // first_code lookups.
-    for (uint32_t i = tid; i < kIdxEntries; i += kThreads) {
-        uint32_t syms = 0, bits = 0, n = 0;
-#pragma unroll
-        for (int j = 0; j < 3; j++) {
-            const uint32_t fc = first_code[(i << bits) & (kIdxEntries - 1)];
-            const uint32_t len = fc >> 8;
-            if (len != 0 && len + bits <= kIdxBits && n == (uint32_t)j) {
-                syms |= ror8(fc & 0xFFu) << (8 * j);
-                bits += len;
-                n++;
-            }
-        }
-        // exponents in bytes 0..2, total length in bits 24..28, count in 29..30
-        sym_tab[i] = syms | (bits << 24) | (n << 29);
-    }
-    if (tid < 16) {
-        // codes formed by d trailing zero bits, d = 0..15: the all-zero code
-        // (the canonical first code, of length lmin) repeated d / lmin times;
-        // bit 7 flags d as a multiple of lmin
-        bool bad = false;
-        const uint32_t lmin = lut_decode(0u, luts, cl, p.num_luts, &bad) >> 8;
-        const uint32_t d = (uint32_t)tid;
-        zq[tid] = (lmin >= 1 && !bad) ? (uint8_t)((d / lmin) | ((d % lmin == 0) << 7)) : (uint8_t)0;
-    }
-    __syncthreads();
+    build_tables(p.luts, p.cl, p.num_luts, smem, (uint32_t)tid, (uint32_t)kThreads);
 
-    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(sym_tab));
+    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * kSlotStride;
 
@@ -597,135 +250,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     for (; b < p.nblocks; b += stride) {
         if (b + stride < p.nblocks)
             load_block<C>(p, b + stride, lane, nxt);
-        const uint32_t o0 = cur.o0, o1 = cur.o1;
-        const uint32_t lo_off = o0 & 15u;
-        const uint64_t g0 = (uint64_t)o0 - lo_off;  // multiple of 16
-        const bool offs_ok = o1 >= o0 && (uint64_t)o1 <= p.n && (uint64_t)lo_off + (o1 - o0) + 16u <= p.cap;
-
-        // ---- the block's sign/mantissa bytes: into L2 now, read by the merge
-        const uint32_t nbytes = offs_ok ? align16(lo_off + (o1 - o0)) : 0u;
-        if (nbytes && lane == 0)
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + g0), "r"(nbytes) : "memory");
-
-        // ---- locate: chain k's codes start in [pos0, pend) of its window
-        bool bad = false;
-        int pos0[2] = {0, 0}, pend[2] = {0, 0};
-        uint32_t h[2] = {0u, 0u}, m[2] = {0u, 0u}, l[2] = {0u, 0u};
-#pragma unroll
-        for (int k = 0; k < C; k++) {
-            const uint64_t seg = (uint64_t)b * T + lane + 32 * k;
-            const uint32_t off = (uint32_t)((5 * seg) & 31);
-            const uint64_t v = (((uint64_t)cur.g1[k] << 32) | cur.g0[k]) >> off;
-            const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
-            if (seg < p.nseg) {
-                pos0[k] = (int)gap;
-                pend[k] = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
-            }
-            h[k] = bswap32(cur.s01[k].x);
-            m[k] = bswap32(cur.s01[k].y);
-            l[k] = bswap32(cur.s2[k]);
-            // bits from pend on belong to the next chain: zeros instead
-            const uint32_t pe = (uint32_t)pend[k];
-            h[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe);
-            m[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 32u ? pe - 32u : 0u);
-            l[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 64u ? pe - 64u : 0u);
-            shift_window(h[k], m[k], l[k], (uint32_t)pos0[k]);
-        }
-
-        // ---- decode each chain once into its staging slot.  Past pend the
-        // window reads zeros, which decode as the all-zero code (the
-        // canonical first code, of length lmin); the last lookup of a chain
-        // starts on one of its own codes, so at most its two further codes
-        // are such zero codes: pos overshoots pend by a multiple of lmin
-        // (< 12) and the count by overshoot / lmin.
-        uint32_t cnt[2];
-        {
-            uint32_t q[2], q0[2], e[2] = {1u, 1u};
-            int pos[2];
-#pragma unroll
-            for (int k = 0; k < 2; k++) {
-                q0[k] = slot_base + k * (32 * kSlotStride);
-                q[k] = q0[k];
-                pos[k] = pos0[k];
-            }
-            for (;;) {  // each pass resolves >= 1 code or ends both chains
-                decode_bulk2(h[0], m[0], l[0], q[0], pos[0], e[0], h[1], m[1], l[1], q[1], pos[1], e[1], pend[0],
-                             pend[1], sym_base);
-                bool any_long = false;
-#pragma unroll
-                for (int k = 0; k < 2; k++) {
-                    if (pos[k] < pend[k]) {
-                        // stopped on a code longer than 12 bits: the page's LUTs
-                        const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
-                        const uint32_t len = (d >> 8) ? (d >> 8) : 1u;
-                        st_u8(q[k], ror8(d & 0xFFu));
-                        q[k] += 1;
-                        pos[k] += (int)len;
-                        shift_window(h[k], m[k], l[k], len);
-                        e[k] = 1u;
-                        any_long = true;
-                    }
-                }
-                if (!any_long)
-                    break;
-            }
-#pragma unroll
-            for (int k = 0; k < 2; k++) {
-                const uint32_t d = (uint32_t)(pos[k] - pend[k]);  // >= 0
-                const uint32_t z = zq[d & 15u];
-                bad |= d > 15u || !(z & 0x80u);
-                cnt[k] = q[k] - q0[k] - (z & 0x7Fu);
-            }
-        }
-
-        // ---- warp prefix sum of the counts; both chains in one packed scan
-        // (a chain holds at most 64 codes, a block at most 2048 per chain)
-        uint32_t packed = 0;
-#pragma unroll
-        for (int k = 0; k < C; k++)
-            packed |= (cnt[k] & 0xFFFFu) << (16 * k);
-        uint32_t incl = packed;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d)
-                incl += y;
-        }
-        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-        uint32_t first[2] = {0u, 0u};
-        uint32_t total = 0;
-#pragma unroll
-        for (int k = 0; k < C; k++) {
-            first[k] = total + ((incl >> (16 * k)) & 0xFFFFu) - cnt[k];
-            total += (tot >> (16 * k)) & 0xFFFFu;
-            bad |= cnt[k] > 64u;
-        }
-        const bool block_bad = __any_sync(0xffffffffu, bad) || !offs_ok || total != o1 - o0;
-        if (block_bad) {
-            if (lane == 0)
-                atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
-            __syncwarp();
-        } else {
-            // ---- place: each chain's slot into the write buffer; whole words
-            // when every chain holds >= 3 codes (the normal case), else
-            // with single bytes at the chains' edges
-            {
-                const uint32_t srcs[2] = {slot_base, slot_base + 32 * kSlotStride};
-                bool short_chain = cnt[0] < 3u;
-                if (C == 2)
-                    short_chain |= cnt[1] < 3u;
-                if (!__any_sync(0xffffffffu, short_chain)) {
-                    const uint32_t offs2[2] = {lo_off + first[0], lo_off + first[1]};
-                    place_words<C>(exp_base, offs2, srcs, cnt, lane);
-                } else {
-                    const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
-                    copy_slots2(dsts, srcs, cnt);
-                }
-            }
-            __syncwarp();
-
+        BlockOut bo;
+        if (decode_block<C>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
             // ---- merge with sign/mantissa (from L2)
-            const uint32_t hi = lo_off + total;
+            const uint64_t g0 = bo.g0;
+            const uint32_t lo_off = bo.lo_off, hi = bo.hi;
             const uint8_t *smg = p.sm + g0;
             if (MODE == 1) {
                 gemv_block(p, g0, lo_off, hi, exp_s, lane);
@@ -816,8 +345,6 @@ df11_status device_facts(DeviceFacts **out)
     return DF11_OK;
 }
 
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
 template <int C, int WARPS, int MODE>
 df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, DeviceFacts *f, uint32_t &granted)
 {
@@ -866,49 +393,6 @@ df11_status launch(const Params &prm, cudaStream_t stream)
 }  // namespace
 
 namespace {
-// Checks a stream's arrays (device pointers) and fills the launch fields they
-// determine.
-df11_status stream_params(const df11_arrays *a, uint32_t *status_dev, Params &prm)
-{
-    if (!a || !status_dev)
-        return DF11_ERR_INVALID_ARG;
-    const uint32_t T = a->threads_per_block;
-    if (T != 32 && T != 64)
-        return DF11_ERR_INVALID_ARG;
-    if (!a->encoded_exponent || !a->packed_sign_mantissa || !a->gaps || !a->block_offset || !a->luts ||
-        !a->code_lengths)
-        return DF11_ERR_INVALID_ARG;
-    if (!aligned(a->encoded_exponent, 16) || !aligned(a->packed_sign_mantissa, 16) || !aligned(a->gaps, 8) ||
-        !aligned(a->block_offset, 4))
-        return DF11_ERR_INVALID_ARG;
-    if (a->num_luts < 1 || a->num_luts > DF11_MAX_LUTS || a->n >= (1ull << 32))
-        return DF11_ERR_INVALID_ARG;
-    const uint64_t nseg = (a->total_bits + 63) / 64;
-    if (nseg != a->num_segments || (nseg + T - 1) / T != a->num_blocks || a->num_blocks == 0)
-        return DF11_ERR_INVALID_ARG;
-    // every load stays inside its array
-    if (a->encoded_exponent_bytes < (uint64_t)a->num_blocks * T * 8 + 16 ||
-        a->packed_sign_mantissa_bytes < ((a->n + 15) / 16) * 16 ||
-        a->gaps_words < (5ull * a->num_blocks * T + 63) / 64 + 2 || a->max_block_elems > 64u * T)
-        return DF11_ERR_INVALID_ARG;
-    std::memset(&prm, 0, sizeof(prm));
-    prm.stream = a->encoded_exponent;
-    prm.sm = a->packed_sign_mantissa;
-    prm.gaps = reinterpret_cast<const uint32_t *>(a->gaps);
-    prm.offs = a->block_offset;
-    prm.luts = a->luts;
-    prm.cl = a->code_lengths;
-    prm.status = status_dev;
-    prm.n = a->n;
-    prm.total_bits = a->total_bits;
-    prm.nseg = nseg;
-    prm.nblocks = a->num_blocks;
-    prm.num_luts = a->num_luts;
-    // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
-    prm.cap = align16(a->max_block_elems + 32);
-    return DF11_OK;
-}
-
 df11_status decompress_impl(const df11_arrays *a, uint16_t *dst, uint32_t *status_dev, void *stream,
                             uint32_t max_sms)
 {

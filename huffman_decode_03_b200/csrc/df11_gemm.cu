@@ -1,0 +1,731 @@
+// df11_gemm.cu -- sm_100a: DF11 weights decoded straight into tensor-core
+// operand tiles and multiplied by a batch of activation vectors
+// (tcgen05.mma, float32 accumulators in tensor memory).  The BF16 weights
+// never exist in global memory.
+//
+// "DFloat11: Kompresi inferensi GPU lossless ..." (id.news.hada.io/topic?id=20542),
+// "Dekompresi yang disesuaikan untuk inferensi GPU": weights are decompressed
+// right before the matrix multiplication that uses them and discarded after
+// it; the page's discussion proposes a GEMM that decompresses each tile just
+// before its arithmetic.  This is that GEMM: Y_m += X_m W_m^T for every matrix
+// m of a stream, X_m holding `batch` activation vectors of cols_m elements.
+//
+// Element order.  A DF11 stream is one run of elements whose order the page
+// leaves to the compressor.  Here each matrix is stored in 128 x 64 tiles:
+// its row tiles (128 rows) in order, within a row tile its column tiles (64
+// columns) in order, within a tile its 128 rows of 64 elements
+// (df11_tile_major writes this order).  So 8192 consecutive stream elements
+// are one A operand tile of the MMA (M = 128 rows, K = 64), and the K chunks
+// of a row tile follow one another.
+//
+// Work unit: up to 16 consecutive K chunks of one row tile of one matrix.  A
+// prep kernel packs every 64-column chunk of X into the shared-memory image
+// the tensor core reads and finds each unit's first and last format block.
+// Then one persistent CTA per SM takes units blockIdx.x, + gridDim.x, ...:
+//   * 16 decode warps: warp w decodes the unit's format blocks w, w + 16, ...
+//     with the per-block decode shared with the other kernels, merges each
+//     exponent with its sign/mantissa byte and stores the BF16 weight at its
+//     place in a ring of S operand tiles in shared memory (K-major, 128-byte
+//     swizzle).  A warp arrives on a tile's "full" barrier as soon as its next
+//     block starts past that tile;
+//   * 1 control warp: allocates tensor memory; one of its threads copies each
+//     K chunk of X into the ring by a bulk copy (cp.async.bulk, no tensor
+//     map), waits for the tile to be full, issues four tcgen05.mma (K = 16
+//     each) into the unit's accumulator and frees the ring slot with
+//     tcgen05.commit;
+//   * 4 epilogue warps: read the 128 x batch float32 accumulator with
+//     tcgen05.ld and add it into Y by atomic adds (the units of one row tile
+//     share its rows).  Two accumulators let the next unit's MMAs start while
+//     the last one is read out.
+// Every wait on a barrier is bounded.  When one runs out, the kernel sets bit
+// 31 of the status word and an abort flag on which every role stops, waits
+// (bounded) for its own copies and MMAs in flight, frees its tensor memory and
+// ends.  Inconsistent data sets DF11_ERR_CORRUPT as in the other kernels; a
+// unit whose tiles did not receive exactly their elements is reported too.
+#include "df11.h"
+#include "df11_block.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+namespace {
+
+constexpr uint32_t kTileRows = 128, kTileCols = 64;
+constexpr uint32_t kTileElems = kTileRows * kTileCols;  // 8192
+constexpr uint32_t kTileShift = 13;
+constexpr uint32_t kTileBytes = kTileElems * 2;          // 16 KB
+constexpr uint32_t kDecodeWarps = 16;
+constexpr uint32_t kControlWarp = kDecodeWarps;  // then 4 epilogue warps
+constexpr uint32_t kGemmThreads = (kDecodeWarps + 1 + 4) * 32;
+constexpr uint32_t kMaxStages = 8;
+constexpr uint32_t kUnitChunks = 16;  // K chunks per work unit, at most
+constexpr uint32_t kMaxGemmMats = 16;
+constexpr uint32_t kCoverSlots = 16;  // > kMaxStages + 2 units in flight
+constexpr uint32_t kSpinLimit = 1u << 20;
+constexpr uint32_t kTimeoutFlag = 0x80000000u;
+
+// Barrier and flag area after the decode warps' buffers: full[8], empty[8],
+// xfull[8], accf[2], tfree[2], drain (8 bytes each), then the tensor-memory
+// address, the abort flag and the coverage counters.
+constexpr uint32_t kBarFull = 0, kBarEmpty = 8, kBarX = 16, kBarAcc = 24, kBarFree = 26, kBarDrain = 28;
+constexpr uint32_t kNumBars = 29;
+constexpr uint32_t kCtrlBytes = 512;
+static_assert(kNumBars * 8 + 8 + 4 * kCoverSlots <= kCtrlBytes, "control area");
+
+struct GemmMat {
+    uint32_t off;           // first stream element
+    uint32_t rows, cols;    // multiples of 128 and 64
+    uint32_t unit0;         // its first work unit
+    uint32_t units_per_rt;  // work units per row tile
+    uint32_t piece0;        // its first 16-byte piece of X (packing)
+    uint64_t xoff;          // byte offset of its packed X
+    const uint16_t *x;      // batch x cols BF16, row-major
+    float *y;               // batch x rows float32, row-major
+};
+
+struct GemmParams {
+    // the stream: the fields the shared per-block decode reads
+    const uint8_t *stream;
+    const uint8_t *sm;
+    const uint32_t *gaps;
+    const uint32_t *offs;
+    const uint8_t *luts;
+    const uint8_t *cl;
+    uint32_t *status;
+    uint64_t n;
+    uint64_t total_bits;
+    uint64_t nseg;
+    uint32_t nblocks;
+    uint32_t num_luts;
+    uint32_t cap;
+    // the product
+    uint32_t batch;      // N of the MMA
+    uint32_t stages;     // S, operand tiles in the ring
+    uint32_t tmem_cols;  // power of two >= 2 * batch
+    uint32_t num_mats;
+    uint32_t num_units;
+    uint32_t num_pieces;
+    uint8_t *xpack;           // packed X of every matrix
+    uint32_t *unit_blocks;    // per unit: first block, end block (exclusive)
+    GemmMat mats[kMaxGemmMats];
+};
+
+__host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap)
+{
+    return align16(Smem::bufs + kDecodeWarps * Smem::per_warp(cap));
+}
+
+// Dynamic shared memory of a launch: tables, decode buffers, control area,
+// 1 KB to align the ring, the ring.
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages)
+{
+    return ctrl_offset(cap) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: BF16 A and B, both
+// K-major, float32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t m, uint32_t n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzled layout: rows of 64 BF16 (128 bytes) at a 128-byte pitch, groups of
+// 8 rows 1024 bytes apart; saddr 1024-byte aligned (K step k adds 32 k bytes).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Byte offset of element i (row-major 128 x 64) of an operand tile in that
+// layout: the 16-byte group of 8 columns is XORed with the row mod 8.
+__device__ __forceinline__ uint32_t tile_offset(uint32_t i)
+{
+    const uint32_t r = i >> 6, c = i & 63u;
+    return (r << 7) + ((((c >> 3) ^ r) & 7u) << 4) + ((c & 7u) << 1);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits until the barrier's phase of the given parity has completed.  Gives
+// up (false) when the kernel is aborting, or after kSpinLimit polls, which
+// starts the abort.  With honour_abort false it keeps waiting during an abort
+// (used to drain the kernel's own copies and MMAs).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
+                                          uint32_t *status, bool honour_abort = true)
+{
+    for (uint32_t i = 0; i < kSpinLimit; i++) {
+        if (mbar_try(bar, parity))
+            return true;
+        if (honour_abort && *abort_flag)
+            return false;
+    }
+    *abort_flag = 1u;
+    atomicOr(status, kTimeoutFlag);
+    return false;
+}
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((uint16_t)v) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives on the barrier once every tcgen05 operation this thread issued
+// before has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive float32 columns of tensor memory.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Work unit u: its matrix, first row, first K chunk, number of K chunks and
+// first stream element.
+struct Unit {
+    uint32_t m, row0, kc0, ntiles, e0;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmParams &p, uint32_t u)
+{
+    uint32_t m = 0;
+    while (m + 1 < p.num_mats && u >= p.mats[m + 1].unit0)
+        m++;
+    const GemmMat &M = p.mats[m];
+    const uint32_t rel = u - M.unit0, rt = rel / M.units_per_rt, ku = rel - rt * M.units_per_rt;
+    const uint32_t kchunks = M.cols / kTileCols, kc0 = ku * kUnitChunks;
+    Unit U;
+    U.m = m;
+    U.row0 = rt * kTileRows;
+    U.kc0 = kc0;
+    U.ntiles = kchunks - kc0 < kUnitChunks ? kchunks - kc0 : kUnitChunks;
+    U.e0 = M.off + (rt * kchunks + kc0) * kTileElems;
+    return U;
+}
+
+// Largest block b < nblocks with offs[b] <= x (offs[0] = 0).
+__device__ __forceinline__ uint32_t block_of(const uint32_t *offs, uint32_t nblocks, uint32_t x)
+{
+    uint32_t lo = 0, hi = nblocks - 1;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (__ldg(offs + mid) <= x)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Packs X (one thread per 16-byte piece: 8 activations of one vector) into
+// the operand image of each K chunk, and finds each unit's blocks.
+__global__ void gemm_prep_kernel(const GemmParams p)
+{
+    const uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g < p.num_pieces) {
+        uint32_t m = 0;
+        while (m + 1 < p.num_mats && g >= p.mats[m + 1].piece0)
+            m++;
+        const GemmMat &M = p.mats[m];
+        const uint32_t per_vec = M.cols / 8, idx = g - M.piece0;
+        const uint32_t v = idx / per_vec, j8 = idx - v * per_vec, kc = j8 >> 3, j = j8 & 7u;
+        const uint4 d = __ldg(reinterpret_cast<const uint4 *>(M.x + (uint64_t)v * M.cols + 8 * j8));
+        uint8_t *dst = p.xpack + M.xoff + (uint64_t)kc * p.batch * 128 + v * 128 + (((j ^ v) & 7u) << 4);
+        *reinterpret_cast<uint4 *>(dst) = d;
+    }
+    if (g < p.num_units) {
+        const Unit U = unit_of(p, g);
+        const uint32_t e1 = U.e0 + U.ntiles * kTileElems;
+        p.unit_blocks[2 * g] = block_of(p.offs, p.nblocks, U.e0);
+        p.unit_blocks[2 * g + 1] = block_of(p.offs, p.nblocks, e1 - 1) + 1;
+    }
+}
+
+struct Roles {
+    uint32_t ring_a, ring_b, bars;  // shared addresses
+    volatile uint32_t *abort_flag;
+    uint32_t *cover;
+    uint32_t tmem;
+};
+
+__device__ __forceinline__ uint32_t bar(const Roles &R, uint32_t i) { return R.bars + 8 * i; }
+
+// Decode warp: every unit of the CTA, blocks warp, warp + 16, ... of it.
+template <int C>
+__device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R, uint8_t *smem, uint32_t warp,
+                                            int lane)
+{
+    const uint32_t S = p.stages;
+    uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
+    const uint8_t *luts = smem + Smem::luts;
+    const uint8_t *cl = smem + Smem::cl;
+    const uint8_t *zq = smem + Smem::zq;
+    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
+    const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
+    const uint32_t slot_base =
+        static_cast<uint32_t>(__cvta_generic_to_shared(exp_s + p.cap)) + (uint32_t)lane * kSlotStride;
+
+    uint32_t q0 = 0, k = 0;  // tile sequence number of the unit's first tile; unit count
+    // waits until tile q's ring slot is free (the MMA of tile q - S is done)
+    auto slot_free = [&](uint32_t q) -> bool {
+        if (q < S)
+            return true;
+        return __all_sync(0xffffffffu, mbar_wait(bar(R, kBarEmpty + q % S), (q / S - 1) & 1u, R.abort_flag, p.status));
+    };
+    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
+        if (*R.abort_flag)
+            return;
+        const Unit U = unit_of(p, u);
+        const uint64_t e0 = U.e0, e1 = e0 + (uint64_t)U.ntiles * kTileElems;
+        const uint32_t bb = p.unit_blocks[2 * u], be = p.unit_blocks[2 * u + 1];
+        uint32_t arrived = 0;
+        bool ok = true;
+        BlockRegs<C> cur, nxt;
+        uint32_t b = bb + warp;
+        if (b < be)
+            load_block<C>(p, b, lane, cur);
+        for (; b < be && ok; b += kDecodeWarps) {
+            const bool more = b + kDecodeWarps < be;
+            if (more)
+                load_block<C>(p, b + kDecodeWarps, lane, nxt);
+            BlockOut bo;
+            if (decode_block<C>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
+                // the block's outputs inside the unit: [lo, hi) relative to g0
+                const uint64_t g0 = bo.g0;
+                const uint32_t lo = (uint32_t)(g0 + bo.lo_off < e0 ? e0 - g0 : bo.lo_off);
+                const uint32_t hi = (uint32_t)(g0 + bo.hi > e1 ? e1 - g0 : bo.hi);
+                if (lo < hi) {
+                    const uint32_t t_first = (uint32_t)((g0 + lo - e0) >> kTileShift);
+                    const uint32_t t_last = (uint32_t)((g0 + hi - 1 - e0) >> kTileShift);
+                    for (uint32_t t = t_first; t <= t_last && ok; t++)
+                        ok = slot_free(q0 + t);
+                    if (!ok)
+                        break;
+                    const uint32_t sa0 = R.ring_a + ((q0 + t_first) % S) * kTileBytes;
+                    const uint32_t sa1 = R.ring_a + ((q0 + t_first + 1) % S) * kTileBytes;
+                    const uint8_t *smg = p.sm + g0;
+                    auto addr = [&](uint32_t l) {
+                        const uint32_t v = (uint32_t)(g0 + l - e0);
+                        return ((v >> kTileShift) == t_first ? sa0 : sa1) + tile_offset(v & (kTileElems - 1));
+                    };
+                    // whole groups of 8 (16 bytes of the tile) ...
+                    const uint32_t c_lo = (lo + 7u) & ~7u, c_hi = hi & ~7u;
+                    for (uint32_t l0 = c_lo + 8u * lane; l0 < c_hi; l0 += 256u) {
+                        const uint2 s2 = __ldg(reinterpret_cast<const uint2 *>(smg + l0));
+                        const uint2 e2 = *reinterpret_cast<const uint2 *>(exp_s + l0);
+                        uint4 r;
+                        merge4(s2.x, e2.x, r.x, r.y);
+                        merge4(s2.y, e2.y, r.z, r.w);
+                        st_shared_v4(addr(l0), r);
+                    }
+                    // ... and up to 7 single elements at each end
+                    const uint32_t head_end = c_lo < hi ? c_lo : hi, tail0 = c_hi > c_lo ? c_hi : c_lo;
+                    const uint32_t l = lane < 8 ? lo + lane : tail0 + (lane - 8);
+                    if ((lane < 8 && l < head_end) || (lane >= 8 && lane < 16 && l < hi))
+                        st_shared_u16(addr(l), merge1(__ldg(smg + l), exp_s[l]));
+                    fence_proxy_async();  // the tiles are read by the tensor core (async proxy)
+                    __syncwarp();
+                    // counted before this warp arrives on any of these tiles
+                    if (lane == 0)
+                        atomicAdd(R.cover + k % kCoverSlots, hi - lo);
+                }
+            }
+            // tiles this warp will not write again: up to the next block's first
+            const uint64_t next0 = more ? (uint64_t)nxt.o0 : e1;
+            const uint32_t t_next =
+                next0 >= e1 ? U.ntiles : (next0 <= e0 ? 0u : (uint32_t)((next0 - e0) >> kTileShift));
+            for (; arrived < t_next && ok; arrived++) {
+                ok = slot_free(q0 + arrived);
+                if (ok && lane == 0)
+                    mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
+            }
+            cur = nxt;
+        }
+        for (; arrived < U.ntiles && ok; arrived++) {
+            ok = slot_free(q0 + arrived);
+            if (ok && lane == 0)
+                mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
+        }
+        if (!ok)
+            return;
+        q0 += U.ntiles;
+    }
+}
+
+// Control thread: X copies, MMAs, commits.
+__device__ __forceinline__ void control_role(const GemmParams &p, const Roles &R)
+{
+    const uint32_t S = p.stages, N = p.batch, xbytes = N * 128;
+    const uint32_t idesc = idesc_bf16(kTileRows, N);
+    uint32_t expect[kCoverSlots];
+#pragma unroll
+    for (uint32_t i = 0; i < kCoverSlots; i++)
+        expect[i] = 0;
+    uint32_t q0 = 0, k = 0, x_issued = 0, x_used = 0, committed = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, k++) {
+        const Unit U = unit_of(p, u);
+        const GemmMat &M = p.mats[U.m];
+        const uint8_t *xsrc = p.xpack + M.xoff + (uint64_t)U.kc0 * xbytes;
+        const uint32_t d = k & 1u;
+        // X chunk of tile t of the unit into its slot, once the slot is free
+        auto issue_x = [&](uint32_t t) -> bool {
+            const uint32_t q = q0 + t, s = q % S;
+            if (q >= S && !mbar_wait(bar(R, kBarEmpty + s), (q / S - 1) & 1u, R.abort_flag, p.status))
+                return false;
+            mbar_arrive_tx(bar(R, kBarX + s), xbytes);
+            bulk_copy_g2s(R.ring_b + s * xbytes, xsrc + (uint64_t)t * xbytes, xbytes, bar(R, kBarX + s));
+            x_issued = q + 1;
+            return true;
+        };
+        const uint32_t ahead = S - 1 < U.ntiles ? S - 1 : U.ntiles;
+        for (uint32_t t = 0; t < ahead && ok; t++)
+            ok = issue_x(t);
+        // the accumulator is free once the epilogue has read unit k - 2
+        if (ok && k >= 2)
+            ok = mbar_wait(bar(R, kBarFree + d), ((k >> 1) - 1) & 1u, R.abort_flag, p.status);
+        for (uint32_t t = 0; t < U.ntiles && ok; t++) {
+            const uint32_t q = q0 + t, s = q % S, ph = (q / S) & 1u;
+            ok = mbar_wait(bar(R, kBarFull + s), ph, R.abort_flag, p.status) &&
+                 mbar_wait(bar(R, kBarX + s), ph, R.abort_flag, p.status);
+            if (!ok)
+                break;
+            x_used = q + 1;
+            tc_fence_after();
+            const uint64_t ad = sw128_desc(R.ring_a + s * kTileBytes), bd = sw128_desc(R.ring_b + s * xbytes);
+#pragma unroll
+            for (uint32_t kk = 0; kk < 4; kk++)
+                umma_bf16(R.tmem + d * N, ad + 2 * kk, bd + 2 * kk, idesc, (t | kk) != 0);
+            umma_commit(bar(R, kBarEmpty + s));
+            committed = 1;
+            if (t + S - 1 < U.ntiles)
+                ok = issue_x(t + S - 1);
+        }
+        if (!ok)
+            break;
+        // every tile of the unit is full: the decode warps' element counts
+        // are final and must add up to the unit's elements
+        const uint32_t c = k % kCoverSlots;
+        expect[c] += U.ntiles * kTileElems;
+        if (*reinterpret_cast<volatile uint32_t *>(R.cover + c) != expect[c])
+            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+        umma_commit(bar(R, kBarAcc + d));
+        q0 += U.ntiles;
+    }
+    // drain: copies issued but never waited for, and every MMA
+    for (uint32_t q = x_used; q < x_issued; q++)
+        mbar_wait(bar(R, kBarX + q % S), (q / S) & 1u, R.abort_flag, p.status, false);
+    if (committed) {
+        umma_commit(bar(R, kBarDrain));
+        mbar_wait(bar(R, kBarDrain), 0u, R.abort_flag, p.status, false);
+    }
+}
+
+// Epilogue warp: adds each unit's accumulator rows 32 q .. 32 q + 31 (q =
+// warp mod 4, the tensor-memory lanes this warp may read) into Y.
+__device__ __forceinline__ void epilogue_role(const GemmParams &p, const Roles &R, uint32_t warp, int lane)
+{
+    const uint32_t quarter = warp & 3u, N = p.batch;
+    uint32_t k = 0;
+    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
+        const uint32_t d = k & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(R, kBarAcc + d), (k >> 1) & 1u, R.abort_flag, p.status)))
+            return;
+        tc_fence_after();
+        const Unit U = unit_of(p, u);
+        const GemmMat &M = p.mats[U.m];
+        const uint32_t row = U.row0 + 32 * quarter + (uint32_t)lane;
+        const uint32_t taddr = R.tmem + ((32 * quarter) << 16) + d * N;
+        for (uint32_t c0 = 0; c0 < N; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(taddr + c0, r);
+#pragma unroll
+            for (uint32_t j = 0; j < 16; j++)
+                atomicAdd(M.y + (uint64_t)(c0 + j) * M.rows + row, __uint_as_float(r[j]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar(R, kBarFree + d));
+    }
+}
+
+template <int C>
+__global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t tid = threadIdx.x, warp = tid >> 5;
+    const int lane = (int)(tid & 31u);
+    const uint32_t S = p.stages;
+    uint8_t *ctrl = smem + ctrl_offset(p.cap);
+    Roles R;
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    R.bars = static_cast<uint32_t>(__cvta_generic_to_shared(ctrl));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + kNumBars * 8);
+    R.abort_flag = tmem_slot + 1;
+    R.cover = tmem_slot + 2;
+    R.ring_a = (base + ctrl_offset(p.cap) + kCtrlBytes + 1023u) & ~1023u;
+    R.ring_b = R.ring_a + S * kTileBytes;
+
+    if (tid == 0) {
+        for (uint32_t s = 0; s < S; s++) {
+            mbar_init(bar(R, kBarFull + s), kDecodeWarps);
+            mbar_init(bar(R, kBarEmpty + s), 1);
+            mbar_init(bar(R, kBarX + s), 1);
+        }
+        for (uint32_t d = 0; d < 2; d++) {
+            mbar_init(bar(R, kBarAcc + d), 1);
+            mbar_init(bar(R, kBarFree + d), 4);
+        }
+        mbar_init(bar(R, kBarDrain), 1);
+        *R.abort_flag = 0u;
+        for (uint32_t i = 0; i < kCoverSlots; i++)
+            R.cover[i] = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async();
+    }
+    if (warp == kControlWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         static_cast<uint32_t>(__cvta_generic_to_shared(tmem_slot))),
+                     "r"(p.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        tc_fence_before();
+    }
+    // the tables (the barriers, flags and tensor-memory address above are
+    // published by its __syncthreads)
+    build_tables(p.luts, p.cl, p.num_luts, smem, tid, kGemmThreads);
+    tc_fence_after();
+    R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+    if (warp < kDecodeWarps) {
+        decode_role<C>(p, R, smem, warp, lane);
+    } else if (warp == kControlWarp) {
+        if (lane == 0)
+            control_role(p, R);
+        __syncwarp();
+    } else {
+        epilogue_role(p, R, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kControlWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(R.tmem), "r"(p.tmem_cols)
+                     : "memory");
+    }
+}
+
+// SM count and opt-in shared memory per device, and the dynamic shared
+// memory already granted to each kernel.
+struct GemmFacts {
+    int sms = 0;
+    int smem_optin = 0;
+    uint32_t granted[2] = {0, 0};
+};
+std::mutex g_gemm_mu;
+GemmFacts g_gemm[64];
+
+// Work units and packed-X bytes of a matrix list; false if it is invalid.
+bool plan_units(const df11_gemm_matrix *mats, uint32_t num_mats, uint32_t batch, uint64_t *units, uint64_t *xbytes)
+{
+    if (!mats || num_mats < 1 || num_mats > kMaxGemmMats || batch < 16 || batch > 256 || batch % 16)
+        return false;
+    uint64_t nu = 0, xb = 0;
+    for (uint32_t m = 0; m < num_mats; m++) {
+        const df11_gemm_matrix &M = mats[m];
+        if (M.rows == 0 || M.cols == 0 || M.rows % kTileRows || M.cols % kTileCols)
+            return false;
+        const uint64_t kchunks = M.cols / kTileCols;
+        nu += (uint64_t)(M.rows / kTileRows) * ((kchunks + kUnitChunks - 1) / kUnitChunks);
+        xb += (uint64_t)M.cols * batch * 2;
+    }
+    if (nu >= (1ull << 31))
+        return false;
+    *units = nu;
+    *xbytes = xb;
+    return true;
+}
+
+}  // namespace
+
+extern "C" uint64_t df11_gemm_scratch_bytes(const df11_gemm_matrix *mats, uint32_t num_mats, uint32_t batch)
+{
+    uint64_t units = 0, xbytes = 0;
+    if (!plan_units(mats, num_mats, batch, &units, &xbytes))
+        return 0;
+    return xbytes + 8 * units;
+}
+
+extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gemm_matrix *mats, uint32_t num_mats,
+                                            uint32_t batch, void *scratch, uint64_t scratch_bytes,
+                                            uint32_t *status_dev, void *stream)
+{
+    uint64_t units = 0, xbytes = 0;
+    if (!a || !status_dev || !plan_units(mats, num_mats, batch, &units, &xbytes) || a->n == 0)
+        return DF11_ERR_INVALID_ARG;
+    if (!scratch || !aligned(scratch, 16) || scratch_bytes < xbytes + 8 * units)
+        return DF11_ERR_INVALID_ARG;
+    GemmParams prm;
+    const df11_status st = stream_params(a, status_dev, prm);
+    if (st != DF11_OK)
+        return st;
+    uint64_t off = 0, unit0 = 0, piece0 = 0, xoff = 0;
+    for (uint32_t m = 0; m < num_mats; m++) {
+        const df11_gemm_matrix &M = mats[m];
+        if (!M.x || !M.y || !aligned(M.x, 16) || !aligned(M.y, 4))
+            return DF11_ERR_INVALID_ARG;
+        GemmMat &G = prm.mats[m];
+        G.off = (uint32_t)off;
+        G.rows = M.rows;
+        G.cols = M.cols;
+        G.unit0 = (uint32_t)unit0;
+        G.units_per_rt = (M.cols / kTileCols + kUnitChunks - 1) / kUnitChunks;
+        G.piece0 = (uint32_t)piece0;
+        G.xoff = xoff;
+        G.x = M.x;
+        G.y = M.y;
+        off += (uint64_t)M.rows * M.cols;
+        if (off > a->n)
+            return DF11_ERR_INVALID_ARG;
+        unit0 += (uint64_t)(M.rows / kTileRows) * G.units_per_rt;
+        piece0 += (uint64_t)M.cols / 8 * batch;
+        xoff += (uint64_t)M.cols * batch * 2;
+    }
+    if (off != a->n || piece0 >= (1ull << 31))
+        return DF11_ERR_INVALID_ARG;  // the matrices must cover the stream exactly
+    prm.batch = batch;
+    prm.num_mats = num_mats;
+    prm.num_units = (uint32_t)units;
+    prm.num_pieces = (uint32_t)piece0;
+    prm.xpack = static_cast<uint8_t *>(scratch);
+    prm.unit_blocks = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(scratch) + xbytes);
+    uint32_t cols = 32;
+    while (cols < 2 * batch)
+        cols <<= 1;
+    prm.tmem_cols = cols;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return DF11_ERR_CUDA;
+    GemmFacts *f = &g_gemm[dev];
+    {
+        std::lock_guard<std::mutex> lock(g_gemm_mu);
+        if (!f->sms) {
+            int sms = 0, optin = 0;
+            if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+                return DF11_ERR_CUDA;
+            f->smem_optin = optin;
+            f->sms = sms;
+        }
+    }
+    // as many ring stages as fit (at least 2)
+    uint32_t stages = kMaxStages;
+    while (stages >= 2 && gemm_smem_bytes(prm.cap, batch, stages) > (uint32_t)f->smem_optin)
+        stages--;
+    if (stages < 2)
+        return DF11_ERR_INVALID_ARG;
+    prm.stages = stages;
+    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages);
+    const int ci = a->threads_per_block == 32 ? 0 : 1;
+    auto kern = ci == 0 ? df11_gemm_kernel<1> : df11_gemm_kernel<2>;
+    {
+        std::lock_guard<std::mutex> lock(g_gemm_mu);
+        if (smem > f->granted[ci]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return DF11_ERR_CUDA;
+            f->granted[ci] = smem;
+        }
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint64_t prep = prm.num_pieces > prm.num_units ? prm.num_pieces : prm.num_units;
+    gemm_prep_kernel<<<(unsigned)((prep + 255) / 256), 256, 0, s>>>(prm);
+    if (cudaGetLastError() != cudaSuccess)
+        return DF11_ERR_CUDA;
+    const uint32_t grid = (uint32_t)f->sms < prm.num_units ? (uint32_t)f->sms : prm.num_units;
+    kern<<<grid, kGemmThreads, smem, s>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}
+
+extern "C" df11_status df11_tile_major(const uint16_t *src, uint32_t rows, uint32_t cols, uint16_t *dst)
+{
+    if (!src || !dst || rows % kTileRows || cols % kTileCols)
+        return DF11_ERR_INVALID_ARG;
+    uint64_t o = 0;
+    for (uint32_t r0 = 0; r0 < rows; r0 += kTileRows)
+        for (uint32_t c0 = 0; c0 < cols; c0 += kTileCols)
+            for (uint32_t r = r0; r < r0 + kTileRows; r++) {
+                std::memcpy(dst + o, src + (uint64_t)r * cols + c0, kTileCols * 2);
+                o += kTileCols;
+            }
+    return DF11_OK;
+}

@@ -19,7 +19,9 @@ only orders launches.  Run as a module it times one such pass with a
 stand-in consumer (the block's seven GEMMs against a batch of activations):
 ``python -m huffman_decode_03_b200.pipeline --blocks 8 --batch 64``; with
 ``--gemv`` it compares, at batch 1, decompress + cuBLAS matrix-vector
-products against the fused ``df11_decompress_gemv``.
+products against the fused ``df11_decompress_gemv``; with ``--gemm``, at
+``--batch`` activation vectors, decompress + cuBLAS GEMMs against the fused
+tensor-core ``df11_decompress_gemm`` (weights stored tile-major).
 """
 from __future__ import annotations
 
@@ -240,6 +242,83 @@ def _bench_gemv(args):
     print(json.dumps(res))
 
 
+def _bench_gemm(args):
+    """Batch-B use of each block: decompress, then the seven GEMMs with
+    cuBLAS, against df11_decompress_gemm (decode into tensor-core operand
+    tiles and multiply in one kernel, no BF16 weights written)."""
+    import numpy as np
+    import torch
+
+    from . import decompress_gemm, gemm_scratch_bytes, tile_major
+
+    dev = torch.device("cuda")
+    shapes = [s for _, s in inputs.LLAMA3_8B]
+    B = args.batch
+    rowmajor, tiled, dense = [], [], []
+    for b in range(args.blocks):
+        mats = [m for _, _, m in inputs.block(5, b)]
+        rowmajor.append(DeviceFormat(build_format(mats), dev))
+        tiled.append(DeviceFormat(build_format([tile_major(m, r, c) for m, (r, c) in zip(mats, shapes)]), dev))
+        if args.dense:
+            dense.append(torch.from_numpy(np.concatenate(mats).view(np.int16)).to(dev).view(torch.bfloat16))
+    g = torch.Generator(device="cpu").manual_seed(12)
+    xs = [torch.randn(B, c, generator=g).to(torch.bfloat16).to(dev) for _, c in shapes]
+    ys = [torch.zeros(B, r, dtype=torch.float32, device=dev) for r, _ in shapes]
+    buf = torch.empty(max(f.n for f in rowmajor), dtype=torch.bfloat16, device=dev)
+    scratch = torch.empty(gemm_scratch_bytes(shapes, B), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def gemms(w):
+        off, outs = 0, []
+        for (r, c), x in zip(shapes, xs):
+            outs.append(x @ w[off:off + r * c].view(r, c).T)
+            off += r * c
+        return outs
+
+    def separate():
+        for f in rowmajor:
+            decompress(f, buf[:f.n], st)
+            gemms(buf[:f.n])
+
+    def fused():
+        for y in ys:
+            y.zero_()
+        for f in tiled:
+            decompress_gemm(f, shapes, xs, ys, st, scratch=scratch)
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
+    nb = args.blocks
+    res = {"blocks": nb, "batch": B, "block": "llama3_8b (q,k,v,o,gate,up,down)",
+           "decode_then_cublas_gemm_ms": timed(separate, args.reps),
+           "fused_decode_gemm_ms": timed(fused, args.reps)}
+    if args.dense:
+        res["cublas_gemm_dense_ms"] = timed(lambda: [gemms(w) for w in dense], args.reps)
+        # the fused result of the last block against cuBLAS on the original weights
+        for y in ys:
+            y.zero_()
+        decompress_gemm(tiled[-1], shapes, xs, ys, st, scratch=scratch)
+        ref = gemms(dense[-1])
+        torch.cuda.synchronize()
+        res["max_rel_diff_vs_cublas_bf16_out"] = max(
+            float(((y - r.float()).abs().max() / r.float().abs().max()).item()) for y, r in zip(ys, ref))
+    torch.cuda.synchronize()
+    res["status"] = int(st.item())
+    res["per_block_us"] = {k[:-3]: round(1000 * v / nb, 1) for k, v in res.items() if k.endswith("_ms")}
+    print(json.dumps(res))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--blocks", type=int, default=8)
@@ -252,7 +331,12 @@ def main(argv=None):
     ap.add_argument("--no-check", dest="check", action="store_false")
     ap.add_argument("--gemv", action="store_true",
                     help="batch-1 comparison: decompress + cuBLAS matrix-vector products vs df11_decompress_gemv")
+    ap.add_argument("--gemm", action="store_true",
+                    help="batch-B comparison: decompress + cuBLAS GEMMs vs df11_decompress_gemm")
     args = ap.parse_args(argv)
+    if args.gemm:
+        _bench_gemm(args)
+        return
     if args.gemv:
         _bench_gemv(args)
         return

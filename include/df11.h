@@ -220,6 +220,62 @@ typedef struct df11_gemv_matrix {
 df11_status df11_decompress_gemv(const df11_arrays *dev, const df11_gemv_matrix *mats, uint32_t num_mats,
                                  uint32_t *status_dev, void *stream);
 
+/* One matrix of df11_decompress_gemm: `rows` x `cols` BF16 weights W, the
+ * next rows*cols elements of the stream (matrices in stream order), stored
+ * in TILE-MAJOR order (df11_tile_major): 128 x 64 tiles, row tiles in order,
+ * within a row tile the column tiles in order, within a tile 128 rows of 64
+ * elements. */
+typedef struct df11_gemm_matrix {
+    uint32_t rows;       /* a multiple of 128 */
+    uint32_t cols;       /* a multiple of 64 */
+    const uint16_t *x;   /* device: batch x cols BF16 activations, row-major, 16-byte aligned */
+    float *y;            /* device: batch x rows float32 outputs, row-major, 4-byte aligned */
+} df11_gemm_matrix;
+
+/*
+ * df11_decompress_gemm -- decode and multiply for a batch of activation
+ * vectors: Y_m += X_m W_m^T for every matrix m of the stream, on the tensor
+ * cores (tcgen05.mma, BF16 inputs, float32 accumulation), W_m decoded tile by
+ * tile into shared memory and never written to global memory ("Dekompresi
+ * yang disesuaikan untuk inferensi GPU": decompress right before the matrix
+ * multiplication; the page's discussion proposes a GEMM that decompresses
+ * each tile before its arithmetic).  Every output is a float32 sum of cols
+ * exact BF16 products, accumulated by the tensor core over K chunks of 64 and
+ * by atomic adds over groups of 16 chunks (so the last bits of Y vary between
+ * runs).
+ *   dev        the stream's arrays (device pointers), as df11_decompress;
+ *              the matrices' elements in tile-major order.
+ *   mats       host array of num_mats (1..16) matrices whose rows*cols add
+ *              up to dev->n; Y is accumulated, not overwritten.
+ *   batch      number of activation vectors: a multiple of 16, 16..256.
+ *   scratch    device buffer of at least df11_gemm_scratch_bytes(mats,
+ *              num_mats, batch) bytes, 16-byte aligned, owned by the caller
+ *              and not in use by other work until this call's kernels end
+ *              (it receives X repacked for the tensor core and each work
+ *              unit's format blocks).
+ *   status_dev, stream: as df11_decompress.  Bit 31 of *status_dev set means
+ *              a bounded wait inside the kernel ran out (Y incomplete).
+ * Asynchronous (two launches on `stream`); DF11_ERR_INVALID_ARG for bad
+ * arguments (nothing launched), DF11_ERR_CUDA if a launch fails.
+ */
+df11_status df11_decompress_gemm(const df11_arrays *dev, const df11_gemm_matrix *mats, uint32_t num_mats,
+                                 uint32_t batch, void *scratch, uint64_t scratch_bytes,
+                                 uint32_t *status_dev, void *stream);
+
+/* Scratch bytes df11_decompress_gemm needs for these matrices and batch;
+ * 0 if the arguments are invalid (see df11_decompress_gemm). */
+uint64_t df11_gemm_scratch_bytes(const df11_gemm_matrix *mats, uint32_t num_mats, uint32_t batch);
+
+/*
+ * df11_tile_major -- host: writes the rows x cols row-major BF16 matrix src
+ * (host memory) to dst (host, rows*cols elements, not overlapping src) in the
+ * tile-major order df11_decompress_gemm reads: for each row tile of 128 rows,
+ * for each column tile of 64 columns, its 128 rows of 64 elements.  Compress
+ * the result with df11_build_format.  DF11_ERR_INVALID_ARG unless rows is a
+ * multiple of 128 and cols of 64.
+ */
+df11_status df11_tile_major(const uint16_t *src, uint32_t rows, uint32_t cols, uint16_t *dst);
+
 /*
  * df11_decompress_host -- the same decode, starting and ending in host
  * memory: copies every array of *host (host pointers, ideally pinned) into
