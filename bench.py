@@ -37,7 +37,8 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAME = "df11_decode_kernel"
-KERNEL_SOURCE = os.path.join(ROOT, "huffman_decode_03_b200", "csrc", "df11_decode.cu")
+# the decode kernel's source: the kernel and its shared per-block decode
+KERNEL_SOURCES = [os.path.join(ROOT, "huffman_decode_03_b200", "csrc", f) for f in ("df11_decode.cu", "df11_block.cuh")]
 PROFILES = os.path.join(ROOT, "profiles")
 
 
@@ -108,8 +109,11 @@ def load_peak():
 
 
 def kernel_source_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for path in KERNEL_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: int, n_elems: int):

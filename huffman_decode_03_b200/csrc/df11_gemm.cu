@@ -26,8 +26,9 @@
 //     with the per-block decode shared with the other kernels, merges each
 //     exponent with its sign/mantissa byte and stores the BF16 weight at its
 //     place in a ring of S operand tiles in shared memory (K-major, 128-byte
-//     swizzle).  A warp arrives on a tile's "full" barrier as soon as its next
-//     block starts past that tile;
+//     swizzle).  A warp arrives on a tile's "full" barrier once no block it
+//     still has to decode reaches into that tile, and on every tile before a
+//     block before it waits for a ring slot for that block;
 //   * 1 control warp: allocates tensor memory; one of its threads copies each
 //     K chunk of X into the ring by a bulk copy (cp.async.bulk, no tensor
 //     map), waits for the tile to be full, issues four tcgen05.mma (K = 16
@@ -348,6 +349,20 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
         const uint32_t bb = p.unit_blocks[2 * u], be = p.unit_blocks[2 * u + 1];
         uint32_t arrived = 0;
         bool ok = true;
+        // tile of the unit holding stream element x (0 before it, ntiles past it)
+        auto tile_of = [&](uint64_t x) -> uint32_t {
+            return x >= e1 ? U.ntiles : (x <= e0 ? 0u : (uint32_t)((x - e0) >> kTileShift));
+        };
+        // arrives on tiles [arrived, t_end): this warp writes nothing more there
+        auto arrive_upto = [&](uint32_t t_end) -> bool {
+            for (; arrived < t_end; arrived++) {
+                if (!slot_free(q0 + arrived))
+                    return false;
+                if (lane == 0)
+                    mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
+            }
+            return true;
+        };
         BlockRegs<C> cur, nxt;
         uint32_t b = bb + warp;
         if (b < be)
@@ -356,6 +371,12 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
             const bool more = b + kDecodeWarps < be;
             if (more)
                 load_block<C>(p, b + kDecodeWarps, lane, nxt);
+            // Before waiting for any ring slot: arrive on the tiles before
+            // this block.  The MMA of a tile needs every warp's arrival, and
+            // a slot frees only when the MMA of the tile S earlier is done.
+            ok = arrive_upto(tile_of(cur.o0));
+            if (!ok)
+                break;
             BlockOut bo;
             if (decode_block<C>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
                 // the block's outputs inside the unit: [lo, hi) relative to g0
@@ -398,22 +419,11 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
                         atomicAdd(R.cover + k % kCoverSlots, hi - lo);
                 }
             }
-            // tiles this warp will not write again: up to the next block's first
-            const uint64_t next0 = more ? (uint64_t)nxt.o0 : e1;
-            const uint32_t t_next =
-                next0 >= e1 ? U.ntiles : (next0 <= e0 ? 0u : (uint32_t)((next0 - e0) >> kTileShift));
-            for (; arrived < t_next && ok; arrived++) {
-                ok = slot_free(q0 + arrived);
-                if (ok && lane == 0)
-                    mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
-            }
+            // and, right away, on the tiles before the next block
+            ok = arrive_upto(more ? tile_of(nxt.o0) : U.ntiles);
             cur = nxt;
         }
-        for (; arrived < U.ntiles && ok; arrived++) {
-            ok = slot_free(q0 + arrived);
-            if (ok && lane == 0)
-                mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
-        }
+        ok = ok && arrive_upto(U.ntiles);
         if (!ok)
             return;
         q0 += U.ntiles;
