@@ -199,10 +199,12 @@ class Format:
             return np.zeros(0, dtype)
         nbytes = int(count) * np.dtype(dtype).itemsize
         buf = (ctypes.c_uint8 * nbytes).from_address(ptr)
+        buf._owner = self  # the array keeps the buffer, the buffer keeps the handle
         return np.frombuffer(buf, dtype=dtype, count=int(count))
 
     def arrays(self) -> dict:
-        """Borrowed numpy views of the host arrays (valid while self lives)."""
+        """numpy views of the host arrays; each view keeps this handle (and
+        so its memory) alive."""
         a = self.c_arrays
         return {
             "encoded_exponent": self._view(a.encoded_exponent, a.encoded_exponent_bytes, np.uint8),

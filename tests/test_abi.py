@@ -5,6 +5,8 @@ import os
 import re
 import subprocess
 
+import numpy as np
+
 import huffman_decode_03_b200 as df11
 from huffman_decode_03_b200 import build as build_mod
 
@@ -63,3 +65,19 @@ def test_strerror_covers_all_codes():
     lib = df11.load_library()
     texts = {lib.df11_strerror(i).decode() for i in range(8)}
     assert len(texts) == 8 and "unknown status" not in texts
+
+
+def test_array_views_keep_the_format_alive():
+    # views of a temporary Format stay valid: each keeps the handle alive
+    import gc
+
+    from huffman_decode_03_b200 import inputs
+
+    w = inputs.gaussian(1 << 20, [5])
+    ref = df11.build_format(w)
+    want = ref.arrays()["block_offset"].copy()
+    offs = df11.build_format(w).arrays()["block_offset"]
+    gc.collect()
+    others = [df11.build_format(inputs.gaussian(1 << 18, [6, i])) for i in range(4)]  # reuse freed memory
+    assert np.array_equal(offs, want)
+    assert len(others) == 4
