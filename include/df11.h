@@ -19,7 +19,10 @@
  *   - device decode: df11_decompress rebuilds the BF16 matrix on a CUDA
  *     stream (df11_decompress_sms on at most a given number of SMs);
  *     df11_decompress_gemv decodes and multiplies by vectors without storing
- *     the weights; df11_decompress_host takes the arrays in host memory and
+ *     the weights (CUDA cores); df11_decompress_gemm does the same for a
+ *     batch of vectors on the tensor cores (tile-major streams, see
+ *     df11_tile_major; df11_gemm_scratch_bytes sizes its scratch);
+ *     df11_decompress_host takes the arrays in host memory and
  *     overlaps the copies with the decode; df11_read_status reads the
  *     kernels' error word;
  *   - device encode: df11_device_histogram counts exponents of a device

@@ -20,7 +20,6 @@ version of the kernel) deadlocks on these streams once the first block of the
 last warp starts S or more tiles into a unit; the model shows that too, as
 the kernel did on a B200 (its bounded waits ran out and it reported the
 timeout instead of hanging)."""
-import numpy as np
 import pytest
 
 import huffman_decode_03_b200 as df11
@@ -166,3 +165,15 @@ def test_arriving_only_after_the_first_block_deadlocks():
     for S in (2, 3):
         assert not _run_cta(offs, units[:1], S, arrive_first=False)
         assert _run_cta(offs, units[:1], S)
+
+
+@pytest.mark.slow
+def test_protocol_finishes_on_the_llama3_8b_block():
+    # the fused GEMM's workload: 1,664 units over 148 CTAs, T = 64, the ring
+    # depths of batch 256 (S = 2) and batch 64 (S = 4)
+    shapes = [s for _, s in inputs.LLAMA3_8B]
+    offs = _offsets(shapes, [m for _, _, m in inputs.block(2, 0)], 64)
+    units = _units(shapes)
+    for S in (2, 4):
+        for cta in range(148):
+            assert _run_cta(offs, units[cta::148], S), (S, cta)
