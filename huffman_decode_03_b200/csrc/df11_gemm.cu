@@ -26,9 +26,11 @@
 //     with the per-block decode shared with the other kernels, merges each
 //     exponent with its sign/mantissa byte and stores the BF16 weight at its
 //     place in a ring of S operand tiles in shared memory (K-major, 128-byte
-//     swizzle).  A warp arrives on a tile's "full" barrier once no block it
-//     still has to decode reaches into that tile, and on every tile before a
-//     block before it waits for a ring slot for that block;
+//     swizzle).  A warp arrives on a tile's "full" barrier as soon as none
+//     of its remaining blocks reaches into that tile: on the tiles before a
+//     block's first output BEFORE it waits for that block's ring slots (a
+//     slot frees only after the MMA of an earlier tile, which needs every
+//     warp's arrival), and on those before its next block right after;
 //   * 1 control warp: allocates tensor memory; one of its threads copies each
 //     K chunk of X into the ring by a bulk copy (cp.async.bulk, no tensor
 //     map), waits for the tile to be full, issues four tcgen05.mma (K = 16
