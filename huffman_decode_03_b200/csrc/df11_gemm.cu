@@ -399,20 +399,25 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
                         const uint32_t v = (uint32_t)(g0 + l - e0);
                         return ((v >> kTileShift) == t_first ? sa0 : sa1) + tile_offset(v & (kTileElems - 1));
                     };
-                    // whole groups of 8 (16 bytes of the tile) ...
-                    const uint32_t c_lo = (lo + 7u) & ~7u, c_hi = hi & ~7u;
-                    for (uint32_t l0 = c_lo + 8u * lane; l0 < c_hi; l0 += 256u) {
-                        const uint2 s2 = __ldg(reinterpret_cast<const uint2 *>(smg + l0));
-                        const uint2 e2 = *reinterpret_cast<const uint2 *>(exp_s + l0);
-                        uint4 r;
-                        merge4(s2.x, e2.x, r.x, r.y);
-                        merge4(s2.y, e2.y, r.z, r.w);
-                        st_shared_v4(addr(l0), r);
+                    // whole groups of 16 (two 16-byte pieces of one tile row:
+                    // a group never crosses a row of 64 or a tile) ...
+                    const uint32_t c_lo = (lo + 15u) & ~15u, c_hi = hi & ~15u;
+                    for (uint32_t l0 = c_lo + 16u * lane; l0 < c_hi; l0 += 512u) {
+                        const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(smg + l0));
+                        const uint4 e4 = *reinterpret_cast<const uint4 *>(exp_s + l0);
+                        uint4 r0, r1;
+                        merge4(s4.x, e4.x, r0.x, r0.y);
+                        merge4(s4.y, e4.y, r0.z, r0.w);
+                        merge4(s4.z, e4.z, r1.x, r1.y);
+                        merge4(s4.w, e4.w, r1.z, r1.w);
+                        const uint32_t a0 = addr(l0);
+                        st_shared_v4(a0, r0);
+                        st_shared_v4(a0 ^ 16u, r1);  // the next 8 columns: group index + 1, XOR row
                     }
-                    // ... and up to 7 single elements at each end
+                    // ... and up to 15 single elements at each end
                     const uint32_t head_end = c_lo < hi ? c_lo : hi, tail0 = c_hi > c_lo ? c_hi : c_lo;
-                    const uint32_t l = lane < 8 ? lo + lane : tail0 + (lane - 8);
-                    if ((lane < 8 && l < head_end) || (lane >= 8 && lane < 16 && l < hi))
+                    const uint32_t l = lane < 16 ? lo + lane : tail0 + (lane - 16);
+                    if (lane < 16 ? l < head_end : l < hi)
                         st_shared_u16(addr(l), merge1(__ldg(smg + l), exp_s[l]));
                     fence_proxy_async();  // the tiles are read by the tensor core (async proxy)
                     __syncwarp();
