@@ -299,8 +299,10 @@ df11_status df11_decompress_host(const df11_arrays *host, const df11_arrays *dev
 
 /*
  * df11_read_status -- synchronises `stream`, reads *status_dev (device
- * pointer) and returns DF11_OK or DF11_ERR_CORRUPT (DF11_ERR_CUDA if the
- * copy fails).
+ * pointer) and returns DF11_OK if it is 0, else DF11_ERR_CORRUPT
+ * (DF11_ERR_CUDA if the copy fails).  The kernels only OR bits into the word:
+ * DF11_ERR_CORRUPT's value for inconsistent data, bit 31 for a bounded wait
+ * of df11_decompress_gemm that ran out.  Zero it before the calls it covers.
  */
 df11_status df11_read_status(const uint32_t *status_dev, void *stream);
 
