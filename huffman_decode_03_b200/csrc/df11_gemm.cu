@@ -22,8 +22,10 @@
 // prep kernel packs every 64-column chunk of X into the shared-memory image
 // the tensor core reads and finds each unit's first and last format block.
 // Then one persistent CTA per SM takes units blockIdx.x, + gridDim.x, ...:
-//   * 16 decode warps: warp w decodes the unit's format blocks w, w + 16, ...
-//     with the per-block decode shared with the other kernels, merges each
+//   * DW decode warps (20 when at least 3 ring stages fit beside them, which
+//     holds up to batch 64; else 16): warp w decodes the unit's format blocks
+//     w, w + DW, ... with the per-block decode shared with the other kernels,
+//     merges each
 //     exponent with its sign/mantissa byte and stores the BF16 weight at its
 //     place in a ring of S operand tiles in shared memory (K-major, 128-byte
 //     swizzle).  A warp arrives on a tile's "full" barrier as soon as none
@@ -60,9 +62,12 @@ constexpr uint32_t kTileRows = 128, kTileCols = 64;
 constexpr uint32_t kTileElems = kTileRows * kTileCols;  // 8192
 constexpr uint32_t kTileShift = 13;
 constexpr uint32_t kTileBytes = kTileElems * 2;          // 16 KB
-constexpr uint32_t kDecodeWarps = 16;
-constexpr uint32_t kControlWarp = kDecodeWarps;  // then 4 epilogue warps
-constexpr uint32_t kGemmThreads = (kDecodeWarps + 1 + 4) * 32;
+// DW decode warps, then the control warp (warp DW), then 4 epilogue warps.
+// 20 decode warps when at least kMinStages20 ring stages fit beside them,
+// else 16 (more warps hide more of the decode loop's latency; a ring of 2
+// stalls the decode warps more often).
+__host__ __device__ constexpr uint32_t gemm_threads(uint32_t dw) { return (dw + 1 + 4) * 32; }
+constexpr uint32_t kMinStages20 = 3;
 constexpr uint32_t kMaxStages = 8;
 constexpr uint32_t kUnitChunks = 16;  // K chunks per work unit, at most
 constexpr uint32_t kMaxGemmMats = 16;
@@ -116,16 +121,16 @@ struct GemmParams {
     GemmMat mats[kMaxGemmMats];
 };
 
-__host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap)
+__host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap, uint32_t dw)
 {
-    return align16(Smem::bufs + kDecodeWarps * Smem::per_warp(cap));
+    return align16(Smem::bufs + dw * Smem::per_warp(cap));
 }
 
 // Dynamic shared memory of a launch: tables, decode buffers, control area,
 // 1 KB to align the ring, the ring.
-__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages)
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages, uint32_t dw)
 {
-    return ctrl_offset(cap) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
+    return ctrl_offset(cap, dw) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: BF16 A and B, both
@@ -321,8 +326,8 @@ struct Roles {
 
 __device__ __forceinline__ uint32_t bar(const Roles &R, uint32_t i) { return R.bars + 8 * i; }
 
-// Decode warp: every unit of the CTA, blocks warp, warp + 16, ... of it.
-template <int C>
+// Decode warp: every unit of the CTA, blocks warp, warp + DW, ... of it.
+template <int C, int DW>
 __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R, uint8_t *smem, uint32_t warp,
                                             int lane)
 {
@@ -369,10 +374,10 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
         uint32_t b = bb + warp;
         if (b < be)
             load_block<C>(p, b, lane, cur);
-        for (; b < be && ok; b += kDecodeWarps) {
-            const bool more = b + kDecodeWarps < be;
+        for (; b < be && ok; b += DW) {
+            const bool more = b + DW < be;
             if (more)
-                load_block<C>(p, b + kDecodeWarps, lane, nxt);
+                load_block<C>(p, b + DW, lane, nxt);
             // Before waiting for any ring slot: arrive on the tiles before
             // this block.  The MMA of a tile needs every warp's arrival, and
             // a slot frees only when the MMA of the tile S earlier is done.
@@ -535,26 +540,26 @@ __device__ __forceinline__ void epilogue_role(const GemmParams &p, const Roles &
     }
 }
 
-template <int C>
-__global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmParams p)
+template <int C, int DW>
+__global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const GemmParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t tid = threadIdx.x, warp = tid >> 5;
     const int lane = (int)(tid & 31u);
     const uint32_t S = p.stages;
-    uint8_t *ctrl = smem + ctrl_offset(p.cap);
+    uint8_t *ctrl = smem + ctrl_offset(p.cap, DW);
     Roles R;
     const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     R.bars = static_cast<uint32_t>(__cvta_generic_to_shared(ctrl));
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + kNumBars * 8);
     R.abort_flag = tmem_slot + 1;
     R.cover = tmem_slot + 2;
-    R.ring_a = (base + ctrl_offset(p.cap) + kCtrlBytes + 1023u) & ~1023u;
+    R.ring_a = (base + ctrl_offset(p.cap, DW) + kCtrlBytes + 1023u) & ~1023u;
     R.ring_b = R.ring_a + S * kTileBytes;
 
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
-            mbar_init(bar(R, kBarFull + s), kDecodeWarps);
+            mbar_init(bar(R, kBarFull + s), DW);
             mbar_init(bar(R, kBarEmpty + s), 1);
             mbar_init(bar(R, kBarX + s), 1);
         }
@@ -569,7 +574,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmPa
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
     }
-    if (warp == kControlWarp) {
+    if (warp == DW) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          static_cast<uint32_t>(__cvta_generic_to_shared(tmem_slot))),
                      "r"(p.tmem_cols)
@@ -579,13 +584,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmPa
     }
     // the tables (the barriers, flags and tensor-memory address above are
     // published by its __syncthreads)
-    build_tables(p.luts, p.cl, p.num_luts, smem, tid, kGemmThreads);
+    build_tables(p.luts, p.cl, p.num_luts, smem, tid, gemm_threads(DW));
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
-    if (warp < kDecodeWarps) {
-        decode_role<C>(p, R, smem, warp, lane);
-    } else if (warp == kControlWarp) {
+    if (warp < DW) {
+        decode_role<C, DW>(p, R, smem, warp, lane);
+    } else if (warp == DW) {
         if (lane == 0)
             control_role(p, R);
         __syncwarp();
@@ -594,7 +599,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmPa
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kControlWarp) {
+    if (warp == DW) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(R.tmem), "r"(p.tmem_cols)
                      : "memory");
@@ -606,7 +611,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) df11_gemm_kernel(const GemmPa
 struct GemmFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2] = {0, 0};
+    uint32_t granted[2][2] = {};  // [C - 1][16 or 20 decode warps]
 };
 std::mutex g_gemm_mu;
 GemmFacts g_gemm[64];
@@ -705,22 +710,33 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
             f->sms = sms;
         }
     }
-    // as many ring stages as fit (at least 2)
-    uint32_t stages = kMaxStages;
-    while (stages >= 2 && gemm_smem_bytes(prm.cap, batch, stages) > (uint32_t)f->smem_optin)
-        stages--;
+    // as many ring stages as fit; 20 decode warps if that leaves at least
+    // kMinStages20 stages, else 16 decode warps and at least 2 stages
+    const uint32_t optin = (uint32_t)f->smem_optin;
+    auto max_stages = [&](uint32_t dw) {
+        uint32_t st = kMaxStages;
+        while (st >= 1 && gemm_smem_bytes(prm.cap, batch, st, dw) > optin)
+            st--;
+        return st;
+    };
+    uint32_t dw = 20, stages = max_stages(20);
+    if (stages < kMinStages20) {
+        dw = 16;
+        stages = max_stages(16);
+    }
     if (stages < 2)
         return DF11_ERR_INVALID_ARG;
     prm.stages = stages;
-    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages);
-    const int ci = a->threads_per_block == 32 ? 0 : 1;
-    auto kern = ci == 0 ? df11_gemm_kernel<1> : df11_gemm_kernel<2>;
+    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages, dw);
+    const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 20 ? 1 : 0;
+    auto kern = ci == 0 ? (wi ? df11_gemm_kernel<1, 20> : df11_gemm_kernel<1, 16>)
+                        : (wi ? df11_gemm_kernel<2, 20> : df11_gemm_kernel<2, 16>);
     {
         std::lock_guard<std::mutex> lock(g_gemm_mu);
-        if (smem > f->granted[ci]) {
+        if (smem > f->granted[ci][wi]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return DF11_ERR_CUDA;
-            f->granted[ci] = smem;
+            f->granted[ci][wi] = smem;
         }
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -729,7 +745,7 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
     if (cudaGetLastError() != cudaSuccess)
         return DF11_ERR_CUDA;
     const uint32_t grid = (uint32_t)f->sms < prm.num_units ? (uint32_t)f->sms : prm.num_units;
-    kern<<<grid, kGemmThreads, smem, s>>>(prm);
+    kern<<<grid, gemm_threads(dw), smem, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 

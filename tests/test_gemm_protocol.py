@@ -4,14 +4,15 @@ on the block offsets of real tile-major streams, and must all finish (no
 deadlock) for every ring depth the launch can choose (S = 2..8).
 
 Agents (one CTA, its units in order; tiles numbered q across units):
-  * decode warp w: for each of its blocks b = first + w, first + w + 16, ...
-    of a unit: arrive on every tile before the block's first output, wait
+  * decode warp w (of 16 or 20): for each of its blocks b = first + w,
+    first + w + warps, ... of a unit: arrive on every tile before the
+    block's first output, wait
     until the ring slots of the tiles the block writes are free (the MMA of
     tile q - S is done), then arrive on every tile before its next block's
     first output; at the end of the unit, arrive on the rest;
   * control: per unit, bulk copies of the first S - 1 activation chunks
     (each once its slot is free), then the accumulator two units back must
-    have been read; per tile: wait until all 16 warps arrived and its
+    have been read; per tile: wait until all decode warps arrived and its
     activations were issued, MMA (frees the slot), issue the chunk S - 1
     ahead; then the accumulator is full;
   * epilogue: per unit, wait for the full accumulator, then free it.
@@ -26,7 +27,6 @@ import huffman_decode_03_b200 as df11
 from huffman_decode_03_b200 import inputs
 
 TILE = 8192
-WARPS = 16
 
 
 def _units(shapes):
@@ -51,8 +51,9 @@ def _block_of(offs, x):
     return lo
 
 
-def _run_cta(offs, units, S, arrive_first=True):
+def _run_cta(offs, units, S, arrive_first=True, warps=16):
     """True when every agent of a CTA that takes all `units` finishes."""
+    WARPS = warps
     full, mma_done, x_issued, acc_full, acc_free = {}, set(), set(), set(), set()
 
     def slot_free(q):
@@ -145,15 +146,16 @@ def _offsets(shapes, mats, T):
 SMALL = [(128, 64), (256, 128), (384, 1088), (128, 2048)]
 
 
+@pytest.mark.parametrize("warps", [16, 20])
 @pytest.mark.parametrize("T", [32, 64])
 @pytest.mark.parametrize("S", [2, 3, 4, 8])
-def test_protocol_finishes(T, S):
+def test_protocol_finishes(T, S, warps):
     mats = [inputs.gaussian(r * c, [73, m]) for m, (r, c) in enumerate(SMALL)]
     offs = _offsets(SMALL, mats, T)
     units = _units(SMALL)
     for grid in (1, 3, 148):  # units blockIdx.x, + grid, ... per CTA
         for cta in range(min(grid, len(units))):
-            assert _run_cta(offs, units[cta::grid], S), (grid, cta)
+            assert _run_cta(offs, units[cta::grid], S, warps=warps), (grid, cta)
 
 
 def test_arriving_only_after_the_first_block_deadlocks():
@@ -169,11 +171,12 @@ def test_arriving_only_after_the_first_block_deadlocks():
 
 @pytest.mark.slow
 def test_protocol_finishes_on_the_llama3_8b_block():
-    # the fused GEMM's workload: 1,664 units over 148 CTAs, T = 64, the ring
-    # depths of batch 256 (S = 2) and batch 64 (S = 4)
+    # the fused GEMM's workload: 1,664 units over 148 CTAs, T = 64, the
+    # launch configurations of batch 256 and 128 (16 decode warps, S = 2 and
+    # 3), 64 and 16 (20 decode warps, S = 3 and 4)
     shapes = [s for _, s in inputs.LLAMA3_8B]
     offs = _offsets(shapes, [m for _, _, m in inputs.block(2, 0)], 64)
     units = _units(shapes)
-    for S in (2, 4):
+    for warps, S in ((16, 2), (16, 3), (20, 3), (20, 4)):
         for cta in range(148):
-            assert _run_cta(offs, units[cta::148], S), (S, cta)
+            assert _run_cta(offs, units[cta::148], S, warps=warps), (warps, S, cta)
