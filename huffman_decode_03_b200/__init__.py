@@ -22,8 +22,8 @@ from . import build as _build
 
 __all__ = [
     "Df11Error", "Format", "DeviceFormat", "build_format", "decompress",
-    "decompress_gemv", "decompress_gemm", "decompress_host", "encode_device", "read_status",
-    "tile_major", "load_library",
+    "decompress_gemv", "decompress_gemm", "gemm_scratch_bytes", "decompress_host", "encode_device",
+    "read_status", "tile_major", "load_library",
 ]
 
 DF11_OK = 0
