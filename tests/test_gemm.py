@@ -45,6 +45,21 @@ def test_tile_major_order(rows, cols):
     assert t[i] == w[r * cols + c]
 
 
+def test_tile_major_stream_has_the_same_code_and_size():
+    # the element order is the compressor's choice: the histogram, and so the
+    # code, the LUTs and the compressed size, do not depend on it
+    shapes = [(256, 128), (128, 1088)]
+    mats = [inputs.gaussian(r * c, [79, m]) for m, (r, c) in enumerate(shapes)]
+    row = df11.build_format(mats)
+    tiled = df11.build_format([df11.tile_major(w, r, c) for (r, c), w in zip(shapes, mats)])
+    a, b = row.arrays(), tiled.arrays()
+    assert np.array_equal(a["code_lengths"], b["code_lengths"])
+    assert np.array_equal(a["luts"], b["luts"])
+    assert row.scalars()["total_bits"] == tiled.scalars()["total_bits"]
+    assert row.info()["compressed_bytes"] == tiled.info()["compressed_bytes"]
+    assert not np.array_equal(a["encoded_exponent"], b["encoded_exponent"])
+
+
 def test_tile_major_rejects_ragged_shapes():
     with pytest.raises(df11.Df11Error):
         df11.tile_major(np.zeros(100 * 64, np.uint16), 100, 64)
