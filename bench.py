@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 METRIC = "DF11 decompress GB/s (BF16 out) and % of HBM roofline, 1×B200, bit-exact"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, vendor figure (7.7 TB/s HGX, 8 TB/s DGX)
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAME = "df11_decode_kernel"
 # the decode kernel's source: the kernel and its shared per-block decode
@@ -58,6 +59,9 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between timed steps")
+    ap.add_argument("--per-workload", default="4,3,1",
+                    help="further workloads measured after the headline one at N=1, reported in the "
+                         "line's per_workload object (comma-separated ids, or 'none')")
     return ap.parse_args(argv)
 
 
@@ -209,7 +213,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- GPU arm
-def prepare_streams(streams, T, device, verify=True):
+def prepare_streams(streams, T, device, verify=True, pin_host=True):
     """Builds (host) and uploads each stream; checks one decode bit-exactly."""
     import torch
 
@@ -217,23 +221,118 @@ def prepare_streams(streams, T, device, verify=True):
     from huffman_decode_03_b200 import inputs
 
     out = []
-    for wl, blk in streams:
+    for i, (wl, blk) in enumerate(streams):
         mats = [m for _, _, m in inputs.workload_arrays(wl, blk)]
         fmt = df11.build_format(mats, T)
-        dev = df11.DeviceFormat(fmt, device, pin_host=True)
+        dev = df11.DeviceFormat(fmt, device, pin_host=pin_host)
         info = fmt.info()
         exact = None
+        w = torch.from_numpy(np.concatenate(mats).view(np.int16) if len(mats) > 1 else mats[0].view(np.int16))
         if verify:
-            w = torch.from_numpy(np.concatenate(mats).view(np.int16) if len(mats) > 1 else mats[0].view(np.int16))
             status = torch.zeros(1, dtype=torch.int32, device=device)
             got = df11.decompress(dev, None, status)
             ok_status = df11.read_status(status) == 0
             exact = bool(ok_status and torch.equal(got.view(torch.int16), w.to(device)))
-            del got, w
+            del got
         del mats
         fmt.free()
-        out.append({"dev": dev, "info": info, "exact": exact})
+        # the last stream's original bits stay (host) for the check after the timed loop
+        out.append({"dev": dev, "info": info, "exact": exact, "bits": w if i == len(streams) - 1 else None})
+        del w
     return out
+
+
+def time_steps(prepared, outbuf, status, stream, flush, steps, warmup, between=None):
+    """Per-step CUDA-event times (ms) of `steps` steps after `warmup` untimed
+    ones; a step decodes every prepared stream into outbuf, one launch each;
+    the L2 flush (if any) runs before each step, outside its events."""
+    import torch
+
+    import huffman_decode_03_b200 as df11
+
+    def step():
+        for p in prepared:
+            df11.decompress(p["dev"], outbuf, status, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if between:
+        between("t0")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if between:
+        between("t1")
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def last_output_exact(prepared, outbuf) -> bool:
+    """After timed steps: outbuf holds the last stream's decode; it must equal
+    that stream's original bits."""
+    import torch
+
+    p = prepared[-1]
+    n = p["info"]["n"]
+    return bool(torch.equal(outbuf[:n].view(torch.int16), p["bits"].to(outbuf.device)))
+
+
+def roofline_fraction(prepared, ms_per_launch, peak):
+    alg = sum(stream_algorithmic_bytes(p["dev"].scalars) for p in prepared) / len(prepared)
+    achieved = alg / (ms_per_launch * 1e-3) / 1e9
+    return alg, achieved, achieved / peak
+
+
+def measure_workload(wl, args, device, peak):
+    """One further workload at N=1: build, upload, check, time; its record for
+    the line's per_workload object."""
+    import torch
+
+    streams = shard(wl, 0, 1)
+    prepared = prepare_streams(streams, args.threads_per_block, device, pin_host=False)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    n_max = max(p["info"]["n"] for p in prepared)
+    outbuf = torch.empty(n_max, dtype=torch.bfloat16, device=device)
+    flush = None if args.no_flush else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    ms = time_steps(prepared, outbuf, status, stream, flush, args.steps, args.warmup)
+    import huffman_decode_03_b200 as df11
+
+    exact = all(p["exact"] for p in prepared) and df11.read_status(status) == 0 and last_output_exact(prepared,
+                                                                                                      outbuf)
+    med = float(statistics.median(ms))
+    n_total = sum(p["info"]["n"] for p in prepared)
+    per_launch = med / len(prepared)
+    alg, achieved, frac = roofline_fraction(prepared, per_launch, peak)
+    info0 = prepared[0]["info"]
+    rec = {
+        "workload": _workload_name(wl),
+        "elements": int(n_total),
+        "launches_per_step": len(prepared),
+        "ms_per_step": round(med, 5),
+        "ms_per_launch": round(per_launch, 5),
+        "value": round(2.0 * n_total / (med * 1e-3) / 1e9, 2),
+        "unit": UNIT,
+        "roofline_achieved_gbs": round(achieved, 1),
+        "frac": round(frac, 4),
+        "frac_vs_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+        "algorithmic_bytes_per_launch": int(alg),
+        "bits_per_weight": round(8 + info0["avg_code_len"], 4),
+        "max_code_len": info0["max_code_len"],
+        "num_luts": info0["num_luts"],
+        "bit_exact": bool(exact),
+        "steps": args.steps,
+        "timing": "median of per-step CUDA-event times",
+    }
+    del prepared, outbuf, flush
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_gpu(args):
@@ -255,42 +354,24 @@ def run_gpu(args):
     exact = all(p["exact"] for p in prepared)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     outbuf = torch.empty(max(p["info"]["n"] for p in prepared), dtype=torch.bfloat16, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = None if args.no_flush else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
-
-    def step():
-        for p in prepared:
-            df11.decompress(p["dev"], outbuf, status, stream)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(device)
 
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
         time.sleep(0.5)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(device)
-    if sampler:
-        sampler.mark("t0")
-    for i in range(args.steps):
-        if not args.no_flush:
-            flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(device)
-    if sampler:
-        sampler.mark("t1")
+    ms = time_steps(prepared, outbuf, status, stream, flush, args.steps, args.warmup,
+                    between=sampler.mark if sampler else None)
     if world > 1:
         dist.barrier()
-    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_med = float(statistics.median(ms))
     ms_mean = float(np.mean(ms))
-    ok = df11.read_status(status) == 0
+    # the timed launches' own result: status word, and the last stream's output
+    ok = df11.read_status(status) == 0 and last_output_exact(prepared, outbuf)
 
     # end to end through the host-buffer entry point (pinned host memory)
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
@@ -310,16 +391,17 @@ def run_gpu(args):
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     ok = ok and df11.read_status(status) == 0
+    last_n = prepared[-1]["info"]["n"]
+    ok = ok and bool(torch.equal(host_out[:last_n], prepared[-1]["bits"]))
     clocks = sampler.stop() if sampler else None
 
-    ms_step, e2e_ms, n_all, good = reduce_over_ranks(ms_mean, e2e_ms, n_total, exact and ok, device, world)
+    ms_step, e2e_ms, n_all, good = reduce_over_ranks(ms_med, e2e_ms, n_total, exact and ok, device, world)
 
     if rank == 0:
         info0 = prepared[0]["info"]
-        alg = sum(stream_algorithmic_bytes(p["dev"].scalars) for p in prepared) / len(prepared)
-        per_launch_ms = ms_mean / len(prepared)
+        per_launch_ms = ms_med / len(prepared)
         peak, peak_src = load_peak()
-        achieved = alg / (per_launch_ms * 1e-3) / 1e9
+        alg, achieved, frac = roofline_fraction(prepared, per_launch_ms, peak)
         traffic = recorded_traffic(args.workload, prepared[0]["info"]["n"])
         value = 2.0 * n_all / (ms_step * 1e-3) / 1e9
         line = {
@@ -330,6 +412,8 @@ def run_gpu(args):
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": round(ms_step, 5),
+            "ms_per_step_mean": round(ms_mean, 5),
+            "timing": "ms_per_step and value: median of the per-step CUDA-event times (max over ranks)",
             "higher_is_better": True,
             "scaling": scaling_kind(args.workload),
             "vs_baseline": None,
@@ -356,10 +440,12 @@ def run_gpu(args):
                 "achieved": round(achieved, 1),
                 "peak": peak,
                 "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
+                "frac": round(frac, 4),
                 "traffic": None if traffic is None else int(traffic),
                 "algorithmic_bytes_per_launch": int(alg),
                 "peak_source": peak_src,
+                "frac_vs_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                "nominal_peak": NOMINAL_HBM_GBS,
             },
             "e2e": {
                 "value": round(2.0 * n_all / (e2e_ms * 1e-3) / 1e9, 2),
@@ -372,6 +458,17 @@ def run_gpu(args):
             "gpu_launches": args.steps * len(prepared),
             "clocks": clocks,
         }
+    # further workloads, measured the same way, at N=1 only
+    extra = [] if args.per_workload.strip().lower() in ("", "none") else \
+        [int(x) for x in args.per_workload.split(",") if int(x) != args.workload]
+    if world == 1 and extra:
+        del prepared, outbuf, flush, host_out
+        torch.cuda.empty_cache()
+        peak, _ = load_peak()
+        per = [measure_workload(wl, args, device, peak) for wl in extra]
+        line["per_workload"] = per
+        line["gpu_launches"] += sum(r["steps"] * r["launches_per_step"] for r in per)
+    if rank == 0:
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
@@ -387,33 +484,105 @@ def _workload_name(w):
 
 
 # ------------------------------------------------------------ CPU oracle
-def _oracle_sample(workload: int, elems: int):
+def _oracle_sample(workload: int, elems: int, keep: bool = False):
     from huffman_decode_03_b200 import inputs
     from oracle import oracle
 
     mats = [m for _, _, m in inputs.workload_arrays(1 if workload == 1 else (2 if workload == 5 else workload), 0)]
     w = np.concatenate(mats) if len(mats) > 1 else mats[0]
     w = np.ascontiguousarray(w[:elems])
-    return oracle, oracle.build_format(w, 64)
+    fmt = oracle.build_format(w, 64)
+    return (oracle, fmt, w) if keep else (oracle, fmt)
+
+
+def host_cpu() -> dict:
+    """The host's CPU model and the cores this process may run on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": cores}
+
+
+CPU_BASELINE_MAX_ELEMS = 1 << 28
+
+
+def _oracle_decode_all_cores(oracle, fmt, threads: int) -> np.ndarray:
+    """The oracle's tree walk run on `threads` threads at once: each decodes
+    the exponents of a run of whole format blocks (df11o_decode_range from the
+    run's first code start to the next run's), and the BF16 values are then
+    reassembled from them and the sign/mantissa bytes.  ctypes releases the
+    GIL during the C calls."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    T = fmt["threads_per_block"]
+    offs = fmt["block_offset"]
+    gaps = fmt["gaps"]
+    nb = len(offs) - 1
+    bits = int(fmt["total_bits"])
+    out = np.empty(fmt["n"], np.uint16)
+    sm = fmt["packed_sign_mantissa"]
+    cuts = [nb * k // (4 * threads) for k in range(4 * threads + 1)]
+
+    def start(b):
+        return bits if b >= nb else 64 * T * b + int(gaps[T * b])
+
+    def work(k):
+        b0, b1 = cuts[k], cuts[k + 1]
+        if b0 == b1:
+            return
+        e = oracle.decode_range(fmt["encoded_exponent"], bits, start(b0), start(b1), fmt["code_lengths"],
+                                fmt["codes"]).astype(np.uint16)
+        o0, o1 = int(offs[b0]), int(offs[b1])
+        m = sm[o0:o1].astype(np.uint16)
+        out[o0:o1] = ((m & 0x80) << 8) | (e << 7) | (m & 0x7F)
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(len(cuts) - 1)))
+    return out
 
 
 def cpu_baseline(workload: int, seconds: float) -> dict:
-    """The oracle's bit-by-bit tree-walk decode, single thread, on a bounded
-    sample of the same workload (its leading elements), repeated for about
-    `seconds` of CPU time."""
-    elems = 1 << 22
-    oracle, fmt = _oracle_sample(workload, elems)
+    """The oracle's bit-by-bit tree-walk decode of the workload's stream
+    (the whole stream, or its first 2^28 elements; one block of the 32-block
+    workload) on the host: on one core (df11o_decode), and on every core
+    (df11o_decode_range over runs of whole blocks, one thread each); each
+    repeated for about seconds / 2."""
+    hc = host_cpu()
+    oracle, fmt, w = _oracle_sample(workload, CPU_BASELINE_MAX_ELEMS, keep=True)
     n = fmt["n"]
-    reps, t = 0, 0.0
-    while t < seconds:
-        t0 = time.perf_counter()
-        oracle.decode_format(fmt)
-        t += time.perf_counter() - t0
-        reps += 1
-    gbs = 2.0 * n * reps / t / 1e9
-    return {"value": round(gbs, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"first {n} elements of {_workload_name(workload)}, decoded {reps}x "
-                      f"({t:.1f} s) by the bit-by-bit tree walk"}
+
+    def timed(fn):
+        reps, t, exact = 0, 0.0, True
+        while reps == 0 or t < seconds / 2:
+            t0 = time.perf_counter()
+            got = fn()
+            t += time.perf_counter() - t0
+            reps += 1
+            exact = exact and np.array_equal(got, w)
+        return 2.0 * n * reps / t / 1e9, reps, t, exact
+
+    one, r1, t1, x1 = timed(lambda: oracle.decode_format(fmt))
+    allc, ra, ta, xa = timed(lambda: _oracle_decode_all_cores(oracle, fmt, hc["nproc"]))
+    what = "whole stream" if n < CPU_BASELINE_MAX_ELEMS else "first elements"
+    return {"value": round(one, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{what} of {_workload_name(workload)} ({n} elements), decoded {r1}x ({t1:.1f} s) "
+                      f"by the bit-by-bit tree walk on one core",
+            "bit_exact": bool(x1),
+            "all_cores": {"value": round(allc, 4), "unit": UNIT, "cores": hc["nproc"], "reps": ra,
+                          "seconds": round(ta, 2), "bit_exact": bool(xa),
+                          "how": "the same tree walk over runs of whole format blocks, one thread per run "
+                                 "(df11o_decode_range), BF16 reassembled per run"},
+            **hc}
 
 
 def run_reference(args):
@@ -453,7 +622,9 @@ def run_reference(args):
         "dtype": "u16",
         "data": "synthetic (seeded numpy PCG64)",
         "config": {"workload": _workload_name(args.workload), "elements_per_step": n},
-        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                         **host_cpu()},
+        "timing": "ms_per_step and value: mean of the per-step wall-clock times of the oracle decode",
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

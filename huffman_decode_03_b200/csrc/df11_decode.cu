@@ -498,7 +498,11 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
 
     // Pieces of whole format blocks, ~8 Mi outputs each: piece k's arrays go
     // up on `up`, it decodes on `s`, its outputs come down on `down`, so the
-    // copies of one piece overlap the decode of its neighbours.
+    // copies of one piece overlap the decode of its neighbours.  A piece's
+    // decode reads a few bytes past its last block (the stream's 16-byte
+    // tail, the sign/mantissa bytes up to the next 16-byte boundary); the
+    // next piece's uploads start where the previous ones ended, so no copy
+    // rewrites bytes that a running decode reads.
     const uint32_t nb = h->num_blocks;
     const uint64_t per_piece = 8ull << 20;
     uint32_t pieces = (uint32_t)((h->n + per_piece - 1) / per_piece);
@@ -521,6 +525,7 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
     };
     if (!event(&start) || !event(&done))
         return cleanup(DF11_ERR_CUDA);
+    uint64_t stream_done = 0, sm_done = 0;  // bytes uploaded so far, from 0
     bool ok = cudaEventRecord(start, s) == cudaSuccess && cudaStreamWaitEvent(up, start, 0) == cudaSuccess &&
               cudaStreamWaitEvent(down, start, 0) == cudaSuccess;
     // the small arrays whole, first
@@ -538,20 +543,25 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
         uint32_t b0 = (uint32_t)((uint64_t)nb * k / pieces), b1 = (uint32_t)((uint64_t)nb * (k + 1) / pieces);
         if (b0 == b1)
             continue;
-        // stream bytes of the blocks plus the 16 the last chain reads beyond
-        const uint64_t s0 = b0 * T * 8, s1 = std::min<uint64_t>(b1 * T * 8 + 16, h->encoded_exponent_bytes);
+        // stream bytes of the blocks plus the 16 the last chain reads beyond,
+        // from where the previous piece's upload ended
+        const uint64_t s0 = std::max<uint64_t>(b0 * T * 8, stream_done);
+        const uint64_t s1 = std::min<uint64_t>(b1 * T * 8 + 16, h->encoded_exponent_bytes);
         // the piece's outputs: BlockOffset entries clamped to n, so that a
         // corrupt host copy (which the kernel reports) cannot move a copy
         // outside the arrays
         const uint64_t e0 = std::min<uint64_t>(offs[b0], h->n), e1 = std::min<uint64_t>(offs[b1], h->n);
-        // their sign/mantissa bytes, in whole 16-byte units
-        const uint64_t m0 = e0 & ~15ull;
+        // their sign/mantissa bytes, in whole 16-byte units, from where the
+        // previous piece's upload ended
+        const uint64_t m0 = std::max<uint64_t>(e0 & ~15ull, sm_done);
         const uint64_t m1 = std::min<uint64_t>((e1 + 15ull) & ~15ull, h->packed_sign_mantissa_bytes);
         cudaEvent_t in, dec;
         if (!event(&in) || !event(&dec))
             return cleanup(DF11_ERR_CUDA);
-        ok = cudaMemcpyAsync(const_cast<uint8_t *>(d->encoded_exponent) + s0, h->encoded_exponent + s0, s1 - s0,
-                             cudaMemcpyHostToDevice, up) == cudaSuccess;
+        ok = s1 <= s0 || cudaMemcpyAsync(const_cast<uint8_t *>(d->encoded_exponent) + s0, h->encoded_exponent + s0,
+                                         s1 - s0, cudaMemcpyHostToDevice, up) == cudaSuccess;
+        stream_done = std::max(stream_done, s1);
+        sm_done = std::max(sm_done, m1);
         ok = ok && (m1 <= m0 || cudaMemcpyAsync(const_cast<uint8_t *>(d->packed_sign_mantissa) + m0,
                                                 h->packed_sign_mantissa + m0, m1 - m0, cudaMemcpyHostToDevice,
                                                 up) == cudaSuccess);

@@ -433,20 +433,30 @@ constexpr uint64_t kStaticMaxChunks = 1ull << 16;
 static __device__ __align__(256) uint64_t g_static_scratch[kStaticMaxChunks + 1];
 
 std::mutex g_static_mu;
-uint64_t *g_static_addr[64] = {};  // per device, looked up once
+uint64_t *g_static_addr[64] = {};  // per device, the last address looked up
 
-df11_status static_scratch(uint64_t **out)
+// The array's device address on the current device.  It is looked up again
+// on every call made while `s` is not being captured, so that a device reset
+// (which reloads the module and may move the array) is picked up; a call
+// made during a capture reuses the device's last looked-up address and fails
+// with DF11_ERR_CUDA if there is none yet.
+df11_status static_scratch(cudaStream_t s, uint64_t **out)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return DF11_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess)
+        return DF11_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *addr = nullptr;
         if (cudaGetSymbolAddress(&addr, g_static_scratch) != cudaSuccess || !addr)
             return DF11_ERR_CUDA;
         g_static_addr[dev] = static_cast<uint64_t *>(addr);
     }
+    if (!g_static_addr[dev])
+        return DF11_ERR_CUDA;
     *out = g_static_addr[dev];
     return DF11_OK;
 }
@@ -560,7 +570,7 @@ extern "C" df11_status df11_device_encode_static(const df11_format *plan, const 
     if (df11_device_encode_scratch_words(a.n) > kStaticMaxChunks + 1)
         return DF11_ERR_TOO_LARGE;  // more than 2^29 elements
     uint64_t *scratch = nullptr;
-    const df11_status st = static_scratch(&scratch);
+    const df11_status st = static_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch);
     if (st != DF11_OK)
         return st;
     return df11_device_encode(plan, w_dev, dst, scratch, kStaticMaxChunks + 1, max_block_dev, status_dev, stream);

@@ -388,9 +388,12 @@ df11_status df11_device_encode(const df11_format *plan, const uint16_t *w_dev, c
  * (on other streams or from other threads) race on it and must be
  * serialised by the caller.  No entry of it has to start at zero (a call
  * writes every entry it reads before reading it), so it is never cleared.
- * The first call on a device looks up the array's address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  DF11_ERR_CUDA if the lookup fails.
+ * Each call made while `stream` is not being captured looks up the array's
+ * address on the current device (cudaGetSymbolAddress), so a device reset
+ * between calls, which may move the array, is picked up.  A call made while
+ * `stream` is being captured reuses the last address looked up on that
+ * device; make the first call on a device before any stream capture.
+ * DF11_ERR_CUDA if the lookup fails or no address has been looked up yet.
  */
 df11_status df11_device_encode_static(const df11_format *plan, const uint16_t *w_dev, const df11_arrays *dst_dev,
                                       uint32_t *max_block_elems_dev, uint32_t *status_dev, void *stream);

@@ -87,3 +87,20 @@ def test_algorithmic_bytes_of_a_stream():
         + 4 * (s["num_blocks"] + 1) + 256 * (s["num_luts"] + 1)
     assert 3 * n + bits / 8 < got < 3 * n + bits / 8 + 4 * (s["num_blocks"] + 1) + 256 * 18 + 2
     assert 3.3 < got / n < 3.4  # ~2.6 code bits + 0.08 Gaps bits per element on N(0, 0.02)
+
+
+def test_all_core_oracle_baseline_rebuilds_the_stream(oracle_mod):
+    # the all-core CPU baseline splits one stream at format-block boundaries
+    # (each run from its first code start to the next run's) and must give
+    # back every element, for several run counts and both block sizes
+    for T in (32, 64):
+        w = inputs.stress(300_001, key=(41, T))
+        fmt = oracle_mod.build_format(w, T)
+        for threads in (1, 3, 8):
+            got = bench._oracle_decode_all_cores(oracle_mod, fmt, threads)
+            assert np.array_equal(got, w)
+
+
+def test_host_cpu_record():
+    rec = bench.host_cpu()
+    assert rec["nproc"] >= 1 and isinstance(rec["cpu_model"], str) and rec["cpu_model"]
