@@ -65,7 +65,7 @@ class df11_arrays(ctypes.Structure):
         ("num_luts", ctypes.c_uint32),
         ("max_code_len", ctypes.c_uint32),
         ("max_block_elems", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("min_code_len", ctypes.c_uint32),
         ("encoded_exponent", ctypes.c_void_p),
         ("encoded_exponent_bytes", ctypes.c_uint64),
         ("packed_sign_mantissa", ctypes.c_void_p),
@@ -232,7 +232,7 @@ class Format:
         a = self.c_arrays
         return {f: int(getattr(a, f)) for f in (
             "n", "total_bits", "num_segments", "threads_per_block", "num_blocks", "num_luts",
-            "max_code_len", "max_block_elems")}
+            "max_code_len", "max_block_elems", "min_code_len")}
 
 
 def build_format(mats: Sequence[np.ndarray] | np.ndarray, threads_per_block: int = 64) -> Format:

@@ -10,8 +10,8 @@
 // memory, a dot product, a tensor-core operand tile) is up to the kernel.
 //
 // A kernel's parameter struct P provides: stream, sm, gaps (uint32 halves of
-// the Gaps words), offs, luts, cl, status, n, total_bits, nseg, num_luts and
-// cap (bytes of one warp's exponent buffer).
+// the Gaps words), offs, luts, cl, status, n, total_bits, nseg, nblocks,
+// num_luts, min_code_len and cap (bytes of one warp's exponent buffer).
 #pragma once
 
 #include "df11.h"
@@ -27,11 +27,16 @@ constexpr int kIdxBits = 12;  // index width of the derived table
 constexpr int kIdxEntries = 1 << kIdxBits;
 constexpr int kLutBytes = DF11_MAX_LUTS * 256;
 constexpr uint32_t kPointerBase = 240;
-constexpr uint32_t kSlotStride = 68;  // bytes per lane's staging slot (64 codes + 2 spill + 2)
+// bytes per lane's staging slot: codes start at most every lmin bits of a
+// 64-bit segment, plus two zero-fill codes and the two bytes the decode
+// loop's last 3-byte store may write past its codes: 36 when the shortest
+// code has >= 2 bits, 68 otherwise (both odd word counts, so the 32 lanes'
+// slots start in 32 distinct banks)
+constexpr uint32_t kSlotShort = 36, kSlotLong = 68;
 // per warp: two chains x 32 lanes, plus 32 bytes so that a chain of
-// inconsistent data (up to 95 one-bit codes + 2 spill bytes) stays inside the
-// warp's own slots; such a block is reported and writes nothing
-constexpr uint32_t kSlotBytes = 2 * 32 * kSlotStride + 32;
+// inconsistent data stays inside the warp's own slots; such a block is
+// reported and writes nothing
+__host__ __device__ constexpr uint32_t slot_bytes(uint32_t stride) { return 2 * 32 * stride + 32; }
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
@@ -43,11 +48,18 @@ struct Smem {
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
     static constexpr uint32_t zq = cl + 256;                 // uint8[16]
     static constexpr uint32_t bufs = zq + 16;
-    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap) { return cap + kSlotBytes; }
-    __host__ __device__ static constexpr uint32_t bytes(uint32_t cap, uint32_t warps) { return bufs + warps * per_warp(cap); }
+    __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap, uint32_t stride)
+    {
+        return cap + slot_bytes(stride);
+    }
+    __host__ __device__ static constexpr uint32_t bytes(uint32_t cap, uint32_t warps, uint32_t stride)
+    {
+        return bufs + warps * per_warp(cap, stride);
+    }
 };
 static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
-static_assert(kSlotBytes % 16 == 0, "slots keep the buffers 16-byte aligned");
+static_assert(slot_bytes(kSlotShort) % 16 == 0 && slot_bytes(kSlotLong) % 16 == 0,
+              "slots keep the buffers 16-byte aligned");
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
@@ -211,15 +223,17 @@ struct BlockRegs {
 template <int C, class P>
 __device__ __forceinline__ void load_block(const P &p, uint32_t b, int lane, BlockRegs<C> &r)
 {
+    // segment seg = 32 (C b + k) + lane: its 12 stream bytes at 8 seg; its
+    // Gap field and the next one are Gaps bits [5 seg, 5 seg + 10), which
+    // start in 32-bit word 5 (C b + k) + (5 lane >> 5), at bit 5 lane mod 32
+    const uint8_t *s = p.stream + 8ull * ((uint64_t)b * (32 * C) + (uint32_t)lane);
+    const uint32_t *g = p.gaps + (uint64_t)(5 * C) * b + ((5u * (uint32_t)lane) >> 5);
 #pragma unroll
     for (int k = 0; k < C; k++) {
-        const uint64_t seg = (uint64_t)b * (32 * C) + lane + 32 * k;
-        const uint8_t *s = p.stream + 8 * seg;
-        r.s01[k] = __ldg(reinterpret_cast<const uint2 *>(s));
-        r.s2[k] = __ldg(reinterpret_cast<const uint32_t *>(s + 8));
-        const uint64_t w = (5 * seg) >> 5;
-        r.g0[k] = __ldg(p.gaps + w);
-        r.g1[k] = __ldg(p.gaps + w + 1);
+        r.s01[k] = __ldg(reinterpret_cast<const uint2 *>(s + 256 * k));
+        r.s2[k] = __ldg(reinterpret_cast<const uint32_t *>(s + 256 * k + 8));
+        r.g0[k] = __ldg(g + 5 * k);
+        r.g1[k] = __ldg(g + 5 * k + 1);
     }
     r.o0 = __ldg(p.offs + b);
     r.o1 = __ldg(p.offs + b + 1);
@@ -273,7 +287,8 @@ __device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32
 }
 
 // Places every chain's staging slot in the write buffer with 32-bit stores
-// only; valid when every chain of the block holds >= 3 codes.  Chain c covers
+// only; valid when every chain of the block holds >= 3 codes.  Chain B's slot
+// must lie 32 slots after chain A's.  Chain c covers
 // bytes [s_c, s_c + cnt_c) of the buffer.  It writes the words from the one
 // holding s_c up to, not including, the word that holds its own last byte
 // (the next chain writes that one); the block's last chain also writes its
@@ -282,7 +297,7 @@ __device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32
 // as one word and passes it on by shuffle.  src[k]: the chain's slot (4-byte
 // aligned shared address); s[k]: its byte offset in the buffer at shared
 // address exp_base.
-template <int C>
+template <int C, uint32_t SLOT>
 __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[2], const uint32_t src[2],
                                             const uint32_t cnt[2], int lane)
 {
@@ -300,27 +315,55 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
         if (lane == 0)
             prev[1] = x;
     }
-    uint32_t dst[2] = {0u, 0u}, sa[2] = {0u, 0u}, nw[2] = {0u, 0u}, sh[2] = {0u, 0u};
+    uint32_t dst[2] = {0u, 0u}, nw[2] = {0u, 0u}, sh[2] = {0u, 0u};
 #pragma unroll
     for (int k = 0; k < C; k++) {
         const uint32_t e = s[k] + cnt[k];
         const bool final_chain = lane == 31 && k == C - 1;
         dst[k] = exp_base + (s[k] & ~3u);
-        sa[k] = src[k];
         nw[k] = (final_chain ? (e + 3u) >> 2 : e >> 2) - (s[k] >> 2);
         sh[k] = 8u * (s[k] & 3u);
     }
-    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
-    for (uint32_t w = 0; w < nmax; w++) {
-#pragma unroll
-        for (int k = 0; k < C; k++) {
-            if (w < nw[k]) {
-                const uint32_t cur = ld_u32(sa[k] + 4 * w);
-                st_u32(dst[k] + 4 * w, __funnelshift_l(prev[k], cur, sh[k]));
-                prev[k] = cur;
-            }
-        }
-    }
+    // words i and i + 1 of each chain per pass: slot word i (chain B's slot
+    // lies 32 slots after chain A's) funnel-shifted with the word before it,
+    // predicated per chain and word, no divergent branch inside
+    const int nw1m[2] = {(int)nw[0] - 1, (int)nw[1] - 1};
+    uint32_t sa = src[0], i = 0;
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p0, p1, r0, r1, pz;\n\t"
+        ".reg .u32 c0, c1, d0, d1, w0, w1;\n\t"
+        "PW_TOP:\n\t"
+        "setp.lt.u32 p0, %5, %6;\n\t"
+        "setp.lt.u32 p1, %5, %7;\n\t"
+        "or.pred pz, p0, p1;\n\t"
+        "@!pz bra PW_END;\n\t"
+        "setp.lt.s32 r0, %5, %11;\n\t"
+        "setp.lt.s32 r1, %5, %12;\n\t"
+        "@p0 ld.shared.u32 c0, [%4];\n\t"
+        "@p1 ld.shared.u32 c1, [%4+%10];\n\t"
+        "@r0 ld.shared.u32 d0, [%4+4];\n\t"
+        "@r1 ld.shared.u32 d1, [%4+%10+4];\n\t"
+        "@p0 shf.l.clamp.b32 w0, %0, c0, %8;\n\t"
+        "@p1 shf.l.clamp.b32 w1, %1, c1, %9;\n\t"
+        "@p0 st.shared.u32 [%2], w0;\n\t"
+        "@p1 st.shared.u32 [%3], w1;\n\t"
+        "@r0 shf.l.clamp.b32 w0, c0, d0, %8;\n\t"
+        "@r1 shf.l.clamp.b32 w1, c1, d1, %9;\n\t"
+        "@r0 st.shared.u32 [%2+4], w0;\n\t"
+        "@r1 st.shared.u32 [%3+4], w1;\n\t"
+        "mov.b32 %0, d0;\n\t"
+        "mov.b32 %1, d1;\n\t"
+        "add.u32 %4, %4, 8;\n\t"
+        "add.u32 %2, %2, 8;\n\t"
+        "add.u32 %3, %3, 8;\n\t"
+        "add.u32 %5, %5, 2;\n\t"
+        "bra PW_TOP;\n\t"
+        "PW_END:\n\t"
+        "}"
+        : "+r"(prev[0]), "+r"(prev[1]), "+r"(dst[0]), "+r"(dst[1]), "+r"(sa), "+r"(i)
+        : "r"(nw[0]), "r"(nw[1]), "r"(sh[0]), "r"(sh[1]), "n"(32 * SLOT), "r"(nw1m[0]), "r"(nw1m[1])
+        : "memory");
 }
 
 // Once per CTA, called by all its nthreads threads (tid = thread index): the
@@ -397,7 +440,7 @@ struct BlockOut {
 // sign/mantissa bytes first.  Returns false, after setting DF11_ERR_CORRUPT
 // in *p.status, when the block is inconsistent (nothing placed).  Called by
 // all 32 lanes of the warp.
-template <int C, class P>
+template <int C, uint32_t SLOT, class P>
 __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, const BlockRegs<C> &cur,
                                              const uint8_t *luts, const uint8_t *cl, const uint8_t *zq,
                                              uint32_t sym_base, uint32_t exp_base, uint32_t slot_base, BlockOut &out)
@@ -413,28 +456,39 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
     if (nbytes && lane == 0)
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + g0), "r"(nbytes) : "memory");
 
-    // ---- locate: chain k's codes start in [pos0, pend) of its window
+    // ---- locate: chain k's codes start in [pos0, pend) of its window.  In
+    // every block but the stream's last, every segment has a successor, so
+    // pend = 64 + the next Gap and only the window's third word holds bits
+    // past it; the last block checks segments against the stream's end.
     bool bad = false;
     int pos0[2] = {0, 0}, pend[2] = {0, 0};
     uint32_t h[2] = {0u, 0u}, m[2] = {0u, 0u}, l[2] = {0u, 0u};
+    const uint32_t goff = (5u * (uint32_t)lane) & 31u;
+    const bool last_block = b + 1 >= p.nblocks;  // warp-uniform
 #pragma unroll
     for (int k = 0; k < C; k++) {
-        const uint64_t seg = (uint64_t)b * T + lane + 32 * k;
-        const uint32_t off = (uint32_t)((5 * seg) & 31);
-        const uint64_t v = (((uint64_t)cur.g1[k] << 32) | cur.g0[k]) >> off;
-        const uint32_t gap = (uint32_t)v & 31u, gap_next = (uint32_t)(v >> 5) & 31u;
-        if (seg < p.nseg) {
-            pos0[k] = (int)gap;
-            pend[k] = seg + 1 < p.nseg ? 64 + (int)gap_next : (int)(p.total_bits - 64 * seg);
-        }
+        const uint32_t v = __funnelshift_r(cur.g0[k], cur.g1[k], goff);
+        const uint32_t gap = v & 31u, gap_next = (v >> 5) & 31u;
         h[k] = bswap32(cur.s01[k].x);
         m[k] = bswap32(cur.s01[k].y);
         l[k] = bswap32(cur.s2[k]);
-        // bits from pend on belong to the next chain: zeros instead
-        const uint32_t pe = (uint32_t)pend[k];
-        h[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe);
-        m[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 32u ? pe - 32u : 0u);
-        l[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 64u ? pe - 64u : 0u);
+        if (!last_block) {
+            pos0[k] = (int)gap;
+            pend[k] = 64 + (int)gap_next;
+            l[k] &= ~(0xFFFFFFFFu >> gap_next);
+        } else {
+            const uint32_t seg = b * T + (uint32_t)lane + 32u * k;
+            const uint32_t nseg = (uint32_t)p.nseg;
+            if (seg < nseg) {
+                pos0[k] = (int)gap;
+                pend[k] = seg + 1 < nseg ? 64 + (int)gap_next : (int)((uint32_t)p.total_bits - 64u * seg);
+            }
+            // bits from pend on belong to the next chain: zeros instead
+            const uint32_t pe = (uint32_t)pend[k];
+            h[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe);
+            m[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 32u ? pe - 32u : 0u);
+            l[k] &= ~__funnelshift_rc(0xFFFFFFFFu, 0u, pe > 64u ? pe - 64u : 0u);
+        }
         shift_window(h[k], m[k], l[k], (uint32_t)pos0[k]);
     }
 
@@ -450,7 +504,7 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
         int pos[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
-            q0[k] = slot_base + k * (32 * kSlotStride);
+            q0[k] = slot_base + k * (32 * SLOT);
             q[k] = q0[k];
             pos[k] = pos0[k];
         }
@@ -517,13 +571,13 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
     // when every chain holds >= 3 codes (the normal case), else
     // with single bytes at the chains' edges
     {
-        const uint32_t srcs[2] = {slot_base, slot_base + 32 * kSlotStride};
+        const uint32_t srcs[2] = {slot_base, slot_base + 32 * SLOT};
         bool short_chain = cnt[0] < 3u;
         if (C == 2)
             short_chain |= cnt[1] < 3u;
         if (!__any_sync(0xffffffffu, short_chain)) {
             const uint32_t offs2[2] = {lo_off + first[0], lo_off + first[1]};
-            place_words<C>(exp_base, offs2, srcs, cnt, lane);
+            place_words<C, SLOT>(exp_base, offs2, srcs, cnt, lane);
         } else {
             const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
             copy_slots2(dsts, srcs, cnt);
@@ -578,6 +632,7 @@ df11_status stream_params(const df11_arrays *a, uint32_t *status_dev, P &prm)
     prm.nseg = nseg;
     prm.nblocks = a->num_blocks;
     prm.num_luts = a->num_luts;
+    prm.min_code_len = a->min_code_len <= 32 ? a->min_code_len : 0u;
     // the per-warp buffers of 8 warps hold the 8 KB set-up scratch table
     prm.cap = align16(a->max_block_elems + 32);
     return DF11_OK;

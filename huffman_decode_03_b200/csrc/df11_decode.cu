@@ -98,6 +98,7 @@ struct Params {
     uint32_t cap;  // bytes of one warp's exponent (and sign/mantissa) buffer
     uint32_t wide;  // dst is 32-byte aligned: the merge uses 32-byte stores
     uint32_t max_ctas;  // 0 = one CTA on every SM
+    uint32_t min_code_len;  // from the stream's arrays: 0 when not known
     uint32_t num_mats;  // fused matrix-vector product (MODE 1) only
     GemvMat mats[kMaxGemvMats];
 };
@@ -216,42 +217,139 @@ __device__ __forceinline__ void gemv_block(const Params &p, uint64_t g0, uint32_
     }
 }
 
+// A warp's copy of one format block's metadata in shared memory (byte
+// offsets): the stream bytes of its 32 C segments plus the 16 the last chain
+// reads beyond, the 5 C + 1 Gaps words holding its fields and the next
+// block's first, and its two BlockOffset entries.
+template <int C>
+struct NextBuf {
+    static constexpr uint32_t stream = 0;
+    static constexpr uint32_t gaps = 256 * C + 16;
+    static constexpr uint32_t offs = (gaps + 4 * (5 * C + 1) + 7) & ~7u;  // read as one 8-byte word
+    static constexpr uint32_t bytes = (offs + 8 + 15) & ~15u;
+    // 16-byte cp.async targets at multiples of 16, the 8-byte load at a multiple of 8
+    static_assert(stream % 16 == 0 && gaps % 16 == 0 && offs % 8 == 0 && bytes % 16 == 0, "alignment");
+};
+
+// Asynchronous copy (cp.async, no registers held) of format block b's
+// metadata into the warp's buffer at shared address buf; every lane of the
+// warp takes part, one commit group per block.  The stream bytes go in
+// 16-byte pieces (the stream array is 16-byte aligned and padded by 16
+// bytes), Gaps and BlockOffset words in 4-byte pieces: every source lies
+// inside its array (checked by stream_params on the host).
+template <int C>
+__device__ __forceinline__ void prefetch_block(const Params &p, uint32_t b, int lane, uint32_t buf)
+{
+    const uint8_t *st = p.stream + (uint64_t)(256 * C) * b;
+    if (lane < 16 * C)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(buf + 16u * lane), "l"(st + 16 * lane)
+                     : "memory");
+    if (lane == 31)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(buf + 256u * C), "l"(st + 256 * C)
+                     : "memory");
+    const uint32_t *g = p.gaps + (uint64_t)(5 * C) * b;
+    if (lane <= 5 * C)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(buf + NextBuf<C>::gaps + 4u * lane),
+                     "l"(g + lane)
+                     : "memory");
+    if (lane >= 30)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(buf + NextBuf<C>::offs + 4u * (lane - 30)),
+                     "l"(p.offs + b + (lane - 30))
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// The registers of one block (what load_block would load) from the warp's
+// buffer, once its copy has landed; the buffer is free again on return.
+template <int C>
+__device__ __forceinline__ void read_block(uint32_t buf, int lane, BlockRegs<C> &r)
+{
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    const uint32_t L = (5u * (uint32_t)lane) >> 5;
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+        const uint32_t a = buf + 8u * (lane + 32 * k);
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.s01[k].x), "=r"(r.s01[k].y) : "r"(a));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r.s2[k]) : "r"(a + 8));
+        const uint32_t ga = buf + NextBuf<C>::gaps + 4u * (5 * k + L);
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r.g0[k]) : "r"(ga));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r.g1[k]) : "r"(ga + 4));
+    }
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.o0), "=r"(r.o1) : "r"(buf + NextBuf<C>::offs));
+    __syncwarp();
+}
+
+// Per-warp shared memory of a launch: the write buffer, the staging slots
+// and, with short slots, the metadata buffer of the next block.
+template <int C, uint32_t SLOT>
+__host__ __device__ constexpr uint32_t warp_bytes(uint32_t cap)
+{
+    return Smem::per_warp(cap, SLOT) + (SLOT == kSlotShort ? NextBuf<C>::bytes : 0u);
+}
+
 // C = segments per lane: the format block is 32 * C segments, one warp; lane
 // l decodes segments l, l + 32, ... as C independent chains.  WARPS warps per
-// CTA, one CTA per SM.
+// CTA, one CTA per SM.  SLOT: bytes of a chain's staging slot (kSlotShort
+// when no code is 1 bit long; the kernel checks that and reports
+// DF11_ERR_CORRUPT otherwise); with short slots the next block's metadata is
+// copied into shared memory by cp.async, with long slots it is loaded into
+// registers.
 // MODE 0: store the BF16 outputs; MODE 1: fused matrix-vector product.
-template <int C, int WARPS, int MODE>
+template <int C, int WARPS, int MODE, uint32_t SLOT>
 __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params p)
 {
     static_assert(C == 1 || C == 2, "one or two chains per lane");
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
+    constexpr bool kCopy = SLOT == kSlotShort;  // metadata by cp.async
     extern __shared__ __align__(128) uint8_t smem[];
     const uint8_t *luts = smem + Smem::luts;
     const uint8_t *cl = smem + Smem::cl;
     const uint8_t *zq = smem + Smem::zq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
+    uint8_t *exp_s = smem + Smem::bufs + warp * warp_bytes<C, SLOT>(p.cap);
     uint8_t *slots = exp_s + p.cap;
+    const uint32_t nbuf = static_cast<uint32_t>(__cvta_generic_to_shared(slots + slot_bytes(SLOT)));
 
-    // the first block's registers load while the tables are built
+    // with long slots the first block's registers load while the tables are built
     const uint32_t stride = gridDim.x * kWarps;
     uint32_t b = blockIdx.x * kWarps + warp;
     BlockRegs<C> cur, nxt;
-    if (b < p.nblocks)
+    if (!kCopy && b < p.nblocks)
         load_block<C>(p, b, lane, cur);
 
     build_tables(p.luts, p.cl, p.num_luts, smem, (uint32_t)tid, (uint32_t)kThreads);
+    if (SLOT < kSlotLong) {
+        // short slots hold a segment's codes only when no code is 1 bit long
+        // (the all-zero code is the shortest: canonical codes)
+        bool bad = false;
+        const uint32_t lmin = lut_decode(0u, luts, cl, p.num_luts, &bad) >> 8;
+        if (bad || lmin < 2) {
+            if (tid == 0)
+                atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+            return;
+        }
+    }
+    // with short slots the first block's metadata is copied only now: the
+    // table set-up used the start of the per-warp buffers as scratch
+    if (kCopy && b < p.nblocks)
+        prefetch_block<C>(p, b, lane, nbuf);
 
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
-    const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * kSlotStride;
+    const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * SLOT;
 
     // ---- each warp walks its own blocks; no block-wide barrier from here on
     for (; b < p.nblocks; b += stride) {
-        if (b + stride < p.nblocks)
+        if (kCopy) {
+            read_block<C>(nbuf, lane, cur);
+            if (b + stride < p.nblocks)
+                prefetch_block<C>(p, b + stride, lane, nbuf);
+        } else if (b + stride < p.nblocks) {
             load_block<C>(p, b + stride, lane, nxt);
+        }
         BlockOut bo;
-        if (decode_block<C>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
+        if (decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
             // ---- merge with sign/mantissa (from L2)
             const uint64_t g0 = bo.g0;
             const uint32_t lo_off = bo.lo_off, hi = bo.hi;
@@ -309,7 +407,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             }
             __syncwarp();
         }
-        cur = nxt;
+        if (!kCopy)
+            cur = nxt;
     }
 }
 
@@ -320,7 +419,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 struct DeviceFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][2][4] = {};  // [MODE][C - 1][warps 32 / 24 / 16 / 8]
+    uint32_t granted[2][2][2][4] = {};  // [MODE][C - 1][short slots][warps 32 / 24 / 16 / 8]
     cudaStream_t up = nullptr, down = nullptr;  // copy streams of the host path, made on first use
 };
 std::mutex g_mu;
@@ -345,10 +444,10 @@ df11_status device_facts(DeviceFacts **out)
     return DF11_OK;
 }
 
-template <int C, int WARPS, int MODE>
+template <int C, int WARPS, int MODE, uint32_t SLOT>
 df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, DeviceFacts *f, uint32_t &granted)
 {
-    auto kern = df11_decode_kernel<C, WARPS, MODE>;
+    auto kern = df11_decode_kernel<C, WARPS, MODE, SLOT>;
     if (smem > granted) {
         std::lock_guard<std::mutex> lock(g_mu);
         if (smem > granted) {
@@ -371,6 +470,24 @@ df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, 
 
 // As many warps per CTA (32, 24, 16 or 8) as the per-warp buffers allow in
 // shared memory; blocks of very short codes hold up to 64 outputs per segment.
+// Short staging slots when the stream states that no code is 1 bit long.
+template <int C, int MODE, uint32_t SLOT>
+df11_status launch_slots(const Params &prm, cudaStream_t stream, DeviceFacts *f)
+{
+    const uint32_t optin = (uint32_t)f->smem_optin;
+    auto &g = f->granted[MODE][C - 1][SLOT == kSlotShort ? 1 : 0];
+    const uint32_t wb = warp_bytes<C, SLOT>(prm.cap);
+    if (Smem::bufs + 32 * wb <= optin)
+        return launch_warps<C, 32, MODE, SLOT>(prm, stream, Smem::bufs + 32 * wb, f, g[0]);
+    if (Smem::bufs + 24 * wb <= optin)
+        return launch_warps<C, 24, MODE, SLOT>(prm, stream, Smem::bufs + 24 * wb, f, g[1]);
+    if (Smem::bufs + 16 * wb <= optin)
+        return launch_warps<C, 16, MODE, SLOT>(prm, stream, Smem::bufs + 16 * wb, f, g[2]);
+    if (Smem::bufs + 8 * wb <= optin)
+        return launch_warps<C, 8, MODE, SLOT>(prm, stream, Smem::bufs + 8 * wb, f, g[3]);
+    return DF11_ERR_INVALID_ARG;
+}
+
 template <int C, int MODE>
 df11_status launch(const Params &prm, cudaStream_t stream)
 {
@@ -378,16 +495,8 @@ df11_status launch(const Params &prm, cudaStream_t stream)
     df11_status st = device_facts(&f);
     if (st != DF11_OK)
         return st;
-    const uint32_t optin = (uint32_t)f->smem_optin;
-    if (Smem::bytes(prm.cap, 32) <= optin)
-        return launch_warps<C, 32, MODE>(prm, stream, Smem::bytes(prm.cap, 32), f, f->granted[MODE][C - 1][0]);
-    if (Smem::bytes(prm.cap, 24) <= optin)
-        return launch_warps<C, 24, MODE>(prm, stream, Smem::bytes(prm.cap, 24), f, f->granted[MODE][C - 1][1]);
-    if (Smem::bytes(prm.cap, 16) <= optin)
-        return launch_warps<C, 16, MODE>(prm, stream, Smem::bytes(prm.cap, 16), f, f->granted[MODE][C - 1][2]);
-    if (Smem::bytes(prm.cap, 8) <= optin)
-        return launch_warps<C, 8, MODE>(prm, stream, Smem::bytes(prm.cap, 8), f, f->granted[MODE][C - 1][3]);
-    return DF11_ERR_INVALID_ARG;
+    return prm.min_code_len >= 2 ? launch_slots<C, MODE, kSlotShort>(prm, stream, f)
+                                 : launch_slots<C, MODE, kSlotLong>(prm, stream, f);
 }
 
 }  // namespace

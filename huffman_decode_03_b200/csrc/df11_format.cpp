@@ -209,6 +209,16 @@ void canonical_codes(const uint8_t *len, uint32_t *code)
     }
 }
 
+// Length of the shortest code (0 when no symbol has a code).
+uint32_t shortest_code(const uint8_t *len)
+{
+    uint32_t m = 0;
+    for (int s = 0; s < kSymbols; s++)
+        if (len[s] && (m == 0 || len[s] < m))
+            m = len[s];
+    return m;
+}
+
 // ------------------------------------------------------------------- LUTs
 // Height-8 subtrees as 256-entry tables, built from the code values: a code
 // of length l with 8m < l <= 8(m+1) fills 2^(8(m+1)-l) entries of the table
@@ -474,7 +484,7 @@ extern "C" df11_status df11_build_format(const uint16_t *const *mats, const uint
         a.num_blocks = (uint32_t)nblocks;
         a.max_code_len = (uint32_t)longest;
         a.max_block_elems = max_block;
-        a.reserved = 0;
+        a.min_code_len = shortest_code(f->code_lengths);
         a.encoded_exponent = f->stream.data();
         a.encoded_exponent_bytes = f->stream.size();
         a.packed_sign_mantissa = f->sm.data();
@@ -550,7 +560,7 @@ extern "C" df11_status df11_plan_from_histogram(const uint64_t *hist, uint32_t T
         a.num_blocks = (uint32_t)nblocks;
         a.max_code_len = (uint32_t)longest;
         a.max_block_elems = 0;  // known once the elements are encoded
-        a.reserved = 0;
+        a.min_code_len = shortest_code(f->code_lengths);
         a.encoded_exponent = nullptr;
         a.encoded_exponent_bytes = nblocks * T * 8 + 16;
         a.packed_sign_mantissa = nullptr;

@@ -109,6 +109,7 @@ struct GemmParams {
     uint32_t nblocks;
     uint32_t num_luts;
     uint32_t cap;
+    uint32_t min_code_len;  // from the stream's arrays: 0 when not known
     // the product
     uint32_t batch;      // N of the MMA
     uint32_t stages;     // S, operand tiles in the ring
@@ -121,16 +122,17 @@ struct GemmParams {
     GemmMat mats[kMaxGemmMats];
 };
 
-__host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap, uint32_t dw)
+__host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap, uint32_t dw, uint32_t slot)
 {
-    return align16(Smem::bufs + dw * Smem::per_warp(cap));
+    return align16(Smem::bufs + dw * Smem::per_warp(cap, slot));
 }
 
 // Dynamic shared memory of a launch: tables, decode buffers, control area,
 // 1 KB to align the ring, the ring.
-__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages, uint32_t dw)
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages, uint32_t dw,
+                                                      uint32_t slot)
 {
-    return ctrl_offset(cap, dw) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
+    return ctrl_offset(cap, dw, slot) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: BF16 A and B, both
@@ -327,19 +329,19 @@ struct Roles {
 __device__ __forceinline__ uint32_t bar(const Roles &R, uint32_t i) { return R.bars + 8 * i; }
 
 // Decode warp: every unit of the CTA, blocks warp, warp + DW, ... of it.
-template <int C, int DW>
+template <int C, int DW, uint32_t SLOT>
 __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R, uint8_t *smem, uint32_t warp,
                                             int lane)
 {
     const uint32_t S = p.stages;
-    uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap);
+    uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap, SLOT);
     const uint8_t *luts = smem + Smem::luts;
     const uint8_t *cl = smem + Smem::cl;
     const uint8_t *zq = smem + Smem::zq;
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base =
-        static_cast<uint32_t>(__cvta_generic_to_shared(exp_s + p.cap)) + (uint32_t)lane * kSlotStride;
+        static_cast<uint32_t>(__cvta_generic_to_shared(exp_s + p.cap)) + (uint32_t)lane * SLOT;
 
     uint32_t q0 = 0, k = 0;  // tile sequence number of the unit's first tile; unit count
     // waits until tile q's ring slot is free (the MMA of tile q - S is done)
@@ -385,7 +387,7 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
             if (!ok)
                 break;
             BlockOut bo;
-            if (decode_block<C>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
+            if (decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
                 // the block's outputs inside the unit: [lo, hi) relative to g0
                 const uint64_t g0 = bo.g0;
                 const uint32_t lo = (uint32_t)(g0 + bo.lo_off < e0 ? e0 - g0 : bo.lo_off);
@@ -540,21 +542,21 @@ __device__ __forceinline__ void epilogue_role(const GemmParams &p, const Roles &
     }
 }
 
-template <int C, int DW>
+template <int C, int DW, uint32_t SLOT>
 __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const GemmParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t tid = threadIdx.x, warp = tid >> 5;
     const int lane = (int)(tid & 31u);
     const uint32_t S = p.stages;
-    uint8_t *ctrl = smem + ctrl_offset(p.cap, DW);
+    uint8_t *ctrl = smem + ctrl_offset(p.cap, DW, SLOT);
     Roles R;
     const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     R.bars = static_cast<uint32_t>(__cvta_generic_to_shared(ctrl));
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + kNumBars * 8);
     R.abort_flag = tmem_slot + 1;
     R.cover = tmem_slot + 2;
-    R.ring_a = (base + ctrl_offset(p.cap, DW) + kCtrlBytes + 1023u) & ~1023u;
+    R.ring_a = (base + ctrl_offset(p.cap, DW, SLOT) + kCtrlBytes + 1023u) & ~1023u;
     R.ring_b = R.ring_a + S * kTileBytes;
 
     if (tid == 0) {
@@ -588,8 +590,20 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
-    if (warp < DW) {
-        decode_role<C, DW>(p, R, smem, warp, lane);
+    // short staging slots hold a segment's codes only when no code is 1 bit
+    // long (the all-zero code is the shortest): otherwise no role runs, the
+    // stream is reported and the tensor memory is released below
+    bool slots_ok = true;
+    if (SLOT < kSlotLong) {
+        bool bad = false;
+        const uint32_t lmin = lut_decode(0u, smem + Smem::luts, smem + Smem::cl, p.num_luts, &bad) >> 8;
+        slots_ok = !bad && lmin >= 2;
+        if (!slots_ok && tid == 0)
+            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+    }
+    if (!slots_ok) {
+    } else if (warp < DW) {
+        decode_role<C, DW, SLOT>(p, R, smem, warp, lane);
     } else if (warp == DW) {
         if (lane == 0)
             control_role(p, R);
@@ -611,7 +625,7 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
 struct GemmFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][2] = {};  // [C - 1][16 or 20 decode warps]
+    uint32_t granted[2][2][2] = {};  // [C - 1][16 or 20 decode warps][short slots]
 };
 std::mutex g_gemm_mu;
 GemmFacts g_gemm[64];
@@ -711,11 +725,13 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
         }
     }
     // as many ring stages as fit; 20 decode warps if that leaves at least
-    // kMinStages20 stages, else 16 decode warps and at least 2 stages
+    // kMinStages20 stages, else 16 decode warps and at least 2 stages; short
+    // staging slots when the stream states that no code is 1 bit long
     const uint32_t optin = (uint32_t)f->smem_optin;
+    const uint32_t slot = prm.min_code_len >= 2 ? kSlotShort : kSlotLong;
     auto max_stages = [&](uint32_t dw) {
         uint32_t st = kMaxStages;
-        while (st >= 1 && gemm_smem_bytes(prm.cap, batch, st, dw) > optin)
+        while (st >= 1 && gemm_smem_bytes(prm.cap, batch, st, dw, slot) > optin)
             st--;
         return st;
     };
@@ -727,16 +743,18 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
     if (stages < 2)
         return DF11_ERR_INVALID_ARG;
     prm.stages = stages;
-    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages, dw);
-    const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 20 ? 1 : 0;
-    auto kern = ci == 0 ? (wi ? df11_gemm_kernel<1, 20> : df11_gemm_kernel<1, 16>)
-                        : (wi ? df11_gemm_kernel<2, 20> : df11_gemm_kernel<2, 16>);
+    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages, dw, slot);
+    const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 20 ? 1 : 0, si = slot == kSlotShort ? 1 : 0;
+    auto kern = ci == 0 ? (wi ? (si ? df11_gemm_kernel<1, 20, kSlotShort> : df11_gemm_kernel<1, 20, kSlotLong>)
+                              : (si ? df11_gemm_kernel<1, 16, kSlotShort> : df11_gemm_kernel<1, 16, kSlotLong>))
+                        : (wi ? (si ? df11_gemm_kernel<2, 20, kSlotShort> : df11_gemm_kernel<2, 20, kSlotLong>)
+                              : (si ? df11_gemm_kernel<2, 16, kSlotShort> : df11_gemm_kernel<2, 16, kSlotLong>));
     {
         std::lock_guard<std::mutex> lock(g_gemm_mu);
-        if (smem > f->granted[ci][wi]) {
+        if (smem > f->granted[ci][wi][si]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return DF11_ERR_CUDA;
-            f->granted[ci][wi] = smem;
+            f->granted[ci][wi][si] = smem;
         }
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

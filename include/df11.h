@@ -104,7 +104,11 @@ typedef struct df11_arrays {
     uint32_t num_luts;          /* k, 1 .. 17 */
     uint32_t max_code_len;      /* longest code length, <= 32 */
     uint32_t max_block_elems;   /* max_b BlockOffset[b+1] - BlockOffset[b] */
-    uint32_t reserved;
+    uint32_t min_code_len;      /* shortest code length, 1..32; 0 = not known
+                                   (the decoder then assumes 1).  The decoder
+                                   sizes its per-segment staging buffers by it
+                                   and reports DF11_ERR_CORRUPT if a code is
+                                   shorter than stated */
     const uint8_t *encoded_exponent;     /* num_blocks*T*8 + 16 bytes, zero padded, 16-B aligned */
     uint64_t encoded_exponent_bytes;
     const uint8_t *packed_sign_mantissa; /* round_up(n, 16) + 16 bytes, 16-B aligned */

@@ -37,6 +37,8 @@ def compare(fmt, ref):
     assert np.array_equal(a["luts"], ref["luts"])
     assert s["num_segments"] == len(ref["gaps"])
     assert s["max_code_len"] == int(ref["code_lengths"].max()) if n else True
+    used = ref["code_lengths"][ref["code_lengths"] > 0]
+    assert s["min_code_len"] == (int(used.min()) if used.size else 0)
     offs = ref["block_offset"].astype(np.int64)
     assert s["max_block_elems"] == (int(np.diff(offs).max()) if offs.size > 1 else 0)
 
