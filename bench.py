@@ -311,6 +311,7 @@ def measure_workload(wl, args, device, peak):
     per_launch = med / len(prepared)
     alg, achieved, frac = roofline_fraction(prepared, per_launch, peak)
     info0 = prepared[0]["info"]
+    traffic = recorded_traffic(wl, info0["n"])
     rec = {
         "workload": _workload_name(wl),
         "elements": int(n_total),
@@ -323,6 +324,7 @@ def measure_workload(wl, args, device, peak):
         "frac": round(frac, 4),
         "frac_vs_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
         "algorithmic_bytes_per_launch": int(alg),
+        "traffic": None if traffic is None else int(traffic),
         "bits_per_weight": round(8 + info0["avg_code_len"], 4),
         "max_code_len": info0["max_code_len"],
         "num_luts": info0["num_luts"],

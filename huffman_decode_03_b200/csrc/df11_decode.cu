@@ -280,6 +280,47 @@ __device__ __forceinline__ void read_block(uint32_t buf, int lane, BlockRegs<C> 
     __syncwarp();
 }
 
+// The merge of up to four 16-element chunks of one lane, in PTX: chunk k
+// (k < nit) has its 16 sign/mantissa bytes at sp + 512 k (global), its
+// rotated exponents at ea + 512 k (shared) and its 16 outputs at dp + 1024 k
+// (32-byte aligned).  Two sign/mantissa loads are in flight: chunks 0 and 1
+// first, chunk 2 into chunk 0's registers once that is merged, chunk 3 into
+// chunk 1's.  Per 4 elements two bit-selects and two byte permutes (as
+// merge4); the merged words overwrite their inputs.
+#define DF11_MERGE4(S, E)                                  \
+    "lop3.b32 h, " S ", " E ", 0x80808080, 0xE4;\n\t"    \
+    "lop3.b32 l, " E ", " S ", 0x80808080, 0xE4;\n\t"    \
+    "prmt.b32 " S ", l, h, 0x5140;\n\t"                  \
+    "prmt.b32 " E ", l, h, 0x7362;\n\t"
+#define DF11_CHUNK(Q, A, OFFE, OFFD)                                                                        \
+    "@" Q " ld.shared.v4.b32 {e0, e1, e2, e3}, [%2+" OFFE "];\n\t"                                      \
+    DF11_MERGE4(A "0", "e0") DF11_MERGE4(A "1", "e1") DF11_MERGE4(A "2", "e2") DF11_MERGE4(A "3", "e3")   \
+    "@" Q " st.global.v8.b32 [%1+" OFFD "], {" A "0, e0, " A "1, e1, " A "2, e2, " A "3, e3};\n\t"
+__device__ __forceinline__ void merge_chunks4(const uint8_t *sp, uint16_t *dp, uint32_t ea, uint32_t nit)
+{
+    asm volatile(
+        "{\n\t"
+        ".reg .pred q0, q1, q2, q3;\n\t"
+        ".reg .b32 a0, a1, a2, a3, b0, b1, b2, b3, e0, e1, e2, e3, h, l;\n\t"
+        "setp.gt.u32 q0, %3, 0;\n\t"
+        "setp.gt.u32 q1, %3, 1;\n\t"
+        "setp.gt.u32 q2, %3, 2;\n\t"
+        "setp.gt.u32 q3, %3, 3;\n\t"
+        "@q0 ld.global.nc.v4.b32 {a0, a1, a2, a3}, [%0];\n\t"
+        "@q1 ld.global.nc.v4.b32 {b0, b1, b2, b3}, [%0+512];\n\t"
+        DF11_CHUNK("q0", "a", "0", "0")
+        "@q2 ld.global.nc.v4.b32 {a0, a1, a2, a3}, [%0+1024];\n\t"
+        DF11_CHUNK("q1", "b", "512", "1024")
+        "@q3 ld.global.nc.v4.b32 {b0, b1, b2, b3}, [%0+1536];\n\t"
+        DF11_CHUNK("q2", "a", "1024", "2048")
+        DF11_CHUNK("q3", "b", "1536", "3072")
+        "}"
+        ::"l"(sp), "l"(dp), "r"(ea), "r"(nit)
+        : "memory");
+}
+#undef DF11_CHUNK
+#undef DF11_MERGE4
+
 // Per-warp shared memory of a launch: the write buffer, the staging slots
 // and, with short slots, the metadata buffer of the next block.
 template <int C, uint32_t SLOT>
@@ -360,6 +401,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
                 // 16 elements per lane and step, one 32-byte store: a warp's
                 // stores cover 1 KB contiguous
                 const uint32_t c_first = lo_off ? 1u : 0u, c_end = hi >> 4;  // full chunks [c_first, c_end)
+                if (kCopy) {
+                    // (registers free of the next block's metadata) up to
+                    // four chunks of a lane per call
+                    for (uint32_t c0 = c_first + (uint32_t)lane; c0 < c_end; c0 += 128u)
+                        merge_chunks4(smg + 16u * c0, p.dst + g0 + 16u * c0, exp_base + 16u * c0,
+                                      (c_end - c0 + 31u) >> 5);
+                } else
 #pragma unroll 2
                 for (uint32_t c = c_first + lane; c < c_end; c += 32) {
                     const uint32_t l0 = 16 * c;
