@@ -542,3 +542,235 @@ int64_t df11o_decode_range(const uint8_t *stream, uint64_t stream_bits,
     free(tree);
     return count;
 }
+
+/* ===========================================================================
+ * rANS variant of the exponent coder (the page's discussion proposes rANS
+ * as an entropy coder that suits SIMD-style hardware better than Huffman
+ * coding).  The pages give no parameters; this restates the range variant
+ * of asymmetric numeral systems from its published definition (J. Duda,
+ * "Asymmetric numeral systems", 2013, range variant; one 32-bit state,
+ * 16-bit renormalisation words, as in F. Giesen's description), with the
+ * readings below.  TEST INFRASTRUCTURE: plain loops, no fusion.
+ *
+ *   model    : exponent counts h[s] quantised to frequencies f[s] summing to
+ *              M = 2^prob_bits; cumulative c[s] = sum of f[t] for t < s.
+ *   state    : x in [L, 2^32), L = 2^16.
+ *   encode s : if x >= 2^(32 - prob_bits) * f[s]: emit x mod 2^16 (one
+ *              16-bit word), x = floor(x / 2^16); then
+ *              x = floor(x / f[s]) * M + (x mod f[s]) + c[s].
+ *   decode   : slot = x mod M; s = the symbol with c[s] <= slot < c[s] + f[s];
+ *              x = f[s] * floor(x / M) + slot - c[s]; if x < L: x = x * 2^16 +
+ *              the next 16-bit word.
+ *   layout   : blocks of B = 32 * 16 * J elements; lane l (0..31) of block b
+ *              owns elements b B + 512 j + 16 l + i (j = 0..J-1, i = 0..15),
+ *              decoded in the order (j, i); all lanes step together, step
+ *              t = 16 j + i; a lane whose element lies at or past n skips the
+ *              step.  After each step the lanes that renormalise read one word
+ *              each, in lane order, from the block's word sequence.  The
+ *              encoder runs the same steps backwards (t descending, lanes
+ *              descending), starting every lane at x = L; its final states are
+ *              the decoder's start states, and its words, reversed, the block's
+ *              word sequence.
+ * ======================================================================== */
+
+/* Frequencies: f[s] = max(1, floor(h[s] M / n)) for every symbol present,
+ * 0 otherwise; then, while the sum exceeds M, the largest frequency (ties:
+ * smallest symbol) drops by one, and while it is short of M the symbol with
+ * the largest count (ties: smallest symbol) gains one.  Returns 0, or -1 when
+ * no symbol is present or more symbols are present than M allows. */
+int df11o_rans_freqs(const uint64_t *hist, int prob_bits, uint32_t *freq)
+{
+    uint64_t n = 0;
+    int present = 0;
+    for (int s = 0; s < ORACLE_NSYM; s++) {
+        n += hist[s];
+        present += hist[s] > 0;
+    }
+    const uint32_t M = 1u << prob_bits;
+    if (n == 0 || (uint32_t)present > M)
+        return -1;
+    uint64_t sum = 0;
+    for (int s = 0; s < ORACLE_NSYM; s++) {
+        freq[s] = 0;
+        if (hist[s]) {
+            uint64_t f = hist[s] * (uint64_t)M / n;
+            freq[s] = f < 1 ? 1u : (uint32_t)f;
+        }
+        sum += freq[s];
+    }
+    while (sum > M) {
+        int best = -1;
+        for (int s = 0; s < ORACLE_NSYM; s++)
+            if (freq[s] > 1 && (best < 0 || freq[s] > freq[best]))
+                best = s;
+        freq[best]--;
+        sum--;
+    }
+    while (sum < M) {
+        int best = -1;
+        for (int s = 0; s < ORACLE_NSYM; s++)
+            if (hist[s] && (best < 0 || hist[s] > hist[best]))
+                best = s;
+        freq[best]++;
+        sum++;
+    }
+    return 0;
+}
+
+/* Element of block b owned by lane l at step t (J chunks per lane). */
+static uint64_t oracle_rans_pos(uint64_t b, int J, int l, int t)
+{
+    return b * (uint64_t)(512 * J) + 512u * (uint64_t)(t / 16) + 16u * (uint64_t)l + (uint64_t)(t % 16);
+}
+
+/* rANS encode of n exponents, blocks of 512 J elements.  words receives the
+ * 16-bit words of block 0, then block 1, ...; offsets[b] (nblocks + 1
+ * entries) the index of block b's first word; states[32 b + l] the start
+ * state of lane l of block b.  Returns the number of words, or -1 (capacity,
+ * a symbol with frequency 0, or a state outside [L, 2^32)). */
+int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq, int prob_bits, int J,
+                          uint16_t *words, uint64_t cap, uint32_t *states, uint64_t *offsets)
+{
+    const uint64_t L = 1ull << 16, M = 1ull << prob_bits;
+    const uint64_t B = 512ull * (uint64_t)J;
+    const uint64_t nblocks = (n + B - 1) / B;
+    uint64_t cum[ORACLE_NSYM];
+    uint64_t c = 0;
+    for (int s = 0; s < ORACLE_NSYM; s++) {
+        cum[s] = c;
+        c += freq[s];
+    }
+    if (c != M)
+        return -1;
+    uint16_t *stack = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(B ? B : 1));
+    if (!stack)
+        return -1;
+    uint64_t total = 0;
+    for (uint64_t b = 0; b < nblocks; b++) {
+        uint64_t x[32];
+        for (int l = 0; l < 32; l++)
+            x[l] = L;
+        uint64_t depth = 0;
+        for (int t = 16 * J - 1; t >= 0; t--) {
+            for (int l = 31; l >= 0; l--) {
+                const uint64_t pos = oracle_rans_pos(b, J, l, t);
+                if (pos >= n)
+                    continue;
+                const int s = exps[pos];
+                const uint64_t f = freq[s];
+                if (f == 0) {
+                    free(stack);
+                    return -1;
+                }
+                if (x[l] >= (1ull << (32 - prob_bits)) * f) {
+                    stack[depth++] = (uint16_t)(x[l] & 0xFFFFu);
+                    x[l] >>= 16;
+                }
+                x[l] = (x[l] / f) * M + (x[l] % f) + cum[s];
+                if (x[l] < L || x[l] >= (1ull << 32)) {
+                    free(stack);
+                    return -1;
+                }
+            }
+        }
+        offsets[b] = total;
+        if (total + depth > cap) {
+            free(stack);
+            return -1;
+        }
+        for (uint64_t k = 0; k < depth; k++)
+            words[total + k] = stack[depth - 1 - k];
+        total += depth;
+        for (int l = 0; l < 32; l++)
+            states[32 * b + l] = (uint32_t)x[l];
+    }
+    offsets[nblocks] = total;
+    free(stack);
+    return (int64_t)total;
+}
+
+/* rANS decode back to BF16 bits (exponent from the words, sign and mantissa
+ * from sm).  Returns 0, or -1 when the words, states or offsets are
+ * inconsistent (a block reads past its words, does not use all of them, or
+ * does not end every lane at x = L). */
+int df11o_rans_decode(const uint16_t *words, const uint32_t *states, const uint64_t *offsets,
+                      const uint32_t *freq, int prob_bits, int J, uint64_t n, const uint8_t *sm, uint16_t *out)
+{
+    const uint64_t L = 1ull << 16, M = 1ull << prob_bits;
+    const uint64_t B = 512ull * (uint64_t)J;
+    const uint64_t nblocks = (n + B - 1) / B;
+    uint64_t cum[ORACLE_NSYM];
+    uint64_t c = 0;
+    for (int s = 0; s < ORACLE_NSYM; s++) {
+        cum[s] = c;
+        c += freq[s];
+    }
+    if (c != M)
+        return -1;
+    for (uint64_t b = 0; b < nblocks; b++) {
+        uint64_t x[32];
+        for (int l = 0; l < 32; l++)
+            x[l] = states[32 * b + l];
+        uint64_t ptr = offsets[b];
+        for (int t = 0; t < 16 * J; t++) {
+            for (int l = 0; l < 32; l++) {
+                const uint64_t pos = oracle_rans_pos(b, J, l, t);
+                if (pos >= n)
+                    continue;
+                const uint64_t slot = x[l] % M;
+                int s = -1;
+                for (int k = 0; k < ORACLE_NSYM; k++)
+                    if (freq[k] && cum[k] <= slot && slot < cum[k] + freq[k])
+                        s = k;
+                if (s < 0)
+                    return -1;
+                x[l] = freq[s] * (x[l] / M) + slot - cum[s];
+                const unsigned sign = (sm[pos] >> 7) & 1u, mantissa = sm[pos] & 0x7Fu;
+                out[pos] = (uint16_t)((sign << 15) | ((unsigned)s << 7) | mantissa);
+                if (x[l] < L) {
+                    if (ptr >= offsets[b + 1])
+                        return -1;
+                    x[l] = (x[l] << 16) | words[ptr++];
+                }
+            }
+        }
+        if (ptr != offsets[b + 1])
+            return -1;
+        for (int l = 0; l < 32; l++)
+            if (x[l] != L)
+                return -1;
+    }
+    return 0;
+}
+
+/* One rANS step on a single state, for exhaustive checks: encodes s into
+ * x (x in [L, 2^32)) and returns the new state; *word / *emitted receive the
+ * renormalisation word, if any. */
+uint64_t df11o_rans_step_encode(uint64_t x, int s, const uint32_t *freq, int prob_bits, uint32_t *word,
+                                int *emitted)
+{
+    uint64_t cum = 0;
+    for (int k = 0; k < s; k++)
+        cum += freq[k];
+    const uint64_t f = freq[s], M = 1ull << prob_bits;
+    *emitted = 0;
+    if (x >= (1ull << (32 - prob_bits)) * f) {
+        *word = (uint32_t)(x & 0xFFFFu);
+        *emitted = 1;
+        x >>= 16;
+    }
+    return (x / f) * M + (x % f) + cum;
+}
+
+/* BF16 field split for the rANS variant: as df11o_split, but every exponent
+ * 0..255 is allowed (rANS needs no pointer values). */
+void df11o_split_all(const uint16_t *w, uint64_t n, uint8_t *exps, uint8_t *sm)
+{
+    for (uint64_t i = 0; i < n; i++) {
+        unsigned sign = (w[i] >> 15) & 1u;
+        unsigned exponent = (w[i] >> 7) & 0xFFu;
+        unsigned mantissa = w[i] & 0x7Fu;
+        exps[i] = (uint8_t)exponent;
+        sm[i] = (uint8_t)((sign << 7) | mantissa);
+    }
+}

@@ -10,6 +10,13 @@ restates.  ``build_format`` chains them in the page's order: split the BF16
 fields, histogram the exponents, Huffman code lengths (capped at 32 bits),
 canonical codes, bit-pack EncodedExponent, then the decoder metadata (Gaps,
 BlockOffset) and the hierarchical LUTs.
+
+``rans_build_format`` / ``rans_decode_format`` are the rANS variant of the
+exponent coder that the page's discussion proposes (range asymmetric numeral
+systems from their published definition: quantised frequencies, one 32-bit
+state per lane, 16-bit words, blocks of 512 J elements decoded by 32 lanes in
+step); sign and mantissa stay verbatim as in DF11.  Pinned in
+``tests/test_rans_oracle.py``.
 """
 from __future__ import annotations
 
@@ -76,6 +83,16 @@ def _load():
         lib.df11o_decode.restype = ctypes.c_int
         lib.df11o_decode_range.argtypes = [P, U64, U64, U64, P, P, P, U64]
         lib.df11o_decode_range.restype = ctypes.c_int64
+        lib.df11o_split_all.argtypes = [P, U64, P, P]
+        lib.df11o_split_all.restype = None
+        lib.df11o_rans_freqs.argtypes = [P, ctypes.c_int, P]
+        lib.df11o_rans_freqs.restype = ctypes.c_int
+        lib.df11o_rans_encode.argtypes = [P, U64, P, ctypes.c_int, ctypes.c_int, P, U64, P, P]
+        lib.df11o_rans_encode.restype = ctypes.c_int64
+        lib.df11o_rans_decode.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, U64, P, P]
+        lib.df11o_rans_decode.restype = ctypes.c_int
+        lib.df11o_rans_step_encode.argtypes = [U64, ctypes.c_int, P, ctypes.c_int, P, P]
+        lib.df11o_rans_step_encode.restype = U64
         _lib = lib
         return lib
 
@@ -255,3 +272,97 @@ def decode_format(fmt: dict) -> np.ndarray:
         fmt["encoded_exponent"], fmt["total_bits"], fmt["code_lengths"], fmt["codes"],
         fmt["packed_sign_mantissa"], fmt["n"],
     )
+
+
+# ------------------------------------------------------------------ rANS
+# The rANS variant of the exponent coder (the page's discussion proposes rANS
+# as the SIMD-friendlier entropy coder); the C side states the model and the
+# layout.
+RANS_PROB_BITS = 12
+RANS_CHUNKS = 8  # J: chunks of 16 elements per lane and block (4096 elements per block)
+RANS_L = 1 << 16
+
+
+def rans_freqs(hist, prob_bits: int = RANS_PROB_BITS) -> np.ndarray:
+    hist = np.ascontiguousarray(hist, dtype=np.uint64)
+    freq = np.zeros(256, np.uint32)
+    if _load().df11o_rans_freqs(_ptr(hist), prob_bits, _ptr(freq)) != 0:
+        raise ValueError("no symbol, or more symbols than the precision allows")
+    return freq
+
+
+def rans_encode(exps, freq, prob_bits: int = RANS_PROB_BITS, chunks: int = RANS_CHUNKS):
+    """-> (words uint16, states uint32 [nblocks, 32], offsets uint64 [nblocks + 1])"""
+    exps = np.ascontiguousarray(exps, dtype=np.uint8)
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    n = exps.size
+    B = 512 * chunks
+    nblocks = (n + B - 1) // B
+    words = np.zeros(max(n, 1), np.uint16)
+    states = np.zeros(max(32 * nblocks, 1), np.uint32)
+    offsets = np.zeros(nblocks + 1, np.uint64)
+    src = exps if n else np.zeros(1, np.uint8)
+    got = _load().df11o_rans_encode(_ptr(src), n, _ptr(freq), prob_bits, chunks, _ptr(words), words.size,
+                                    _ptr(states), _ptr(offsets))
+    if got < 0:
+        raise ValueError("rANS encode failed")
+    return words[:got].copy(), states[: 32 * nblocks].reshape(nblocks, 32).copy(), offsets
+
+
+def rans_decode(words, states, offsets, freq, sm, n: int, prob_bits: int = RANS_PROB_BITS,
+                chunks: int = RANS_CHUNKS) -> np.ndarray:
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    if words.size == 0:
+        words = np.zeros(1, np.uint16)
+    states = np.ascontiguousarray(states, dtype=np.uint32).reshape(-1)
+    if states.size == 0:
+        states = np.zeros(1, np.uint32)
+    offsets = np.ascontiguousarray(offsets, dtype=np.uint64)
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    sm = np.ascontiguousarray(sm, dtype=np.uint8)
+    if sm.size == 0:
+        sm = np.zeros(1, np.uint8)
+    out = np.empty(max(n, 1), np.uint16)
+    rc = _load().df11o_rans_decode(_ptr(words), _ptr(states), _ptr(offsets), _ptr(freq), prob_bits, chunks, n,
+                                   _ptr(sm), _ptr(out))
+    if rc != 0:
+        raise ValueError("rANS data inconsistent")
+    return out[:n]
+
+
+def rans_step_encode(x: int, s: int, freq, prob_bits: int):
+    """One encode step of one state -> (new state, emitted word or None)."""
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    word = ctypes.c_uint32(0)
+    emitted = ctypes.c_int(0)
+    y = _load().df11o_rans_step_encode(x, s, _ptr(freq), prob_bits, ctypes.byref(word), ctypes.byref(emitted))
+    return int(y), (int(word.value) if emitted.value else None)
+
+
+def split_all(w: np.ndarray):
+    """BF16 bits -> (exponent bytes, sign/mantissa bytes), every exponent
+    allowed (the rANS variant needs no pointer values)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).ravel()
+    exps = np.empty(w.size, np.uint8)
+    sm = np.empty(w.size, np.uint8)
+    if w.size:
+        _load().df11o_split_all(_ptr(w), w.size, _ptr(exps), _ptr(sm))
+    return exps, sm
+
+
+def rans_build_format(w: np.ndarray, prob_bits: int = RANS_PROB_BITS, chunks: int = RANS_CHUNKS) -> dict:
+    """All arrays of the rANS variant for one stream of BF16 bits."""
+    exps, sm = split_all(w)
+    hist = histogram(exps)
+    freq = rans_freqs(hist, prob_bits) if exps.size else np.zeros(256, np.uint32)
+    words, states, offsets = rans_encode(exps, freq, prob_bits, chunks) if exps.size else (
+        np.zeros(0, np.uint16), np.zeros((0, 32), np.uint32), np.zeros(1, np.uint64))
+    return {"n": int(exps.size), "hist": hist, "freq": freq, "words": words, "states": states,
+            "offsets": offsets, "packed_sign_mantissa": sm, "prob_bits": prob_bits, "chunks": chunks}
+
+
+def rans_decode_format(fmt: dict) -> np.ndarray:
+    if fmt["n"] == 0:
+        return np.zeros(0, np.uint16)
+    return rans_decode(fmt["words"], fmt["states"], fmt["offsets"], fmt["freq"], fmt["packed_sign_mantissa"],
+                       fmt["n"], fmt["prob_bits"], fmt["chunks"])
