@@ -59,6 +59,9 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between timed steps")
+    ap.add_argument("--rans", default="2,3",
+                    help="workloads on which the rANS variant of the exponent coder is measured at N=1 and "
+                         "reported in the line's rans object (comma-separated ids, or 'none')")
     ap.add_argument("--per-workload", default="4,3,1",
                     help="further workloads measured after the headline one at N=1, reported in the "
                          "line's per_workload object (comma-separated ids, or 'none')")
@@ -337,6 +340,73 @@ def measure_workload(wl, args, device, peak):
     return rec
 
 
+def rans_algorithmic_bytes(fmt) -> int:
+    """Bytes one rANS-variant launch must move: its compressed arrays read,
+    2 bytes per BF16 written."""
+    return fmt.compressed_bytes() + 2 * fmt.scalars()["n"]
+
+
+def measure_rans(wl, args, device, peak):
+    """The rANS variant of the exponent coder on one workload at N=1: build,
+    upload, check, time (median of per-step CUDA-event times, L2 flushed)."""
+    import torch
+
+    import huffman_decode_03_b200 as df11
+    from huffman_decode_03_b200 import inputs
+
+    mats = [m for _, _, m in inputs.workload_arrays(wl, 0)]
+    w = np.concatenate(mats) if len(mats) > 1 else mats[0]
+    del mats
+    fmt = df11.rans_build_format(w)
+    dev = df11.RansDeviceFormat(fmt, device)
+    n = dev.n
+    alg = rans_algorithmic_bytes(fmt)
+    comp = fmt.compressed_bytes()
+    fmt.free()
+    bits = torch.from_numpy(w.view(np.int16)).to(device)
+    del w
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = None if args.no_flush else torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    df11.rans_decompress(dev, out, status, stream)
+    exact = df11.read_status(status) == 0 and bool(torch.equal(out.view(torch.int16), bits))
+    out.zero_()
+    for _ in range(args.warmup):
+        df11.rans_decompress(dev, out, status, stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        if flush is not None:
+            flush.zero_()
+        e0.record(stream)
+        df11.rans_decompress(dev, out, status, stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    med = float(statistics.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+    exact = exact and df11.read_status(status) == 0 and bool(torch.equal(out.view(torch.int16), bits))
+    achieved = alg / (med * 1e-3) / 1e9
+    rec = {
+        "workload": _workload_name(wl),
+        "kernel": "rans_decode_kernel",
+        "elements": int(n),
+        "compressed_bytes": int(comp),
+        "bits_per_weight": round(8.0 * (comp - n) / n + 8, 4),
+        "ms_per_launch": round(med, 5),
+        "value": round(2.0 * n / (med * 1e-3) / 1e9, 2),
+        "unit": UNIT,
+        "roofline_achieved_gbs": round(achieved, 1),
+        "frac": round(achieved / peak, 4),
+        "algorithmic_bytes_per_launch": int(alg),
+        "bit_exact": bool(exact),
+        "steps": args.steps,
+        "timing": "median of per-step CUDA-event times",
+    }
+    del dev, out, bits, flush
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -470,6 +540,11 @@ def run_gpu(args):
         per = [measure_workload(wl, args, device, peak) for wl in extra]
         line["per_workload"] = per
         line["gpu_launches"] += sum(r["steps"] * r["launches_per_step"] for r in per)
+    rans = [] if args.rans.strip().lower() in ("", "none") else [int(x) for x in args.rans.split(",")]
+    if world == 1 and rans:
+        peak, _ = load_peak()
+        line["rans"] = [measure_rans(wl, args, device, peak) for wl in rans]
+        line["gpu_launches"] += sum(r["steps"] for r in line["rans"])
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)

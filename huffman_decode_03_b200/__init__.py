@@ -23,7 +23,8 @@ from . import build as _build
 __all__ = [
     "Df11Error", "Format", "DeviceFormat", "build_format", "decompress",
     "decompress_gemv", "decompress_gemm", "gemm_scratch_bytes", "decompress_host", "encode_device",
-    "read_status", "tile_major", "load_library",
+    "read_status", "tile_major", "load_library", "RansFormat", "RansDeviceFormat", "rans_build_format",
+    "rans_decompress",
 ]
 
 DF11_OK = 0
@@ -78,6 +79,23 @@ class df11_arrays(ctypes.Structure):
     ]
 
 
+class df11_rans_arrays(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_uint64),
+        ("num_words", ctypes.c_uint64),
+        ("prob_bits", ctypes.c_uint32),
+        ("chunks", ctypes.c_uint32),
+        ("num_blocks", ctypes.c_uint32),
+        ("max_block_words", ctypes.c_uint32),
+        ("words", ctypes.c_void_p),
+        ("states", ctypes.c_void_p),
+        ("block_word", ctypes.c_void_p),
+        ("freq", ctypes.c_void_p),
+        ("packed_sign_mantissa", ctypes.c_void_p),
+        ("packed_sign_mantissa_bytes", ctypes.c_uint64),
+    ]
+
+
 class df11_info(ctypes.Structure):
     _fields_ = [
         ("n", ctypes.c_uint64),
@@ -98,6 +116,7 @@ EXPORTS = (
     "df11_strerror", "df11_decompress", "df11_decompress_sms", "df11_decompress_gemv", "df11_decompress_gemm",
     "df11_gemm_scratch_bytes", "df11_tile_major", "df11_decompress_host", "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
     "df11_device_encode_scratch_words", "df11_device_encode", "df11_device_encode_static",
+    "df11_rans_build", "df11_rans_format_arrays", "df11_rans_free", "df11_rans_decompress",
 )
 
 _lib = None
@@ -153,6 +172,14 @@ def load_library(path: str | None = None):
     lib.df11_device_encode.restype = ctypes.c_int
     lib.df11_device_encode_static.argtypes = [P, P, ctypes.POINTER(df11_arrays), P, P, P]
     lib.df11_device_encode_static.restype = ctypes.c_int
+    lib.df11_rans_build.argtypes = [P, P, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(P)]
+    lib.df11_rans_build.restype = ctypes.c_int
+    lib.df11_rans_format_arrays.argtypes = [P, ctypes.POINTER(df11_rans_arrays)]
+    lib.df11_rans_format_arrays.restype = ctypes.c_int
+    lib.df11_rans_free.argtypes = [P]
+    lib.df11_rans_free.restype = None
+    lib.df11_rans_decompress.argtypes = [ctypes.POINTER(df11_rans_arrays), P, P, P]
+    lib.df11_rans_decompress.restype = ctypes.c_int
     if path == _build.LIB_PATH:
         _lib = lib
     return lib
@@ -524,3 +551,114 @@ def encode_device(w, threads_per_block: int = 64, stream=None, static_scratch: b
 def read_status(status, stream=None) -> int:
     """Synchronises the stream and returns the kernel status (0 = ok)."""
     return int(load_library().df11_read_status(ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)))
+
+
+# --------------------------------------------------------------------- rANS
+class RansFormat:
+    """A host-resident stream of the rANS variant (handle from ``df11_rans_build``):
+    the same BF16 values, exponents coded with rANS instead of Huffman codes."""
+
+    def __init__(self, handle: int, lib):
+        self._h = ctypes.c_void_p(handle)
+        self._lib = lib
+        a = df11_rans_arrays()
+        _check(lib.df11_rans_format_arrays(self._h, ctypes.byref(a)), "df11_rans_format_arrays")
+        self.c_arrays = a
+
+    def __del__(self):
+        self.free()
+
+    def free(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._lib.df11_rans_free(h)
+            self._h = None
+
+    def _view(self, ptr, count, dtype):
+        if count == 0 or not ptr:
+            return np.zeros(0, dtype)
+        nbytes = int(count) * np.dtype(dtype).itemsize
+        buf = (ctypes.c_uint8 * nbytes).from_address(ptr)
+        buf._owner = self
+        return np.frombuffer(buf, dtype=dtype, count=int(count))
+
+    def arrays(self) -> dict:
+        a = self.c_arrays
+        return {
+            "words": self._view(a.words, a.num_words + 8 if a.n else 0, np.uint16),
+            "states": self._view(a.states, 32 * a.num_blocks, np.uint32),
+            "block_word": self._view(a.block_word, a.num_blocks + 1 if a.n else 0, np.uint32),
+            "freq": self._view(a.freq, 256 if a.n else 0, np.uint16),
+            "packed_sign_mantissa": self._view(a.packed_sign_mantissa, a.packed_sign_mantissa_bytes, np.uint8),
+        }
+
+    def scalars(self) -> dict:
+        a = self.c_arrays
+        return {f: int(getattr(a, f)) for f in ("n", "num_words", "prob_bits", "chunks", "num_blocks",
+                                                 "max_block_words")}
+
+    def compressed_bytes(self) -> int:
+        """Bytes of the stream: words, start states, block offsets, the model
+        and the sign/mantissa bytes (without padding)."""
+        s = self.scalars()
+        return 2 * s["num_words"] + 4 * 32 * s["num_blocks"] + 4 * (s["num_blocks"] + 1) + 2 * 256 + s["n"]
+
+
+def rans_build_format(mats, chunks: int = 8) -> RansFormat:
+    """Compresses BF16 bit patterns (uint16 arrays) into one stream of the
+    rANS variant (df11_rans_build); matrices are concatenated in order."""
+    lib = load_library()
+    if isinstance(mats, np.ndarray):
+        mats = [mats]
+    keep = [np.ascontiguousarray(np.asarray(m).view(np.uint16).reshape(-1)) for m in mats]
+    k = len(keep)
+    ptrs = (ctypes.c_void_p * max(k, 1))(*[m.ctypes.data if m.size else None for m in keep])
+    counts = (ctypes.c_uint64 * max(k, 1))(*[m.size for m in keep])
+    h = ctypes.c_void_p()
+    _check(lib.df11_rans_build(ptrs, counts, k, int(chunks), ctypes.byref(h)), "df11_rans_build")
+    return RansFormat(h.value, lib)
+
+
+class RansDeviceFormat:
+    """A rANS-variant stream resident in device memory (torch tensors)."""
+
+    def __init__(self, fmt: RansFormat, device="cuda"):
+        import torch
+
+        self.device = torch.device(device)
+        self.scalars = fmt.scalars()
+        self.tensors = {}
+        for name, arr in fmt.arrays().items():
+            t = torch.from_numpy(np.ascontiguousarray(arr).reshape(-1).view(np.uint8).copy())
+            self.tensors[name] = t.to(self.device)
+        a = df11_rans_arrays()
+        for k, v in self.scalars.items():
+            setattr(a, k, v)
+        ts = self.tensors
+        a.words = ts["words"].data_ptr()
+        a.states = ts["states"].data_ptr()
+        a.block_word = ts["block_word"].data_ptr()
+        a.freq = ts["freq"].data_ptr()
+        a.packed_sign_mantissa = ts["packed_sign_mantissa"].data_ptr()
+        a.packed_sign_mantissa_bytes = ts["packed_sign_mantissa"].numel()
+        self.c_arrays = a
+
+    @property
+    def n(self) -> int:
+        return self.scalars["n"]
+
+
+def rans_decompress(dev: RansDeviceFormat, out=None, status=None, stream=None):
+    """Rebuilds the BF16 stream of the rANS variant on the GPU (asynchronous,
+    stream-ordered); returns ``out`` (allocated if None)."""
+    import torch
+
+    if out is None:
+        out = torch.empty(dev.n, dtype=torch.bfloat16, device=dev.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev.device)
+    assert out.is_cuda and out.is_contiguous() and out.numel() >= dev.n and out.element_size() == 2
+    _check(load_library().df11_rans_decompress(ctypes.byref(dev.c_arrays), ctypes.c_void_p(out.data_ptr()),
+                                               ctypes.c_void_p(status.data_ptr()), _stream_ptr(stream)),
+           "df11_rans_decompress")
+    return out

@@ -18,7 +18,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libdf11_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "df11_decode.cu"), os.path.join(CSRC, "df11_gemm.cu"),
-           os.path.join(CSRC, "df11_encode.cu"), os.path.join(CSRC, "df11_format.cpp")]
+           os.path.join(CSRC, "df11_encode.cu"), os.path.join(CSRC, "df11_format.cpp"),
+           os.path.join(CSRC, "df11_rans.cu"), os.path.join(CSRC, "df11_rans_format.cpp")]
 HEADERS = [os.path.join(INCLUDE, "df11.h"), os.path.join(CSRC, "df11_block.cuh")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -1,0 +1,278 @@
+// df11_rans.cu -- sm_100a decoder of the rANS variant of the exponent coder.
+//
+// The DFloat11 page's discussion proposes rANS (range asymmetric numeral
+// systems) as the entropy coder for the exponents that suits SIMD hardware
+// better than Huffman coding.  The layout (include/df11.h, df11_rans_arrays)
+// is made for a warp: 32 lanes each hold one 32-bit state and step together
+// through a block of 512 * chunks elements; lane l's elements are 16
+// consecutive ones out of every 512, so a lane's 16 decoded exponents are
+// merged with 16 consecutive sign/mantissa bytes and leave in one 32-byte
+// store, and a warp's stores cover 1 KB contiguous -- no prefix sum, no
+// placement through shared memory, unlike the Huffman decoder.
+//
+// Per step and lane: one lookup in a 4096-entry table (the slot's exponent,
+// rotated right by one bit for the merge, slot - cum and freq - 1), one
+// multiply-add for the new state, and, when the state falls below 2^16, one
+// 16-bit word: the lanes that need one take consecutive words of the block
+// in lane order (ballot, popcount of the lanes below).  The next block's words
+// are prefetched into L1 and its sign/mantissa bytes into L2 while the
+// current block decodes.  Every lane must end the block at x = 2^16 and the
+// block must use exactly its words; otherwise DF11_ERR_CORRUPT is set.  Word
+// reads are clamped to the padded array, so inconsistent data never reads
+// out of bounds; nothing traps and every loop has a fixed trip count.
+#include "df11.h"
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+namespace {
+
+constexpr uint32_t kProbBits = 12;
+constexpr uint32_t kSlots = 1u << kProbBits;
+constexpr uint32_t kLow = 1u << 16;
+constexpr int kWarps = 32;
+
+struct RansParams {
+    const uint16_t *words;
+    const uint32_t *states;
+    const uint32_t *block_word;
+    const uint16_t *freq;
+    const uint8_t *sm;
+    uint16_t *dst;
+    uint32_t *status;
+    uint64_t n;
+    uint32_t last_word;  // index of the last readable word (num_words + 7)
+    uint32_t num_blocks;
+    uint32_t chunks;
+    uint32_t wide;  // dst is 32-byte aligned: 32-byte stores
+};
+
+__device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
+
+// BF16 from sign/mantissa bytes S and rotated exponent bytes E (4 each):
+// high byte = sign | e >> 1, low byte = (e & 1) << 7 | mantissa.
+__device__ __forceinline__ void merge4(uint32_t S, uint32_t E, uint32_t &lo2, uint32_t &hi2)
+{
+    const uint32_t HB = (S & 0x80808080u) | (E & 0x7F7F7F7Fu);
+    const uint32_t LB = (E & 0x80808080u) | (S & 0x7F7F7F7Fu);
+    lo2 = __byte_perm(LB, HB, 0x5140);
+    hi2 = __byte_perm(LB, HB, 0x7362);
+}
+
+__device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
+{
+    return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt()
+{
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// One decode step of one lane (all lanes call it together).  valid: the
+// lane's element exists; acc receives the exponent byte at byte position Q.
+template <int Q>
+__device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base, bool valid, const uint32_t *table,
+                                     const RansParams &p, uint32_t lt)
+{
+    if (valid) {
+        const uint32_t e = table[x & (kSlots - 1)];
+        const uint32_t xh = x >> kProbBits;
+        x = (e >> 20) * xh + xh + ((e >> 8) & 0xFFFu);
+        acc = __byte_perm(acc, e, (0x3210 & ~(0xF << (4 * Q))) | (4 << (4 * Q)));
+    }
+    const bool need = valid && x < kLow;
+    const uint32_t m = __ballot_sync(0xffffffffu, need);
+    if (m) {  // warp-uniform
+        if (need) {
+            uint32_t i = base + __popc(m & lt);
+            i = i < p.last_word ? i : p.last_word;
+            x = (x << 16) | __ldg(p.words + i);
+        }
+        base += __popc(m);
+    }
+}
+
+template <bool FULL>
+__device__ __forceinline__ void decode_chunk(uint32_t &x, uint32_t &base, uint64_t pos0, const uint32_t *table,
+                                             const RansParams &p, uint32_t lt, uint32_t acc[4])
+{
+#define DF11_STEP(I) \
+    step<(I) & 3>(x, acc[(I) >> 2], base, FULL || pos0 + (I) < p.n, table, p, lt)
+    DF11_STEP(0); DF11_STEP(1); DF11_STEP(2); DF11_STEP(3);
+    DF11_STEP(4); DF11_STEP(5); DF11_STEP(6); DF11_STEP(7);
+    DF11_STEP(8); DF11_STEP(9); DF11_STEP(10); DF11_STEP(11);
+    DF11_STEP(12); DF11_STEP(13); DF11_STEP(14); DF11_STEP(15);
+#undef DF11_STEP
+}
+
+__global__ void __launch_bounds__(kWarps * 32, 1) rans_decode_kernel(const RansParams p)
+{
+    __shared__ uint32_t table[kSlots];
+    __shared__ uint32_t cum[257];
+    const uint32_t tid = threadIdx.x, warp = tid >> 5;
+    const int lane = (int)(tid & 31u);
+
+    // cumulative frequencies (one warp: 8 per lane, shuffle scan)
+    if (warp == 0) {
+        uint32_t f[8], s = 0;
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            f[k] = p.freq[8 * lane + k];
+            s += f[k];
+        }
+        uint32_t incl = s;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d)
+                incl += y;
+        }
+        uint32_t c = incl - s;
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            cum[8 * lane + k] = c;
+            c += f[k];
+        }
+        if (lane == 31)
+            cum[256] = c;
+    }
+    __syncthreads();
+    // slot -> entry: the exponent whose range holds the slot (binary search)
+    for (uint32_t slot = tid; slot < kSlots; slot += blockDim.x) {
+        uint32_t lo = 0, hi = 256;  // cum[lo] <= slot < cum[hi]
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const uint32_t mid = (lo + hi) >> 1;
+            if (cum[mid] <= slot)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const uint32_t f = cum[lo + 1] - cum[lo];
+        table[slot] = ror8(lo) | ((slot - cum[lo]) << 8) | (((f - 1u) & 0xFFFu) << 20);
+    }
+    __syncthreads();
+    if (cum[256] != kSlots) {  // the model does not sum to 2^12
+        if (tid == 0)
+            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+        return;
+    }
+
+    const uint32_t lt = lanemask_lt();
+    const uint64_t B = 512ull * p.chunks;
+    const uint32_t stride = gridDim.x * kWarps;
+    for (uint32_t b = blockIdx.x * kWarps + warp; b < p.num_blocks; b += stride) {
+        uint32_t x = __ldg(p.states + 32ull * b + lane);
+        uint32_t base = __ldg(p.block_word + b);
+        const uint32_t end = __ldg(p.block_word + b + 1);
+        const bool full = (b + 1) * B <= p.n;  // warp-uniform
+        // the next block's words into L1, its sign/mantissa bytes into L2
+        if (b + stride < p.num_blocks) {
+            const uint32_t nb = b + stride;
+            const uint32_t w0 = __ldg(p.block_word + nb), w1 = __ldg(p.block_word + nb + 1);
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(p.words + w0) & ~(uintptr_t)127;
+            const uintptr_t a1 = reinterpret_cast<uintptr_t>(p.words + w1);
+            for (uintptr_t a = a0 + 128u * (uint32_t)lane; a < a1; a += 32u * 128u)
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a < reinterpret_cast<uintptr_t>(p.words + w0)
+                                                                    ? reinterpret_cast<uintptr_t>(p.words + w0)
+                                                                    : a));
+            const uint64_t s0 = nb * B, s1 = s0 + B < p.n ? s0 + B : p.n;
+            if (lane == 0 && s1 > s0)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + s0),
+                             "r"((uint32_t)(((s1 - s0) + 15) & ~15ull))
+                             : "memory");
+        }
+        for (uint32_t j = 0; j < p.chunks; j++) {
+            const uint64_t pos0 = b * B + 512ull * j + 16u * (uint32_t)lane;
+            uint32_t acc[4] = {0u, 0u, 0u, 0u};
+            if (full)
+                decode_chunk<true>(x, base, pos0, table, p, lt, acc);
+            else
+                decode_chunk<false>(x, base, pos0, table, p, lt, acc);
+            // merge with the 16 sign/mantissa bytes and store
+            if (pos0 + 16 <= p.n) {
+                const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(p.sm + pos0));
+                uint32_t r[8];
+                merge4(s4.x, acc[0], r[0], r[1]);
+                merge4(s4.y, acc[1], r[2], r[3]);
+                merge4(s4.z, acc[2], r[4], r[5]);
+                merge4(s4.w, acc[3], r[6], r[7]);
+                if (p.wide) {
+                    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p.dst + pos0),
+                                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                                 "r"(r[7])
+                                 : "memory");
+                } else {
+                    uint4 *d = reinterpret_cast<uint4 *>(p.dst + pos0);
+                    d[0] = make_uint4(r[0], r[1], r[2], r[3]);
+                    d[1] = make_uint4(r[4], r[5], r[6], r[7]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; i++)
+                    if (pos0 + i < p.n)
+                        p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+            }
+        }
+        const bool bad = x != kLow || base != end;
+        if (__any_sync(0xffffffffu, bad) && lane == 0)
+            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+    }
+}
+
+std::mutex g_rans_mu;
+int g_rans_sms[64] = {0};
+
+}  // namespace
+
+extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t *dst, uint32_t *status_dev,
+                                            void *stream)
+{
+    if (!a || !status_dev)
+        return DF11_ERR_INVALID_ARG;
+    if (a->n == 0)
+        return DF11_OK;
+    if (!dst || (reinterpret_cast<uintptr_t>(dst) & 15) || !a->words || !a->states || !a->block_word || !a->freq ||
+        !a->packed_sign_mantissa || (reinterpret_cast<uintptr_t>(a->packed_sign_mantissa) & 15))
+        return DF11_ERR_INVALID_ARG;
+    if (a->prob_bits != kProbBits || a->chunks < 1 || a->chunks > 64 || a->n >= (1ull << 32))
+        return DF11_ERR_INVALID_ARG;
+    const uint64_t B = 512ull * a->chunks;
+    if (a->num_blocks != (a->n + B - 1) / B || a->num_words + 8 >= (1ull << 32) ||
+        a->packed_sign_mantissa_bytes < ((a->n + 15) / 16) * 16)
+        return DF11_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return DF11_ERR_CUDA;
+    int sms = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_rans_mu);
+        if (!g_rans_sms[dev] &&
+            cudaDeviceGetAttribute(&g_rans_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return DF11_ERR_CUDA;
+        sms = g_rans_sms[dev];
+    }
+    RansParams p;
+    p.words = a->words;
+    p.states = a->states;
+    p.block_word = a->block_word;
+    p.freq = a->freq;
+    p.sm = a->packed_sign_mantissa;
+    p.dst = dst;
+    p.status = status_dev;
+    p.n = a->n;
+    p.last_word = (uint32_t)(a->num_words + 7);
+    p.num_blocks = a->num_blocks;
+    p.chunks = a->chunks;
+    p.wide = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
+    uint32_t grid = (a->num_blocks + kWarps - 1) / kWarps;
+    if (grid > (uint32_t)sms)
+        grid = (uint32_t)sms;
+    rans_decode_kernel<<<grid, kWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
+}

@@ -28,7 +28,11 @@
  *   - device encode: df11_device_histogram counts exponents of a device
  *     array; df11_device_encode (caller scratch) and
  *     df11_device_encode_static (library scratch) write the compressed
- *     arrays of a plan into device buffers.
+ *     arrays of a plan into device buffers;
+ *   - rANS variant of the exponent coder (the page's discussion proposes
+ *     rANS instead of Huffman coding): df11_rans_build compresses on the
+ *     host (df11_rans_format_arrays, df11_rans_free), df11_rans_decompress
+ *     rebuilds the BF16 matrix on the device.
  * No entry point takes or returns framework types; all pointers are plain
  * host or device addresses as stated per argument.
  *
@@ -401,6 +405,77 @@ df11_status df11_device_encode(const df11_format *plan, const uint16_t *w_dev, c
  */
 df11_status df11_device_encode_static(const df11_format *plan, const uint16_t *w_dev, const df11_arrays *dst_dev,
                                       uint32_t *max_block_elems_dev, uint32_t *status_dev, void *stream);
+
+/*
+ * rANS variant of the exponent coder.  The page's discussion proposes rANS
+ * (range asymmetric numeral systems) as an entropy coder better suited to
+ * SIMD-style hardware than Huffman coding; this variant codes the same 8-bit
+ * exponents with it and keeps sign and mantissa verbatim, so the same BF16
+ * matrix comes back bit for bit.  Layout (the pages fix none of it):
+ *   - model: exponent counts quantised to frequencies freq[256] summing to
+ *     2^prob_bits (12): every present exponent gets max(1, floor(h M / n)),
+ *     then the largest frequency (ties: smallest exponent) loses one while
+ *     the sum exceeds M, the largest count (ties: smallest exponent) gains
+ *     one while it falls short.  Every exponent 0..255 is allowed.
+ *   - state: 32 bits in [2^16, 2^32); a decode step takes slot = x mod M,
+ *     the exponent s whose range [cum[s], cum[s] + freq[s]) holds it, and
+ *     x = freq[s] (x >> prob_bits) + slot - cum[s]; below 2^16 the state
+ *     takes the next 16-bit word: x = (x << 16) | word.
+ *   - blocks of 512 * chunks elements; lane l (0..31) of block b owns
+ *     elements b 512 chunks + 512 j + 16 l + i (j < chunks, i < 16), decoded
+ *     in the order (j, i), all lanes stepping together; after a step the
+ *     lanes whose state fell below 2^16 take one word each, in lane order,
+ *     from the block's words; a lane skips steps whose element lies at or
+ *     past n.  Every lane ends the block at x = 2^16.
+ *   - states[32 b + l] is lane l's start state in block b; the words of
+ *     block b are words[block_word[b] .. block_word[b + 1]).
+ */
+typedef struct df11_rans_format df11_rans_format;
+
+typedef struct df11_rans_arrays {
+    uint64_t n;                          /* BF16 elements */
+    uint64_t num_words;                  /* 16-bit words of all blocks */
+    uint32_t prob_bits;                  /* 12 */
+    uint32_t chunks;                     /* 16-element chunks per lane and block, 1..64 */
+    uint32_t num_blocks;                 /* ceil(n / (512 chunks)) */
+    uint32_t max_block_words;            /* largest block_word[b + 1] - block_word[b] */
+    const uint16_t *words;               /* num_words + 8 (zero padding) */
+    const uint32_t *states;              /* 32 * num_blocks */
+    const uint32_t *block_word;          /* num_blocks + 1 */
+    const uint16_t *freq;                /* 256, summing to 2^prob_bits (0 when n = 0) */
+    const uint8_t *packed_sign_mantissa; /* round_up(n, 16) + 16 bytes, 16-B aligned */
+    uint64_t packed_sign_mantissa_bytes;
+} df11_rans_arrays;
+
+/*
+ * df11_rans_build -- host: compress num_mats BF16 matrices (as
+ * df11_build_format; matrices concatenated) with the rANS exponent coder.
+ *   chunks: 16-element chunks per lane and block (0 = 8: 4096-element blocks).
+ * On success *out owns every array (host memory); DF11_ERR_TOO_LARGE for
+ * n >= 2^32, DF11_ERR_INVALID_ARG for bad pointers or chunks > 64.
+ */
+df11_status df11_rans_build(const uint16_t *const *mats, const uint64_t *counts, int num_mats, uint32_t chunks,
+                            df11_rans_format **out);
+
+/* df11_rans_format_arrays -- borrowed host pointers and sizes of a built
+ * stream (valid until df11_rans_free). */
+df11_status df11_rans_format_arrays(const df11_rans_format *f, df11_rans_arrays *out);
+
+/* df11_rans_free -- releases a stream (NULL-safe). */
+void df11_rans_free(df11_rans_format *f);
+
+/*
+ * df11_rans_decompress -- device: rebuild the n BF16 values of a stream whose
+ * arrays the caller has uploaded (dev: the same struct with device pointers)
+ * into dst_dev (16-byte aligned, n elements), asynchronously on `stream`.
+ * One warp decodes one block; the exponents of a lane's 16 elements are
+ * merged with their sign/mantissa bytes and stored with one 32-byte store.
+ * Inconsistent words, states or offsets set DF11_ERR_CORRUPT in
+ * *status_dev (caller-zeroed) and leave that block's outputs unspecified;
+ * nothing traps.  Argument errors return DF11_ERR_INVALID_ARG synchronously.
+ */
+df11_status df11_rans_decompress(const df11_rans_arrays *dev, uint16_t *dst_dev, uint32_t *status_dev,
+                                 void *stream);
 
 #ifdef __cplusplus
 }

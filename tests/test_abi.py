@@ -43,9 +43,11 @@ def test_struct_sizes_match_c():
 #include <stddef.h>
 #include "df11.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(df11_arrays), offsetof(df11_arrays, encoded_exponent),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(df11_arrays), offsetof(df11_arrays, encoded_exponent),
          offsetof(df11_arrays, code_lengths), sizeof(df11_info), offsetof(df11_info, histogram),
-         sizeof(df11_gemv_matrix), offsetof(df11_gemv_matrix, x), offsetof(df11_gemv_matrix, y));
+         sizeof(df11_gemv_matrix), offsetof(df11_gemv_matrix, x), offsetof(df11_gemv_matrix, y),
+         sizeof(df11_rans_arrays), offsetof(df11_rans_arrays, words),
+         offsetof(df11_rans_arrays, packed_sign_mantissa_bytes));
   return 0;
 }
 '''
@@ -56,9 +58,10 @@ int main(void) {
         open(c, "w").write(src)
         subprocess.run(["gcc", "-I", HEADER_DIR, c, "-o", exe], check=True)
         got = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
-    A, I, G = df11.df11_arrays, df11.df11_info, df11.df11_gemv_matrix
+    A, I, G, R = df11.df11_arrays, df11.df11_info, df11.df11_gemv_matrix, df11.df11_rans_arrays
     assert got == [ctypes.sizeof(A), A.encoded_exponent.offset, A.code_lengths.offset,
-                   ctypes.sizeof(I), I.histogram.offset, ctypes.sizeof(G), G.x.offset, G.y.offset]
+                   ctypes.sizeof(I), I.histogram.offset, ctypes.sizeof(G), G.x.offset, G.y.offset,
+                   ctypes.sizeof(R), R.words.offset, R.packed_sign_mantissa_bytes.offset]
 
 
 def test_strerror_covers_all_codes():

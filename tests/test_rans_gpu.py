@@ -1,0 +1,92 @@
+"""GPU decoder of the rANS variant (df11_rans_decompress) against the
+original bits and the CPU oracle's decode, through the C ABI."""
+import numpy as np
+import pytest
+
+import huffman_decode_03_b200 as df11
+from huffman_decode_03_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def torch_cuda():
+    import torch
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch
+
+
+def gpu_decode(w, chunks=8, out=None):
+    torch = torch_cuda()
+    fmt = df11.rans_build_format(w, chunks)
+    dev = df11.RansDeviceFormat(fmt, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = df11.rans_decompress(dev, out, status)
+    assert df11.read_status(status) == 0
+    return got[: w.size].view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("n", [1, 15, 16, 17, 511, 512, 4095, 4096, 4097, 3 * 4096 + 100, 1_000_003])
+def test_round_trip_against_the_oracle(oracle_mod, n):
+    w = inputs.gaussian(n, [100, n])
+    got = gpu_decode(w)
+    assert np.array_equal(got, w)
+    ref = oracle_mod.rans_decode_format(oracle_mod.rans_build_format(w))
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("chunks", [1, 2, 16, 64])
+def test_chunks(chunks):
+    w = inputs.stress(300_007, key=(101, chunks))
+    assert np.array_equal(gpu_decode(w, chunks), w)
+
+
+def test_every_pattern_and_one_symbol():
+    rng = np.random.default_rng(102)
+    allp = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    rng.shuffle(allp)
+    assert np.array_equal(gpu_decode(np.tile(allp, 5)), np.tile(allp, 5))
+    one = np.full(50_001, 0xBF80, np.uint16)
+    assert np.array_equal(gpu_decode(one), one)
+
+
+def test_output_alignment_and_neighbours():
+    torch = torch_cuda()
+    w = inputs.gaussian(70_011, [103])
+    for shift in (0, 8):  # 32-byte and 16-byte aligned outputs
+        buf = torch.full((w.size + 64,), -1, dtype=torch.int16, device="cuda")
+        out = buf[shift: shift + w.size].view(torch.bfloat16)
+        gpu_decode(w, 8, out)
+        host = buf.cpu().numpy().view(np.uint16)
+        assert np.array_equal(host[shift: shift + w.size], w)
+        assert np.all(host[:shift] == 0xFFFF) and np.all(host[shift + w.size:] == 0xFFFF)
+
+
+@pytest.mark.parametrize("workload", [2, 3])
+def test_workloads(workload):
+    mats = [m for _, _, m in inputs.workload_arrays(workload, 0)]
+    w = np.concatenate(mats) if len(mats) > 1 else mats[0]
+    assert np.array_equal(gpu_decode(w), w)
+
+
+def test_corruption_is_reported():
+    torch = torch_cuda()
+    w = inputs.gaussian(200_000, [104])
+    fmt = df11.rans_build_format(w)
+    for name, edit in (("states", lambda t: t.view(torch.int32).__setitem__(5, 12345)),
+                       ("block_word", lambda t: t.view(torch.int32).__setitem__(3, int(t.view(torch.int32)[3]) + 1)),
+                       ("freq", lambda t: t.view(torch.int16).__setitem__(120, 7))):
+        dev = df11.RansDeviceFormat(fmt, "cuda")
+        edit(dev.tensors[name])
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.rans_decompress(dev, None, status)
+        assert df11.read_status(status) != 0, name
+
+
+def test_repeated_launches_are_identical():
+    torch = torch_cuda()
+    w = inputs.gaussian(1 << 20, [105])
+    dev = df11.RansDeviceFormat(df11.rans_build_format(w), "cuda")
+    a = df11.rans_decompress(dev)
+    b = df11.rans_decompress(dev)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
