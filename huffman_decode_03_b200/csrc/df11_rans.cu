@@ -14,12 +14,16 @@
 // rotated right by one bit for the merge, slot - cum and freq - 1), one
 // multiply-add for the new state, and, when the state falls below 2^16, one
 // 16-bit word: the lanes that need one take consecutive words of the block
-// in lane order (ballot, popcount of the lanes below).  The next block's words
-// are prefetched into L1 and its sign/mantissa bytes into L2 while the
-// current block decodes.  Every lane must end the block at x = 2^16 and the
-// block must use exactly its words; otherwise DF11_ERR_CORRUPT is set.  Word
-// reads are clamped to the padded array, so inconsistent data never reads
-// out of bounds; nothing traps and every loop has a fixed trip count.
+// in lane order (ballot, popcount of the lanes below).  A block's words are
+// read from shared memory: each warp has two buffers, and the next block's
+// words are copied into the other one (cp.async) and its sign/mantissa bytes
+// prefetched into L2 while the current block decodes.  The warps per CTA are
+// as many as the buffers fit (32 for blocks of up to about 1,650 words).
+// Every lane must end the block at x = 2^16 and the block must use exactly
+// its words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped to the
+// padded array and to the buffer, word reads to the buffer, so inconsistent
+// data never reads out of bounds; nothing traps and every loop has a fixed
+// trip count.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -32,7 +36,7 @@ namespace {
 constexpr uint32_t kProbBits = 12;
 constexpr uint32_t kSlots = 1u << kProbBits;
 constexpr uint32_t kLow = 1u << 16;
-constexpr int kWarps = 32;
+constexpr int kMaxWarps = 32;
 
 struct RansParams {
     const uint16_t *words;
@@ -43,10 +47,11 @@ struct RansParams {
     uint16_t *dst;
     uint32_t *status;
     uint64_t n;
-    uint32_t last_word;  // index of the last readable word (num_words + 7)
     uint32_t num_blocks;
     uint32_t chunks;
     uint32_t wide;  // dst is 32-byte aligned: 32-byte stores
+    uint32_t cap;        // words of one block buffer in shared memory (multiple of 8, >= max block words + 14)
+    uint32_t words_end;  // copies end at or below this word: num_words rounded down to 8, plus the 8 padding words
 };
 
 __device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
@@ -77,7 +82,7 @@ __device__ __forceinline__ uint32_t lanemask_lt()
 // lane's element exists; acc receives the exponent byte at byte position Q.
 template <int Q>
 __device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base, bool valid, const uint32_t *table,
-                                     const RansParams &p, uint32_t lt)
+                                     const uint16_t *wb, const RansParams &p, uint32_t lt)
 {
     if (valid) {
         const uint32_t e = table[x & (kSlots - 1)];
@@ -89,9 +94,9 @@ __device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base,
     const uint32_t m = __ballot_sync(0xffffffffu, need);
     if (m) {  // warp-uniform
         if (need) {
-            uint32_t i = base + __popc(m & lt);
-            i = i < p.last_word ? i : p.last_word;
-            x = (x << 16) | __ldg(p.words + i);
+            uint32_t i = base + __popc(m & lt);  // relative to the buffer's first word
+            i = i < p.cap ? i : p.cap - 1;
+            x = (x << 16) | wb[i];
         }
         base += __popc(m);
     }
@@ -99,10 +104,10 @@ __device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base,
 
 template <bool FULL>
 __device__ __forceinline__ void decode_chunk(uint32_t &x, uint32_t &base, uint64_t pos0, const uint32_t *table,
-                                             const RansParams &p, uint32_t lt, uint32_t acc[4])
+                                             const uint16_t *wb, const RansParams &p, uint32_t lt, uint32_t acc[4])
 {
 #define DF11_STEP(I) \
-    step<(I) & 3>(x, acc[(I) >> 2], base, FULL || pos0 + (I) < p.n, table, p, lt)
+    step<(I) & 3>(x, acc[(I) >> 2], base, FULL || pos0 + (I) < p.n, table, wb, p, lt)
     DF11_STEP(0); DF11_STEP(1); DF11_STEP(2); DF11_STEP(3);
     DF11_STEP(4); DF11_STEP(5); DF11_STEP(6); DF11_STEP(7);
     DF11_STEP(8); DF11_STEP(9); DF11_STEP(10); DF11_STEP(11);
@@ -110,10 +115,29 @@ __device__ __forceinline__ void decode_chunk(uint32_t &x, uint32_t &base, uint64
 #undef DF11_STEP
 }
 
-__global__ void __launch_bounds__(kWarps * 32, 1) rans_decode_kernel(const RansParams p)
+// Asynchronous copy (cp.async) of block b's words into a warp buffer at
+// shared address buf: from the 16-byte boundary at or below its first word
+// to the one at or above its end (inside the array's 8-word padding), one
+// commit group.  Returns the index of the buffer's first word.
+__device__ __forceinline__ uint32_t copy_words(const RansParams &p, uint32_t b, int lane, uint32_t buf)
+{
+    const uint32_t w0 = __ldg(p.block_word + b) & ~7u;
+    uint32_t w1 = (__ldg(p.block_word + b + 1) + 7u) & ~7u;
+    // inconsistent offsets: copy what fits the buffer and the array
+    w1 = w1 < p.words_end ? w1 : p.words_end;
+    const uint32_t w1c = w1 <= w0 ? w0 : (w1 - w0 <= p.cap ? w1 : w0 + p.cap);
+    for (uint32_t o = 8u * (uint32_t)lane; w0 + o < w1c; o += 256u)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(buf + 2u * o), "l"(p.words + w0 + o)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    return w0;
+}
+
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const RansParams p)
 {
     __shared__ uint32_t table[kSlots];
     __shared__ uint32_t cum[257];
+    extern __shared__ __align__(16) uint16_t wbufs[];  // per warp: two buffers of cap words
     const uint32_t tid = threadIdx.x, warp = tid >> 5;
     const int lane = (int)(tid & 31u);
 
@@ -165,22 +189,25 @@ __global__ void __launch_bounds__(kWarps * 32, 1) rans_decode_kernel(const RansP
 
     const uint32_t lt = lanemask_lt();
     const uint64_t B = 512ull * p.chunks;
-    const uint32_t stride = gridDim.x * kWarps;
-    for (uint32_t b = blockIdx.x * kWarps + warp; b < p.num_blocks; b += stride) {
+    const uint32_t warps = blockDim.x >> 5, stride = gridDim.x * warps;
+    uint16_t *wbuf = wbufs + 2u * p.cap * warp;
+    const uint32_t wbuf_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
+    uint32_t b = blockIdx.x * warps + warp, k = 0;
+    uint32_t wfirst = b < p.num_blocks ? copy_words(p, b, lane, wbuf_s) : 0u;
+    for (; b < p.num_blocks; b += stride, k ^= 1u) {
+        // this block's words have landed; the next block's go to the other buffer
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncwarp();
+        const uint16_t *wb = wbuf + k * p.cap;
+        const uint32_t wfirst_cur = wfirst;
         uint32_t x = __ldg(p.states + 32ull * b + lane);
-        uint32_t base = __ldg(p.block_word + b);
-        const uint32_t end = __ldg(p.block_word + b + 1);
+        uint32_t base = __ldg(p.block_word + b) - wfirst_cur;
+        const uint32_t end = __ldg(p.block_word + b + 1) - wfirst_cur;
         const bool full = (b + 1) * B <= p.n;  // warp-uniform
-        // the next block's words into L1, its sign/mantissa bytes into L2
+        // the next block's words into the other buffer, its sign/mantissa bytes into L2
         if (b + stride < p.num_blocks) {
             const uint32_t nb = b + stride;
-            const uint32_t w0 = __ldg(p.block_word + nb), w1 = __ldg(p.block_word + nb + 1);
-            const uintptr_t a0 = reinterpret_cast<uintptr_t>(p.words + w0) & ~(uintptr_t)127;
-            const uintptr_t a1 = reinterpret_cast<uintptr_t>(p.words + w1);
-            for (uintptr_t a = a0 + 128u * (uint32_t)lane; a < a1; a += 32u * 128u)
-                asm volatile("prefetch.global.L1 [%0];" ::"l"(a < reinterpret_cast<uintptr_t>(p.words + w0)
-                                                                    ? reinterpret_cast<uintptr_t>(p.words + w0)
-                                                                    : a));
+            wfirst = copy_words(p, nb, lane, wbuf_s + 2u * p.cap * (k ^ 1u));
             const uint64_t s0 = nb * B, s1 = s0 + B < p.n ? s0 + B : p.n;
             if (lane == 0 && s1 > s0)
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + s0),
@@ -191,9 +218,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) rans_decode_kernel(const RansP
             const uint64_t pos0 = b * B + 512ull * j + 16u * (uint32_t)lane;
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
             if (full)
-                decode_chunk<true>(x, base, pos0, table, p, lt, acc);
+                decode_chunk<true>(x, base, pos0, table, wb, p, lt, acc);
             else
-                decode_chunk<false>(x, base, pos0, table, p, lt, acc);
+                decode_chunk<false>(x, base, pos0, table, wb, p, lt, acc);
             // merge with the 16 sign/mantissa bytes and store
             if (pos0 + 16 <= p.n) {
                 const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(p.sm + pos0));
@@ -219,14 +246,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) rans_decode_kernel(const RansP
                         p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
             }
         }
-        const bool bad = x != kLow || base != end;
+        const bool bad = x != kLow || base != end || end > p.cap;
         if (__any_sync(0xffffffffu, bad) && lane == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+        __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 }
 
 std::mutex g_rans_mu;
 int g_rans_sms[64] = {0};
+int g_rans_optin[64] = {0};
+uint32_t g_rans_granted[64] = {0};
 
 }  // namespace
 
@@ -237,7 +267,8 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
         return DF11_ERR_INVALID_ARG;
     if (a->n == 0)
         return DF11_OK;
-    if (!dst || (reinterpret_cast<uintptr_t>(dst) & 15) || !a->words || !a->states || !a->block_word || !a->freq ||
+    if (!dst || (reinterpret_cast<uintptr_t>(dst) & 15) || !a->words || (reinterpret_cast<uintptr_t>(a->words) & 15) ||
+        !a->states || !a->block_word || !a->freq ||
         !a->packed_sign_mantissa || (reinterpret_cast<uintptr_t>(a->packed_sign_mantissa) & 15))
         return DF11_ERR_INVALID_ARG;
     if (a->prob_bits != kProbBits || a->chunks < 1 || a->chunks > 64 || a->n >= (1ull << 32))
@@ -249,13 +280,15 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return DF11_ERR_CUDA;
-    int sms = 0;
+    int sms = 0, optin = 0;
     {
         std::lock_guard<std::mutex> lock(g_rans_mu);
         if (!g_rans_sms[dev] &&
-            cudaDeviceGetAttribute(&g_rans_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            (cudaDeviceGetAttribute(&g_rans_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+             cudaDeviceGetAttribute(&g_rans_optin[dev], cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess))
             return DF11_ERR_CUDA;
         sms = g_rans_sms[dev];
+        optin = g_rans_optin[dev];
     }
     RansParams p;
     p.words = a->words;
@@ -266,13 +299,29 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     p.dst = dst;
     p.status = status_dev;
     p.n = a->n;
-    p.last_word = (uint32_t)(a->num_words + 7);
     p.num_blocks = a->num_blocks;
     p.chunks = a->chunks;
     p.wide = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
-    uint32_t grid = (a->num_blocks + kWarps - 1) / kWarps;
+    p.cap = ((a->max_block_words + 16u) + 7u) & ~7u;
+    p.words_end = (uint32_t)((a->num_words & ~7ull) + 8);
+    // two buffers of cap words per warp; as many warps as shared memory holds
+    const uint64_t per_warp = 4ull * p.cap, room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
+    const uint64_t warps = room / per_warp < (uint64_t)kMaxWarps ? room / per_warp : (uint64_t)kMaxWarps;
+    if (warps == 0)
+        return DF11_ERR_INVALID_ARG;  // cannot happen for chunks <= 64 (at most 24,576 words per block)
+    const uint64_t dyn = per_warp * warps;
+    {
+        std::lock_guard<std::mutex> lock(g_rans_mu);
+        if (dyn > g_rans_granted[dev]) {
+            if (cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) !=
+                cudaSuccess)
+                return DF11_ERR_CUDA;
+            g_rans_granted[dev] = (uint32_t)dyn;
+        }
+    }
+    uint32_t grid = (uint32_t)((a->num_blocks + warps - 1) / warps);
     if (grid > (uint32_t)sms)
         grid = (uint32_t)sms;
-    rans_decode_kernel<<<grid, kWarps * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    rans_decode_kernel<<<grid, (uint32_t)(warps * 32), (size_t)dyn, reinterpret_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
