@@ -92,22 +92,20 @@ __device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base,
     }
     const bool need = valid && x < kLow;
     const uint32_t m = __ballot_sync(0xffffffffu, need);
-    if (m) {  // warp-uniform
-        if (need) {
-            uint32_t i = base + __popc(m & lt);  // relative to the buffer's first word
-            i = i < p.cap ? i : p.cap - 1;
-            x = (x << 16) | wb[i];
-        }
-        base += __popc(m);
+    if (need) {
+        uint32_t i = base + __popc(m & lt);  // relative to the buffer's first word
+        i = i < p.cap ? i : p.cap - 1;
+        x = (x << 16) | wb[i];
     }
+    base += __popc(m);
 }
 
-template <bool FULL>
-__device__ __forceinline__ void decode_chunk(uint32_t &x, uint32_t &base, uint64_t pos0, const uint32_t *table,
-                                             const uint16_t *wb, const RansParams &p, uint32_t lt, uint32_t acc[4])
+// 16 steps of the last, partial block: elements past n are skipped.
+__device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, uint64_t pos0, const uint32_t *table,
+                                                  const uint16_t *wb, const RansParams &p, uint32_t lt,
+                                                  uint32_t acc[4])
 {
-#define DF11_STEP(I) \
-    step<(I) & 3>(x, acc[(I) >> 2], base, FULL || pos0 + (I) < p.n, table, wb, p, lt)
+#define DF11_STEP(I) step<(I) & 3>(x, acc[(I) >> 2], base, pos0 + (I) < p.n, table, wb, p, lt)
     DF11_STEP(0); DF11_STEP(1); DF11_STEP(2); DF11_STEP(3);
     DF11_STEP(4); DF11_STEP(5); DF11_STEP(6); DF11_STEP(7);
     DF11_STEP(8); DF11_STEP(9); DF11_STEP(10); DF11_STEP(11);
@@ -115,14 +113,58 @@ __device__ __forceinline__ void decode_chunk(uint32_t &x, uint32_t &base, uint64
 #undef DF11_STEP
 }
 
-// Asynchronous copy (cp.async) of block b's words into a warp buffer at
-// shared address buf: from the 16-byte boundary at or below its first word
-// to the one at or above its end (inside the array's 8-word padding), one
-// commit group.  Returns the index of the buffer's first word.
-__device__ __forceinline__ uint32_t copy_words(const RansParams &p, uint32_t b, int lane, uint32_t buf)
+// One step of a full block in PTX, the same arithmetic as step() with the
+// word read predicated instead of branched around.  Operands: %0 the state,
+// %1 the shared address of the warp's next word, A the accumulator that
+// takes the exponent byte at the position SEL selects, %6 the table's
+// shared address, %7 the lanes-below mask, %8 the buffer's last word.
+#define DF11_RSTEP(A, SEL)                       \
+    "and.b32 ts, %0, 4095;\n\t"                  \
+    "shl.b32 ts, ts, 2;\n\t"                     \
+    "add.u32 ts, ts, %6;\n\t"                    \
+    "ld.shared.u32 te, [ts];\n\t"                \
+    "shr.u32 th, %0, 12;\n\t"                    \
+    "shr.u32 tf, te, 20;\n\t"                    \
+    "bfe.u32 to, te, 8, 12;\n\t"                 \
+    "mad.lo.u32 %0, tf, th, th;\n\t"             \
+    "add.u32 %0, %0, to;\n\t"                    \
+    "prmt.b32 " A ", " A ", te, " SEL ";\n\t"    \
+    "setp.lt.u32 tp, %0, 65536;\n\t"             \
+    "vote.sync.ballot.b32 tm, tp, 0xffffffff;\n\t" \
+    "and.b32 tt, tm, %7;\n\t"                    \
+    "popc.b32 tt, tt;\n\t"                       \
+    "mad.lo.u32 ta, tt, 2, %1;\n\t"              \
+    "min.u32 ta, ta, %8;\n\t"                    \
+    "@tp ld.shared.u16 tw, [ta];\n\t"            \
+    "@tp prmt.b32 %0, tw, %0, 0x5410;\n\t"       \
+    "popc.b32 tt, tm;\n\t"                       \
+    "mad.lo.u32 %1, tt, 2, %1;\n\t"
+#define DF11_RSTEP4(A) \
+    DF11_RSTEP(A, "0x3214") DF11_RSTEP(A, "0x3240") DF11_RSTEP(A, "0x3410") DF11_RSTEP(A, "0x4210")
+
+// 16 steps of a full block (all lanes valid, warp converged).
+__device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wa, uint32_t tbl, uint32_t lt, uint32_t last,
+                                                  uint32_t acc[4])
 {
-    const uint32_t w0 = __ldg(p.block_word + b) & ~7u;
-    uint32_t w1 = (__ldg(p.block_word + b + 1) + 7u) & ~7u;
+    asm volatile("{\n\t.reg .b32 ts, te, th, tf, to, tt, ta, tw, tm;\n\t.reg .pred tp;\n\t"
+                 DF11_RSTEP4("%2") DF11_RSTEP4("%3") DF11_RSTEP4("%4") DF11_RSTEP4("%5")
+                 "}"
+                 : "+r"(x), "+r"(wa), "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
+                 : "r"(tbl), "r"(lt), "r"(last)
+                 : "memory");
+}
+#undef DF11_RSTEP4
+#undef DF11_RSTEP
+
+// Asynchronous copy (cp.async) of a block's words [bw0, bw1) into a warp
+// buffer at shared address buf: from the 16-byte boundary at or below bw0 to
+// the one at or above bw1 (inside the array's 8-word padding), one commit
+// group.  Returns the index of the buffer's first word.
+__device__ __forceinline__ uint32_t copy_words(const RansParams &p, uint32_t bw0, uint32_t bw1, int lane,
+                                               uint32_t buf)
+{
+    const uint32_t w0 = bw0 & ~7u;
+    uint32_t w1 = (bw1 + 7u) & ~7u;
     // inconsistent offsets: copy what fits the buffer and the array
     w1 = w1 < p.words_end ? w1 : p.words_end;
     const uint32_t w1c = w1 <= w0 ? w0 : (w1 - w0 <= p.cap ? w1 : w0 + p.cap);
@@ -131,6 +173,12 @@ __device__ __forceinline__ uint32_t copy_words(const RansParams &p, uint32_t b, 
                      : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
     return w0;
+}
+
+// The 16 sign/mantissa bytes at pos (a multiple of 16), or zeros past the end.
+__device__ __forceinline__ uint4 load_sm(const RansParams &p, uint64_t pos)
+{
+    return pos < p.n ? __ldg(reinterpret_cast<const uint4 *>(p.sm + pos)) : make_uint4(0u, 0u, 0u, 0u);
 }
 
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const RansParams p)
@@ -192,38 +240,55 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
     const uint32_t warps = blockDim.x >> 5, stride = gridDim.x * warps;
     uint16_t *wbuf = wbufs + 2u * p.cap * warp;
     const uint32_t wbuf_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
+    const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(table));
     uint32_t b = blockIdx.x * warps + warp, k = 0;
-    uint32_t wfirst = b < p.num_blocks ? copy_words(p, b, lane, wbuf_s) : 0u;
+    // software pipeline: the next block's state and word offsets, and the
+    // next chunk's sign/mantissa bytes, are loaded one step ahead
+    uint32_t x_n = 0, bw0_n = 0, bw1_n = 0, wfirst = 0;
+    uint4 s_n = make_uint4(0u, 0u, 0u, 0u);
+    if (b < p.num_blocks) {
+        x_n = __ldg(p.states + 32ull * b + lane);
+        bw0_n = __ldg(p.block_word + b);
+        bw1_n = __ldg(p.block_word + b + 1);
+        wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s);
+        s_n = load_sm(p, b * B + 16u * (uint32_t)lane);
+    }
     for (; b < p.num_blocks; b += stride, k ^= 1u) {
         // this block's words have landed; the next block's go to the other buffer
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncwarp();
         const uint16_t *wb = wbuf + k * p.cap;
-        const uint32_t wfirst_cur = wfirst;
-        uint32_t x = __ldg(p.states + 32ull * b + lane);
-        uint32_t base = __ldg(p.block_word + b) - wfirst_cur;
-        const uint32_t end = __ldg(p.block_word + b + 1) - wfirst_cur;
+        const uint32_t wb_s = wbuf_s + 2u * p.cap * k, last = wb_s + 2u * (p.cap - 1u);
+        uint32_t x = x_n;
+        uint32_t wa = wb_s + 2u * (bw0_n - wfirst);  // bw0 - wfirst = bw0 mod 8
+        const uint32_t end = bw1_n - wfirst;
         const bool full = (b + 1) * B <= p.n;  // warp-uniform
-        // the next block's words into the other buffer, its sign/mantissa bytes into L2
-        if (b + stride < p.num_blocks) {
-            const uint32_t nb = b + stride;
-            wfirst = copy_words(p, nb, lane, wbuf_s + 2u * p.cap * (k ^ 1u));
+        const uint32_t nb = b + stride;
+        if (nb < p.num_blocks) {
+            x_n = __ldg(p.states + 32ull * nb + lane);
+            bw0_n = __ldg(p.block_word + nb);
+            bw1_n = __ldg(p.block_word + nb + 1);
+            wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.cap * (k ^ 1u));
             const uint64_t s0 = nb * B, s1 = s0 + B < p.n ? s0 + B : p.n;
-            if (lane == 0 && s1 > s0)
+            if (lane == 0)
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + s0),
                              "r"((uint32_t)(((s1 - s0) + 15) & ~15ull))
                              : "memory");
         }
         for (uint32_t j = 0; j < p.chunks; j++) {
             const uint64_t pos0 = b * B + 512ull * j + 16u * (uint32_t)lane;
+            const uint4 s4 = s_n;
+            s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512 : (uint64_t)nb * B + 16u * (uint32_t)lane);
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
-            if (full)
-                decode_chunk<true>(x, base, pos0, table, wb, p, lt, acc);
-            else
-                decode_chunk<false>(x, base, pos0, table, wb, p, lt, acc);
+            if (full) {
+                decode_chunk_full(x, wa, tbl, lt, last, acc);
+            } else {
+                uint32_t base = (wa - wb_s) >> 1;
+                decode_chunk_tail(x, base, pos0, table, wb, p, lt, acc);
+                wa = wb_s + 2u * base;
+            }
             // merge with the 16 sign/mantissa bytes and store
             if (pos0 + 16 <= p.n) {
-                const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(p.sm + pos0));
                 uint32_t r[8];
                 merge4(s4.x, acc[0], r[0], r[1]);
                 merge4(s4.y, acc[1], r[2], r[3]);
@@ -246,7 +311,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
                         p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
             }
         }
-        const bool bad = x != kLow || base != end || end > p.cap;
+        const bool bad = x != kLow || wa != wb_s + 2u * end || end > p.cap;
         if (__any_sync(0xffffffffu, bad) && lane == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         __syncwarp();  // every lane is done with this buffer before it is refilled
