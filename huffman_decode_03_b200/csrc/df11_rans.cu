@@ -18,12 +18,14 @@
 // read from shared memory: each warp has two buffers, and the next block's
 // words are copied into the other one (cp.async) and its sign/mantissa bytes
 // prefetched into L2 while the current block decodes.  The warps per CTA are
-// as many as the buffers fit (32 for blocks of up to about 1,650 words).
+// as many as the buffers fit (32 for blocks of up to about 1,140 words).
 // Every lane must end the block at x = 2^16 and the block must use exactly
 // its words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped to the
-// padded array and to the buffer, word reads to the buffer, so inconsistent
-// data never reads out of bounds; nothing traps and every loop has a fixed
-// trip count.
+// padded array and to the buffer.  Full blocks check the word address once
+// per 16 steps (a chunk reads at most 512 words, and each buffer has 512
+// words of slack past the copied ones); the partial last block clamps every
+// read.  So inconsistent data never reads out of bounds; nothing traps and
+// every loop has a fixed trip count.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -50,7 +52,8 @@ struct RansParams {
     uint32_t num_blocks;
     uint32_t chunks;
     uint32_t wide;  // dst is 32-byte aligned: 32-byte stores
-    uint32_t cap;        // words of one block buffer in shared memory (multiple of 8, >= max block words + 14)
+    uint32_t cap;        // words a block may copy into its buffer (multiple of 8, >= max block words + 14)
+    uint32_t bufw;       // words of one buffer: cap plus 512 words of slack for one chunk's reads
     uint32_t words_end;  // copies end at or below this word: num_words rounded down to 8, plus the 8 padding words
 };
 
@@ -117,7 +120,8 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, u
 // word read predicated instead of branched around.  Operands: %0 the state,
 // %1 the shared address of the warp's next word, A the accumulator that
 // takes the exponent byte at the position SEL selects, %6 the table's
-// shared address, %7 the lanes-below mask, %8 the buffer's last word.
+// shared address, %7 the lanes-below mask.  No clamp: a chunk reads at most
+// 512 words past %1, and the buffer's slack holds them.
 #define DF11_RSTEP(A, SEL)                       \
     "and.b32 ts, %0, 4095;\n\t"                  \
     "shl.b32 ts, ts, 2;\n\t"                     \
@@ -134,7 +138,6 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, u
     "and.b32 tt, tm, %7;\n\t"                    \
     "popc.b32 tt, tt;\n\t"                       \
     "mad.lo.u32 ta, tt, 2, %1;\n\t"              \
-    "min.u32 ta, ta, %8;\n\t"                    \
     "@tp ld.shared.u16 tw, [ta];\n\t"            \
     "@tp prmt.b32 %0, tw, %0, 0x5410;\n\t"       \
     "popc.b32 tt, tm;\n\t"                       \
@@ -143,14 +146,13 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, u
     DF11_RSTEP(A, "0x3214") DF11_RSTEP(A, "0x3240") DF11_RSTEP(A, "0x3410") DF11_RSTEP(A, "0x4210")
 
 // 16 steps of a full block (all lanes valid, warp converged).
-__device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wa, uint32_t tbl, uint32_t lt, uint32_t last,
-                                                  uint32_t acc[4])
+__device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wa, uint32_t tbl, uint32_t lt, uint32_t acc[4])
 {
     asm volatile("{\n\t.reg .b32 ts, te, th, tf, to, tt, ta, tw, tm;\n\t.reg .pred tp;\n\t"
                  DF11_RSTEP4("%2") DF11_RSTEP4("%3") DF11_RSTEP4("%4") DF11_RSTEP4("%5")
                  "}"
                  : "+r"(x), "+r"(wa), "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
-                 : "r"(tbl), "r"(lt), "r"(last)
+                 : "r"(tbl), "r"(lt)
                  : "memory");
 }
 #undef DF11_RSTEP4
@@ -238,7 +240,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
     const uint32_t lt = lanemask_lt();
     const uint64_t B = 512ull * p.chunks;
     const uint32_t warps = blockDim.x >> 5, stride = gridDim.x * warps;
-    uint16_t *wbuf = wbufs + 2u * p.cap * warp;
+    uint16_t *wbuf = wbufs + 2u * p.bufw * warp;
     const uint32_t wbuf_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
     const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(table));
     uint32_t b = blockIdx.x * warps + warp, k = 0;
@@ -257,8 +259,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         // this block's words have landed; the next block's go to the other buffer
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncwarp();
-        const uint16_t *wb = wbuf + k * p.cap;
-        const uint32_t wb_s = wbuf_s + 2u * p.cap * k, last = wb_s + 2u * (p.cap - 1u);
+        const uint16_t *wb = wbuf + k * p.bufw;
+        const uint32_t wb_s = wbuf_s + 2u * p.bufw * k;
+        bool bad = false;
         uint32_t x = x_n;
         uint32_t wa = wb_s + 2u * (bw0_n - wfirst);  // bw0 - wfirst = bw0 mod 8
         const uint32_t end = bw1_n - wfirst;
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
             x_n = __ldg(p.states + 32ull * nb + lane);
             bw0_n = __ldg(p.block_word + nb);
             bw1_n = __ldg(p.block_word + nb + 1);
-            wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.cap * (k ^ 1u));
+            wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.bufw * (k ^ 1u));
             const uint64_t s0 = nb * B, s1 = s0 + B < p.n ? s0 + B : p.n;
             if (lane == 0)
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + s0),
@@ -280,8 +283,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
             const uint4 s4 = s_n;
             s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512 : (uint64_t)nb * B + 16u * (uint32_t)lane);
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
+            if (wa > wb_s + 2u * p.cap) {  // past the copied words: inconsistent data
+                wa = wb_s;
+                bad = true;
+            }
             if (full) {
-                decode_chunk_full(x, wa, tbl, lt, last, acc);
+                decode_chunk_full(x, wa, tbl, lt, acc);
             } else {
                 uint32_t base = (wa - wb_s) >> 1;
                 decode_chunk_tail(x, base, pos0, table, wb, p, lt, acc);
@@ -311,7 +318,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
                         p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
             }
         }
-        const bool bad = x != kLow || wa != wb_s + 2u * end || end > p.cap;
+        bad = bad || x != kLow || wa != wb_s + 2u * end || end > p.cap;
         if (__any_sync(0xffffffffu, bad) && lane == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         __syncwarp();  // every lane is done with this buffer before it is refilled
@@ -370,7 +377,8 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     p.cap = ((a->max_block_words + 16u) + 7u) & ~7u;
     p.words_end = (uint32_t)((a->num_words & ~7ull) + 8);
     // two buffers of cap words per warp; as many warps as shared memory holds
-    const uint64_t per_warp = 4ull * p.cap, room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
+    p.bufw = p.cap + 512u;
+    const uint64_t per_warp = 4ull * p.bufw, room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
     const uint64_t warps = room / per_warp < (uint64_t)kMaxWarps ? room / per_warp : (uint64_t)kMaxWarps;
     if (warps == 0)
         return DF11_ERR_INVALID_ARG;  // cannot happen for chunks <= 64 (at most 24,576 words per block)

@@ -83,6 +83,37 @@ def test_corruption_is_reported():
         assert df11.read_status(status) != 0, name
 
 
+def test_inconsistent_offsets_and_states_stay_in_bounds():
+    # offsets far past the word array or going backwards, and states of 0
+    # (every step then takes a word): the copies are clamped to the array and
+    # the buffer, the word address is checked every 16 steps against the
+    # buffer's slack, and the launch reports the block as corrupt
+    torch = torch_cuda()
+    w = inputs.gaussian(20 * 4096 + 77, [106])
+    fmt = df11.rans_build_format(w)
+
+    def far(t):
+        t.view(torch.int32)[3] = 0x7FFFFFF0
+
+    def backwards(t):
+        t.view(torch.int32)[4] = 0
+
+    def zero_states(t):
+        t.view(torch.int32)[64:96] = 0
+        t.view(torch.int32)[-32:] = 0  # the partial last block too
+
+    for name, edit in (("block_word", far), ("block_word", backwards), ("states", zero_states)):
+        dev = df11.RansDeviceFormat(fmt, "cuda")
+        edit(dev.tensors[name])
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = df11.rans_decompress(dev, None, status)
+        torch.cuda.synchronize()
+        assert df11.read_status(status) != 0, name
+        # blocks that were not touched still decode
+        got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got[:2 * 4096], w[:2 * 4096])
+
+
 def test_repeated_launches_are_identical():
     torch = torch_cuda()
     w = inputs.gaussian(1 << 20, [105])
