@@ -22,11 +22,11 @@
 // prep kernel packs every 64-column chunk of X into the shared-memory image
 // the tensor core reads and finds each unit's first and last format block.
 // Then one persistent CTA per SM takes units blockIdx.x, + gridDim.x, ...:
-//   * DW decode warps (20 when at least 3 ring stages fit beside them, which
-//     holds up to batch 64; else 16): warp w decodes the unit's format blocks
-//     w, w + DW, ... with the per-block decode shared with the other kernels,
-//     merges each
-//     exponent with its sign/mantissa byte and stores the BF16 weight at its
+//   * DW decode warps (27, the most a 1024-thread CTA seats beside the
+//     control and epilogue warps, when at least 3 ring stages fit beside
+//     them; else 20; else 16): warp w decodes the unit's format blocks w,
+//     w + DW, ... with the per-block decode shared with the other kernels,
+//     merges each exponent with its sign/mantissa byte and stores the BF16 weight at its
 //     place in a ring of S operand tiles in shared memory (K-major, 128-byte
 //     swizzle).  A warp arrives on a tile's "full" barrier as soon as none
 //     of its remaining blocks reaches into that tile: on the tiles before a
@@ -63,9 +63,9 @@ constexpr uint32_t kTileElems = kTileRows * kTileCols;  // 8192
 constexpr uint32_t kTileShift = 13;
 constexpr uint32_t kTileBytes = kTileElems * 2;          // 16 KB
 // DW decode warps, then the control warp (warp DW), then 4 epilogue warps.
-// 20 decode warps when at least kMinStages20 ring stages fit beside them,
-// else 16 (more warps hide more of the decode loop's latency; a ring of 2
-// stalls the decode warps more often).
+// 27 or 20 decode warps when at least kMinStages20 ring stages fit beside
+// them, else 16 (more warps hide more of the decode loop's latency; a ring
+// of 2 stalls the decode warps more often).
 __host__ __device__ constexpr uint32_t gemm_threads(uint32_t dw) { return (dw + 1 + 4) * 32; }
 constexpr uint32_t kMinStages20 = 3;
 constexpr uint32_t kMaxStages = 8;
@@ -625,7 +625,7 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
 struct GemmFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][2][2] = {};  // [C - 1][16 or 20 decode warps][short slots]
+    uint32_t granted[2][3][2] = {};  // [C - 1][16, 20 or 27 decode warps][short slots]
 };
 std::mutex g_gemm_mu;
 GemmFacts g_gemm[64];
@@ -724,9 +724,10 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
             f->sms = sms;
         }
     }
-    // as many ring stages as fit; 20 decode warps if that leaves at least
-    // kMinStages20 stages, else 16 decode warps and at least 2 stages; short
-    // staging slots when the stream states that no code is 1 bit long
+    // as many ring stages as fit; the most decode warps (27, else 20) that
+    // leave at least kMinStages20 stages, else 16 decode warps and at least
+    // 2 stages; short staging slots when the stream states that no code is
+    // 1 bit long
     const uint32_t optin = (uint32_t)f->smem_optin;
     const uint32_t slot = prm.min_code_len >= 2 ? kSlotShort : kSlotLong;
     auto max_stages = [&](uint32_t dw) {
@@ -735,7 +736,11 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
             st--;
         return st;
     };
-    uint32_t dw = 20, stages = max_stages(20);
+    uint32_t dw = 27, stages = max_stages(27);
+    if (stages < kMinStages20) {
+        dw = 20;
+        stages = max_stages(20);
+    }
     if (stages < kMinStages20) {
         dw = 16;
         stages = max_stages(16);
@@ -744,11 +749,17 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
         return DF11_ERR_INVALID_ARG;
     prm.stages = stages;
     const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages, dw, slot);
-    const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 20 ? 1 : 0, si = slot == kSlotShort ? 1 : 0;
-    auto kern = ci == 0 ? (wi ? (si ? df11_gemm_kernel<1, 20, kSlotShort> : df11_gemm_kernel<1, 20, kSlotLong>)
-                              : (si ? df11_gemm_kernel<1, 16, kSlotShort> : df11_gemm_kernel<1, 16, kSlotLong>))
-                        : (wi ? (si ? df11_gemm_kernel<2, 20, kSlotShort> : df11_gemm_kernel<2, 20, kSlotLong>)
-                              : (si ? df11_gemm_kernel<2, 16, kSlotShort> : df11_gemm_kernel<2, 16, kSlotLong>));
+    const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 27 ? 2 : (dw == 20 ? 1 : 0),
+              si = slot == kSlotShort ? 1 : 0;
+    using Kernel = void (*)(const GemmParams);
+    static const Kernel kernels[2][3][2] = {
+        {{df11_gemm_kernel<1, 16, kSlotLong>, df11_gemm_kernel<1, 16, kSlotShort>},
+         {df11_gemm_kernel<1, 20, kSlotLong>, df11_gemm_kernel<1, 20, kSlotShort>},
+         {df11_gemm_kernel<1, 27, kSlotLong>, df11_gemm_kernel<1, 27, kSlotShort>}},
+        {{df11_gemm_kernel<2, 16, kSlotLong>, df11_gemm_kernel<2, 16, kSlotShort>},
+         {df11_gemm_kernel<2, 20, kSlotLong>, df11_gemm_kernel<2, 20, kSlotShort>},
+         {df11_gemm_kernel<2, 27, kSlotLong>, df11_gemm_kernel<2, 27, kSlotShort>}}};
+    const Kernel kern = kernels[ci][wi][si];
     {
         std::lock_guard<std::mutex> lock(g_gemm_mu);
         if (smem > f->granted[ci][wi][si]) {
