@@ -117,9 +117,18 @@ __device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(
 
 // Sums v over each run of lanes that hold the same key (a run's key is not
 // used by any other lane) and adds the sum to *y from the run's first lane
-// (y may be null: nothing to add).
+// (y may be null: nothing to add).  When every lane holds the same key, a
+// plain butterfly sum and one atomic add.
 __device__ __forceinline__ void add_runs(float v, uint32_t key, float *y, int lane)
 {
+    if (__all_sync(0xffffffffu, key == __shfl_sync(0xffffffffu, key, 0))) {
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1)
+            v += __shfl_xor_sync(0xffffffffu, v, d);
+        if (lane == 0 && y)
+            atomicAdd(y, v);
+        return;
+    }
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const float o = __shfl_down_sync(0xffffffffu, v, d);
@@ -130,6 +139,24 @@ __device__ __forceinline__ void add_runs(float v, uint32_t key, float *y, int la
     const uint32_t before = __shfl_up_sync(0xffffffffu, key, 1);
     if ((lane == 0 || before != key) && y)
         atomicAdd(y, v);
+}
+
+// v += the dot product of 8 BF16 pairs (w[j], x[j]) held two per word, by
+// the mixed-precision FMA (BF16 operands, fp32 addend and result; the BF16
+// product is exact in fp32, so each step rounds once, as an fp32 FMA of the
+// widened operands does).
+__device__ __forceinline__ float dot16_bf16(float v, const uint32_t w[8], const uint32_t x[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+        asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+            "mov.b32 {wl, wh}, %1;\n\t"
+            "mov.b32 {xl, xh}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+            "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
+            : "+f"(v)
+            : "r"(w[j]), "r"(x[j]));
+    return v;
 }
 
 // Fused use of one decoded block (MODE 1): y += W x for the block's outputs
@@ -171,11 +198,7 @@ __device__ __forceinline__ void gemv_block(const Params &p, uint64_t g0, uint32_
             const uint4 *xp = reinterpret_cast<const uint4 *>(M.x + col);
             const uint4 xa = __ldg(xp), xb = __ldg(xp + 1);
             const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                v = fmaf(bf16_lo(w[j]), bf16_lo(xw[j]), v);
-                v = fmaf(bf16_hi(w[j]), bf16_hi(xw[j]), v);
-            }
+            v = dot16_bf16(v, w, xw);
             key = 2 * (M.rowbase + row);
             y = M.y + row;
             // next chunk of this lane: 512 elements on

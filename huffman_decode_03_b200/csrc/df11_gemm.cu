@@ -72,7 +72,9 @@ constexpr uint32_t kMaxStages = 8;
 constexpr uint32_t kUnitChunks = 16;  // K chunks per work unit, at most
 constexpr uint32_t kMaxGemmMats = 16;
 constexpr uint32_t kCoverSlots = 16;  // > kMaxStages + 2 units in flight
-constexpr uint32_t kSpinLimit = 1u << 20;
+constexpr uint32_t kSpinLimit = 1u << 22;         // polls of one wait, at most
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // and 1 s of waiting
+constexpr uint32_t kSuspendNs = 20000;            // a poll sleeps up to 20 us unless the phase completes
 constexpr uint32_t kTimeoutFlag = 0x80000000u;
 
 // Barrier and flag area after the decode warps' buffers: full[8], empty[8],
@@ -187,18 +189,49 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete is suspended in
+// hardware until it completes or kSuspendNs pass: a waiting warp takes no
+// issue slots from the decode warps while it waits.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Waits until the barrier's phase of the given parity has completed.  Gives
-// up (false) when the kernel is aborting, or after kSpinLimit polls, which
-// starts the abort.  With honour_abort false it keeps waiting during an abort
-// (used to drain the kernel's own copies and MMAs).
+// up (false) when the kernel is aborting (checked every 8 polls), or after
+// kWaitLimitNs or kSpinLimit polls, which starts the abort.  With
+// honour_abort false it keeps waiting during an abort (used to drain the
+// kernel's own copies and MMAs).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
                                           uint32_t *status, bool honour_abort = true)
 {
-    for (uint32_t i = 0; i < kSpinLimit; i++) {
-        if (mbar_try(bar, parity))
+    if (mbar_try(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1; i < kSpinLimit; i++) {
+        if (mbar_try_sleep(bar, parity))
             return true;
-        if (honour_abort && *abort_flag)
-            return false;
+        if ((i & 7u) == 0) {
+            if (honour_abort && *abort_flag)
+                return false;
+            if (global_ns() - t0 > kWaitLimitNs)
+                break;
+        }
     }
     *abort_flag = 1u;
     atomicOr(status, kTimeoutFlag);
