@@ -63,15 +63,13 @@ constexpr uint32_t kTileElems = kTileRows * kTileCols;  // 8192
 constexpr uint32_t kTileShift = 13;
 constexpr uint32_t kTileBytes = kTileElems * 2;          // 16 KB
 // DW decode warps, then the control warp (warp DW), then 4 epilogue warps.
-// 27 or 20 decode warps when at least kMinStages20 ring stages fit beside
-// them, else 16 (more warps hide more of the decode loop's latency; a ring
-// of 2 stalls the decode warps more often).
+// 27, 20 or 16 decode warps, the most that leave room for enough exponent
+// tiles (more warps hide more of the decode loop's latency).
 __host__ __device__ constexpr uint32_t gemm_threads(uint32_t dw) { return (dw + 1 + 4) * 32; }
-constexpr uint32_t kMinStages20 = 3;
-constexpr uint32_t kMaxStages = 8;
+constexpr uint32_t kStages = 2;     // operand tiles in the ring (the MMA is short)
+constexpr uint32_t kMaxETiles = 16;  // exponent tiles, at most
 constexpr uint32_t kUnitChunks = 16;  // K chunks per work unit, at most
 constexpr uint32_t kMaxGemmMats = 16;
-constexpr uint32_t kCoverSlots = 16;  // > kMaxStages + 2 units in flight
 constexpr uint32_t kSpinLimit = 1u << 22;         // polls of one wait, at most
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // and 1 s of waiting
 constexpr uint32_t kSuspendNs = 20000;            // a poll sleeps up to 20 us unless the phase completes
@@ -79,11 +77,15 @@ constexpr uint32_t kTimeoutFlag = 0x80000000u;
 
 // Barrier and flag area after the decode warps' buffers: full[8], empty[8],
 // xfull[8], accf[2], tfree[2], drain (8 bytes each), then the tensor-memory
-// address, the abort flag and the coverage counters.
+// address, the abort flag, the count of MMAs known complete, and per
+// exponent tile its element count and its count of merges (both over all
+// its uses).  Counters, not barriers, for the waits of the decode warps: a
+// warp may run two or more uses ahead of a tile, and an mbarrier's phase
+// parity cannot tell those uses apart.
 constexpr uint32_t kBarFull = 0, kBarEmpty = 8, kBarX = 16, kBarAcc = 24, kBarFree = 26, kBarDrain = 28;
 constexpr uint32_t kNumBars = 29;
-constexpr uint32_t kCtrlBytes = 512;
-static_assert(kNumBars * 8 + 8 + 4 * kCoverSlots <= kCtrlBytes, "control area");
+constexpr uint32_t kCtrlBytes = 1024;
+static_assert(kNumBars * 8 + 12 + 8 * kMaxETiles <= kCtrlBytes, "control area");
 
 struct GemmMat {
     uint32_t off;           // first stream element
@@ -115,6 +117,7 @@ struct GemmParams {
     // the product
     uint32_t batch;      // N of the MMA
     uint32_t stages;     // S, operand tiles in the ring
+    uint32_t etiles;     // E, exponent tiles
     uint32_t tmem_cols;  // power of two >= 2 * batch
     uint32_t num_mats;
     uint32_t num_units;
@@ -130,11 +133,12 @@ __host__ __device__ constexpr uint32_t ctrl_offset(uint32_t cap, uint32_t dw, ui
 }
 
 // Dynamic shared memory of a launch: tables, decode buffers, control area,
-// 1 KB to align the ring, the ring.
-__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages, uint32_t dw,
-                                                      uint32_t slot)
+// 1 KB to align the ring, the operand ring (weight and activation tiles),
+// the exponent tiles.
+__host__ __device__ constexpr uint32_t gemm_smem_bytes(uint32_t cap, uint32_t batch, uint32_t stages, uint32_t etiles,
+                                                      uint32_t dw, uint32_t slot)
 {
-    return ctrl_offset(cap, dw, slot) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128);
+    return ctrl_offset(cap, dw, slot) + kCtrlBytes + 1024 + stages * (kTileBytes + batch * 128) + etiles * kTileElems;
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: BF16 A and B, both
@@ -353,20 +357,96 @@ __global__ void gemm_prep_kernel(const GemmParams p)
 }
 
 struct Roles {
-    uint32_t ring_a, ring_b, bars;  // shared addresses
+    uint32_t ring_a, ring_b, ring_e, bars;  // shared addresses
     volatile uint32_t *abort_flag;
-    uint32_t *cover;
+    volatile uint32_t *mma_done;  // the MMAs of tiles 0 .. mma_done - 1 have completed
+    uint32_t *ecount;             // per exponent tile: elements received, over all its uses
+    volatile uint32_t *emerged;   // per exponent tile: uses merged
     uint32_t tmem;
 };
 
+// Waits until *c >= target (a counter that only grows).  Gives up like
+// mbar_wait: when the kernel is aborting, or after kWaitLimitNs or
+// kSpinLimit polls, which starts the abort.
+__device__ __forceinline__ bool count_wait(const volatile uint32_t *c, uint32_t target, const Roles &R,
+                                           uint32_t *status)
+{
+    if (*c >= target)
+        return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1; i < kSpinLimit; i++) {
+        __nanosleep(200);
+        if (*c >= target)
+            return true;
+        if ((i & 7u) == 0) {
+            if (*R.abort_flag)
+                return false;
+            if (global_ns() - t0 > kWaitLimitNs)
+                break;
+        }
+    }
+    *R.abort_flag = 1u;
+    atomicOr(status, kTimeoutFlag);
+    return false;
+}
+
 __device__ __forceinline__ uint32_t bar(const Roles &R, uint32_t i) { return R.bars + 8 * i; }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// One quarter (2048 elements) of tile q (stream elements tile0 ..), whose
+// 8192 exponents are all in its exponent tile: merged with their
+// sign/mantissa bytes (from L2) into operand slot q mod S, at the swizzled
+// positions the tensor core reads.  The caller has waited until the slot is
+// free.  One warp.
+__device__ __forceinline__ void merge_quarter(const GemmParams &p, const Roles &R, uint32_t q, uint64_t tile0,
+                                              uint32_t quarter, int lane)
+{
+    const uint32_t ea = R.ring_e + (q % p.etiles) * kTileElems, sa = R.ring_a + (q % p.stages) * kTileBytes;
+    const uint8_t *smt = p.sm + tile0;
+    uint4 s4[4];
+#pragma unroll
+    for (uint32_t j = 0; j < 4; j++)
+        s4[j] = __ldg(reinterpret_cast<const uint4 *>(smt + 2048u * quarter + 512u * j + 16u * (uint32_t)lane));
+#pragma unroll
+    for (uint32_t j = 0; j < 4; j++) {
+        const uint32_t l = 2048u * quarter + 512u * j + 16u * (uint32_t)lane;
+        const uint4 e4 = ld_shared_v4(ea + l);
+        uint4 r0, r1;
+        merge4(s4[j].x, e4.x, r0.x, r0.y);
+        merge4(s4[j].y, e4.y, r0.z, r0.w);
+        merge4(s4[j].z, e4.z, r1.x, r1.y);
+        merge4(s4[j].w, e4.w, r1.z, r1.w);
+        const uint32_t a0 = sa + tile_offset(l);
+        st_shared_v4(a0, r0);
+        st_shared_v4(a0 ^ 16u, r1);  // the next 8 columns: group index + 1, XOR row
+    }
+}
+
 // Decode warp: every unit of the CTA, blocks warp, warp + DW, ... of it.
+// Each block is decoded into the warp's own buffer; its exponents are then
+// copied to their places in the exponent tiles of the tiles it covers (once
+// those are free: tile q - E merged), and the tiles' element counters are
+// advanced.  A decode warp waits only for exponent tiles, and the decode
+// itself never waits.
 template <int C, int DW, uint32_t SLOT>
 __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R, uint8_t *smem, uint32_t warp,
                                             int lane)
 {
-    const uint32_t S = p.stages;
+    const uint32_t E = p.etiles;
     uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap, SLOT);
     const uint8_t *luts = smem + Smem::luts;
     const uint8_t *cl = smem + Smem::cl;
@@ -376,103 +456,76 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
     const uint32_t slot_base =
         static_cast<uint32_t>(__cvta_generic_to_shared(exp_s + p.cap)) + (uint32_t)lane * SLOT;
 
-    uint32_t q0 = 0, k = 0;  // tile sequence number of the unit's first tile; unit count
-    // waits until tile q's ring slot is free (the MMA of tile q - S is done)
-    auto slot_free = [&](uint32_t q) -> bool {
-        if (q < S)
+    uint32_t q0 = 0;  // tile sequence number of the unit's first tile
+    // waits until exponent tile q may be written (the four quarters of tile
+    // q - E have been merged)
+    auto etile_free = [&](uint32_t q) -> bool {
+        if (q < E)
             return true;
-        return __all_sync(0xffffffffu, mbar_wait(bar(R, kBarEmpty + q % S), (q / S - 1) & 1u, R.abort_flag, p.status));
+        const bool ok = __all_sync(0xffffffffu, count_wait(R.emerged + q % E, 4 * (q / E), R, p.status));
+        __threadfence_block();
+        return ok;
     };
-    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
+    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         if (*R.abort_flag)
             return;
         const Unit U = unit_of(p, u);
         const uint64_t e0 = U.e0, e1 = e0 + (uint64_t)U.ntiles * kTileElems;
         const uint32_t bb = p.unit_blocks[2 * u], be = p.unit_blocks[2 * u + 1];
-        uint32_t arrived = 0;
-        bool ok = true;
-        // tile of the unit holding stream element x (0 before it, ntiles past it)
-        auto tile_of = [&](uint64_t x) -> uint32_t {
-            return x >= e1 ? U.ntiles : (x <= e0 ? 0u : (uint32_t)((x - e0) >> kTileShift));
-        };
-        // arrives on tiles [arrived, t_end): this warp writes nothing more there
-        auto arrive_upto = [&](uint32_t t_end) -> bool {
-            for (; arrived < t_end; arrived++) {
-                if (!slot_free(q0 + arrived))
-                    return false;
-                if (lane == 0)
-                    mbar_arrive(bar(R, kBarFull + (q0 + arrived) % S));
-            }
-            return true;
-        };
         BlockRegs<C> cur, nxt;
         uint32_t b = bb + warp;
         if (b < be)
             load_block<C>(p, b, lane, cur);
-        for (; b < be && ok; b += DW) {
-            const bool more = b + DW < be;
-            if (more)
+        for (; b < be; b += DW) {
+            if (b + DW < be)
                 load_block<C>(p, b + DW, lane, nxt);
-            // Before waiting for any ring slot: arrive on the tiles before
-            // this block.  The MMA of a tile needs every warp's arrival, and
-            // a slot frees only when the MMA of the tile S earlier is done.
-            ok = arrive_upto(tile_of(cur.o0));
-            if (!ok)
-                break;
+            // the block's share of the unit, by its offsets: [r0, r1)
+            const uint64_t o0 = cur.o0, o1 = cur.o1 > cur.o0 ? cur.o1 : cur.o0;
+            const uint64_t r0 = o0 > e0 ? o0 : e0, r1 = o1 < e1 ? o1 : e1;
             BlockOut bo;
-            if (decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
-                // the block's outputs inside the unit: [lo, hi) relative to g0
-                const uint64_t g0 = bo.g0;
-                const uint32_t lo = (uint32_t)(g0 + bo.lo_off < e0 ? e0 - g0 : bo.lo_off);
-                const uint32_t hi = (uint32_t)(g0 + bo.hi > e1 ? e1 - g0 : bo.hi);
-                if (lo < hi) {
-                    const uint32_t t_first = (uint32_t)((g0 + lo - e0) >> kTileShift);
-                    const uint32_t t_last = (uint32_t)((g0 + hi - 1 - e0) >> kTileShift);
-                    for (uint32_t t = t_first; t <= t_last && ok; t++)
-                        ok = slot_free(q0 + t);
-                    if (!ok)
-                        break;
-                    const uint32_t sa0 = R.ring_a + ((q0 + t_first) % S) * kTileBytes;
-                    const uint32_t sa1 = R.ring_a + ((q0 + t_first + 1) % S) * kTileBytes;
-                    const uint8_t *smg = p.sm + g0;
-                    auto addr = [&](uint32_t l) {
+            const bool dok = decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo);
+            if (r0 < r1) {
+                const uint32_t t_first = (uint32_t)((r0 - e0) >> kTileShift);
+                const uint32_t t_last = (uint32_t)((r1 - 1 - e0) >> kTileShift);
+                for (uint32_t t = t_first; t <= t_last; t++)
+                    if (!etile_free(q0 + t))
+                        return;
+                if (dok) {
+                    // exponents [lo, hi) of the block (relative to g0) to their exponent tiles
+                    const uint64_t g0 = bo.g0;
+                    const uint32_t lo = (uint32_t)(r0 - g0), hi = (uint32_t)(r1 - g0);
+                    const uint32_t ea0 = R.ring_e + ((q0 + t_first) % E) * kTileElems;
+                    const uint32_t ea1 = R.ring_e + ((q0 + t_first + 1) % E) * kTileElems;
+                    auto eaddr = [&](uint32_t l) {
                         const uint32_t v = (uint32_t)(g0 + l - e0);
-                        return ((v >> kTileShift) == t_first ? sa0 : sa1) + tile_offset(v & (kTileElems - 1));
+                        return ((v >> kTileShift) == t_first ? ea0 : ea1) + (v & (kTileElems - 1));
                     };
-                    // whole groups of 16 (two 16-byte pieces of one tile row:
-                    // a group never crosses a row of 64 or a tile) ...
+                    // whole groups of 16 (a group never crosses a tile) ...
                     const uint32_t c_lo = (lo + 15u) & ~15u, c_hi = hi & ~15u;
-                    for (uint32_t l0 = c_lo + 16u * lane; l0 < c_hi; l0 += 512u) {
-                        const uint4 s4 = __ldg(reinterpret_cast<const uint4 *>(smg + l0));
-                        const uint4 e4 = *reinterpret_cast<const uint4 *>(exp_s + l0);
-                        uint4 r0, r1;
-                        merge4(s4.x, e4.x, r0.x, r0.y);
-                        merge4(s4.y, e4.y, r0.z, r0.w);
-                        merge4(s4.z, e4.z, r1.x, r1.y);
-                        merge4(s4.w, e4.w, r1.z, r1.w);
-                        const uint32_t a0 = addr(l0);
-                        st_shared_v4(a0, r0);
-                        st_shared_v4(a0 ^ 16u, r1);  // the next 8 columns: group index + 1, XOR row
-                    }
-                    // ... and up to 15 single elements at each end
+                    for (uint32_t l0 = c_lo + 16u * lane; l0 < c_hi; l0 += 512u)
+                        st_shared_v4(eaddr(l0), *reinterpret_cast<const uint4 *>(exp_s + l0));
+                    // ... and up to 15 single bytes at each end
                     const uint32_t head_end = c_lo < hi ? c_lo : hi, tail0 = c_hi > c_lo ? c_hi : c_lo;
                     const uint32_t l = lane < 16 ? lo + lane : tail0 + (lane - 16);
                     if (lane < 16 ? l < head_end : l < hi)
-                        st_shared_u16(addr(l), merge1(__ldg(smg + l), exp_s[l]));
-                    fence_proxy_async();  // the tiles are read by the tensor core (async proxy)
-                    __syncwarp();
-                    // counted before this warp arrives on any of these tiles
-                    if (lane == 0)
-                        atomicAdd(R.cover + k % kCoverSlots, hi - lo);
+                        st_shared_u8(eaddr(l), exp_s[l]);
+                }
+                // counted after every lane's copies (a corrupt block still
+                // counts its elements, so no tile waits for ever)
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence_block();
+                    for (uint32_t t = t_first; t <= t_last; t++) {
+                        const uint64_t a = e0 + ((uint64_t)t << kTileShift), z = a + kTileElems;
+                        const uint32_t cnt = (uint32_t)((r1 < z ? r1 : z) - (r0 > a ? r0 : a));
+                        const uint32_t q = q0 + t, full = (q / E + 1) * kTileElems;
+                        if (atomicAdd(R.ecount + q % E, cnt) + cnt > full)
+                            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+                    }
                 }
             }
-            // and, right away, on the tiles before the next block
-            ok = arrive_upto(more ? tile_of(nxt.o0) : U.ntiles);
             cur = nxt;
         }
-        ok = ok && arrive_upto(U.ntiles);
-        if (!ok)
-            return;
         q0 += U.ntiles;
     }
 }
@@ -482,10 +535,6 @@ __device__ __forceinline__ void control_role(const GemmParams &p, const Roles &R
 {
     const uint32_t S = p.stages, N = p.batch, xbytes = N * 128;
     const uint32_t idesc = idesc_bf16(kTileRows, N);
-    uint32_t expect[kCoverSlots];
-#pragma unroll
-    for (uint32_t i = 0; i < kCoverSlots; i++)
-        expect[i] = 0;
     uint32_t q0 = 0, k = 0, x_issued = 0, x_used = 0, committed = 0;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, k++) {
@@ -523,17 +572,17 @@ __device__ __forceinline__ void control_role(const GemmParams &p, const Roles &R
                 umma_bf16(R.tmem + d * N, ad + 2 * kk, bd + 2 * kk, idesc, (t | kk) != 0);
             umma_commit(bar(R, kBarEmpty + s));
             committed = 1;
+            // the MMA's completion, published at once: the decode warp that
+            // merges tile q + S waits for it
+            ok = mbar_wait(bar(R, kBarEmpty + s), (q / S) & 1u, R.abort_flag, p.status);
+            if (!ok)
+                break;
+            *R.mma_done = q + 1;
             if (t + S - 1 < U.ntiles)
                 ok = issue_x(t + S - 1);
         }
         if (!ok)
             break;
-        // every tile of the unit is full: the decode warps' element counts
-        // are final and must add up to the unit's elements
-        const uint32_t c = k % kCoverSlots;
-        expect[c] += U.ntiles * kTileElems;
-        if (*reinterpret_cast<volatile uint32_t *>(R.cover + c) != expect[c])
-            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         umma_commit(bar(R, kBarAcc + d));
         q0 += U.ntiles;
     }
@@ -546,16 +595,21 @@ __device__ __forceinline__ void control_role(const GemmParams &p, const Roles &R
     }
 }
 
-// Epilogue warp: adds each unit's accumulator rows 32 q .. 32 q + 31 (q =
-// warp mod 4, the tensor-memory lanes this warp may read) into Y.
-__device__ __forceinline__ void epilogue_role(const GemmParams &p, const Roles &R, uint32_t warp, int lane)
+// Merge and epilogue warp (four of them, warp mod 4 = quarter).  In tile
+// order: wait until the tile's exponents are all in (its counter), and its
+// operand slot free (the MMA of tile q - S complete, as the control thread
+// publishes), merge this warp's quarter, arrive on the tile's full barrier
+// and count the quarter merged (the exponent tile is free after all four).
+// After a unit's tiles, the epilogue of the unit before: add the rows 32
+// quarter .. 32 quarter + 31 of its accumulator (the tensor-memory lanes
+// this warp may read) into Y; the last unit's epilogue at the end.
+__device__ __forceinline__ void merge_epilogue_role(const GemmParams &p, const Roles &R, uint32_t warp, int lane)
 {
-    const uint32_t quarter = warp & 3u, N = p.batch;
-    uint32_t k = 0;
-    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
+    const uint32_t quarter = warp & 3u, N = p.batch, S = p.stages, E = p.etiles;
+    auto epilogue = [&](uint32_t u, uint32_t k) -> bool {
         const uint32_t d = k & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(bar(R, kBarAcc + d), (k >> 1) & 1u, R.abort_flag, p.status)))
-            return;
+            return false;
         tc_fence_after();
         const Unit U = unit_of(p, u);
         const GemmMat &M = p.mats[U.m];
@@ -572,7 +626,33 @@ __device__ __forceinline__ void epilogue_role(const GemmParams &p, const Roles &
         __syncwarp();
         if (lane == 0)
             mbar_arrive(bar(R, kBarFree + d));
+        return true;
+    };
+    uint32_t q0 = 0, k = 0;
+    for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
+        const Unit U = unit_of(p, u);
+        for (uint32_t t = 0; t < U.ntiles; t++) {
+            const uint32_t q = q0 + t;
+            if (!__all_sync(0xffffffffu, count_wait(R.ecount + q % E, (q / E + 1) * kTileElems, R, p.status)))
+                return;
+            if (q >= S && !__all_sync(0xffffffffu, count_wait(R.mma_done, q - S + 1, R, p.status)))
+                return;
+            __threadfence_block();
+            merge_quarter(p, R, q, U.e0 + ((uint64_t)t << kTileShift), quarter, lane);
+            fence_proxy_async();  // the operand tile is read by the tensor core (async proxy)
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(R, kBarFull + q % S));
+                __threadfence_block();
+                atomicAdd(const_cast<uint32_t *>(R.emerged + q % E), 1u);
+            }
+        }
+        q0 += U.ntiles;
+        if (k >= 1 && !epilogue(u - gridDim.x, k - 1))
+            return;
     }
+    if (k >= 1)
+        epilogue(blockIdx.x + (k - 1) * gridDim.x, k - 1);
 }
 
 template <int C, int DW, uint32_t SLOT>
@@ -588,13 +668,16 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     R.bars = static_cast<uint32_t>(__cvta_generic_to_shared(ctrl));
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + kNumBars * 8);
     R.abort_flag = tmem_slot + 1;
-    R.cover = tmem_slot + 2;
+    R.mma_done = tmem_slot + 2;
+    R.ecount = tmem_slot + 3;
+    R.emerged = tmem_slot + 3 + kMaxETiles;
     R.ring_a = (base + ctrl_offset(p.cap, DW, SLOT) + kCtrlBytes + 1023u) & ~1023u;
     R.ring_b = R.ring_a + S * kTileBytes;
+    R.ring_e = R.ring_b + S * p.batch * 128;
 
     if (tid == 0) {
         for (uint32_t s = 0; s < S; s++) {
-            mbar_init(bar(R, kBarFull + s), DW);
+            mbar_init(bar(R, kBarFull + s), 4);  // the four merge warps
             mbar_init(bar(R, kBarEmpty + s), 1);
             mbar_init(bar(R, kBarX + s), 1);
         }
@@ -603,9 +686,12 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
             mbar_init(bar(R, kBarFree + d), 4);
         }
         mbar_init(bar(R, kBarDrain), 1);
+        for (uint32_t i = 0; i < kMaxETiles; i++) {
+            R.ecount[i] = 0u;
+            R.emerged[i] = 0u;
+        }
+        *R.mma_done = 0u;
         *R.abort_flag = 0u;
-        for (uint32_t i = 0; i < kCoverSlots; i++)
-            R.cover[i] = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async();
     }
@@ -642,7 +728,7 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
             control_role(p, R);
         __syncwarp();
     } else {
-        epilogue_role(p, R, warp, lane);
+        merge_epilogue_role(p, R, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -757,31 +843,32 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
             f->sms = sms;
         }
     }
-    // as many ring stages as fit; the most decode warps (27, else 20) that
-    // leave at least kMinStages20 stages, else 16 decode warps and at least
-    // 2 stages; short staging slots when the stream states that no code is
-    // 1 bit long
+    // two operand stages; as many exponent tiles as fit (up to 16) beside
+    // the most decode warps that leave at least 4 of them (27 warps), else 3
+    // (20 warps), else 2 (16 warps; a block covers at most two tiles); short
+    // staging slots when the stream states that no code is 1 bit long
     const uint32_t optin = (uint32_t)f->smem_optin;
     const uint32_t slot = prm.min_code_len >= 2 ? kSlotShort : kSlotLong;
-    auto max_stages = [&](uint32_t dw) {
-        uint32_t st = kMaxStages;
-        while (st >= 1 && gemm_smem_bytes(prm.cap, batch, st, dw, slot) > optin)
-            st--;
-        return st;
+    auto max_etiles = [&](uint32_t dw) {
+        uint32_t e = kMaxETiles;
+        while (e >= 1 && gemm_smem_bytes(prm.cap, batch, kStages, e, dw, slot) > optin)
+            e--;
+        return e;
     };
-    uint32_t dw = 27, stages = max_stages(27);
-    if (stages < kMinStages20) {
+    uint32_t dw = 27, etiles = max_etiles(27);
+    if (etiles < 4) {
         dw = 20;
-        stages = max_stages(20);
+        etiles = max_etiles(20);
     }
-    if (stages < kMinStages20) {
+    if (etiles < 3) {
         dw = 16;
-        stages = max_stages(16);
+        etiles = max_etiles(16);
     }
-    if (stages < 2)
+    if (etiles < 2)
         return DF11_ERR_INVALID_ARG;
-    prm.stages = stages;
-    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, stages, dw, slot);
+    prm.stages = kStages;
+    prm.etiles = etiles;
+    const uint32_t smem = gemm_smem_bytes(prm.cap, batch, kStages, etiles, dw, slot);
     const int ci = a->threads_per_block == 32 ? 0 : 1, wi = dw == 27 ? 2 : (dw == 20 ? 1 : 0),
               si = slot == kSlotShort ? 1 : 0;
     using Kernel = void (*)(const GemmParams);
