@@ -407,20 +407,25 @@ __device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v)
     asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-// One quarter (2048 elements) of tile q (stream elements tile0 ..), whose
-// 8192 exponents are all in its exponent tile: merged with their
-// sign/mantissa bytes (from L2) into operand slot q mod S, at the swizzled
-// positions the tensor core reads.  The caller has waited until the slot is
-// free.  One warp.
-__device__ __forceinline__ void merge_quarter(const GemmParams &p, const Roles &R, uint32_t q, uint64_t tile0,
-                                              uint32_t quarter, int lane)
+// The sign/mantissa bytes of this lane in one quarter (2048 elements) of
+// the tile whose first stream element is tile0 (four 16-byte loads, from L2).
+__device__ __forceinline__ void load_quarter(const GemmParams &p, uint64_t tile0, uint32_t quarter, int lane,
+                                             uint4 (&s4)[4])
 {
-    const uint32_t ea = R.ring_e + (q % p.etiles) * kTileElems, sa = R.ring_a + (q % p.stages) * kTileBytes;
-    const uint8_t *smt = p.sm + tile0;
-    uint4 s4[4];
+    const uint8_t *smt = p.sm + tile0 + 2048u * quarter + 16u * (uint32_t)lane;
 #pragma unroll
     for (uint32_t j = 0; j < 4; j++)
-        s4[j] = __ldg(reinterpret_cast<const uint4 *>(smt + 2048u * quarter + 512u * j + 16u * (uint32_t)lane));
+        s4[j] = __ldg(reinterpret_cast<const uint4 *>(smt + 512u * j));
+}
+
+// One quarter of tile q, whose 8192 exponents are all in its exponent tile:
+// merged with the sign/mantissa bytes s4 (load_quarter) into operand slot
+// q mod S, at the swizzled positions the tensor core reads.  The caller has
+// waited until the slot is free.  One warp.
+__device__ __forceinline__ void merge_quarter(const GemmParams &p, const Roles &R, uint32_t q, uint32_t quarter,
+                                              int lane, const uint4 (&s4)[4])
+{
+    const uint32_t ea = R.ring_e + (q % p.etiles) * kTileElems, sa = R.ring_a + (q % p.stages) * kTileBytes;
 #pragma unroll
     for (uint32_t j = 0; j < 4; j++) {
         const uint32_t l = 2048u * quarter + 512u * j + 16u * (uint32_t)lane;
@@ -629,8 +634,10 @@ __device__ __forceinline__ void merge_epilogue_role(const GemmParams &p, const R
         return true;
     };
     uint32_t q0 = 0, k = 0;
+    uint4 s4[4];  // the next tile's sign/mantissa bytes, loaded before its exponents are all in
     for (uint32_t u = blockIdx.x; u < p.num_units; u += gridDim.x, k++) {
         const Unit U = unit_of(p, u);
+        load_quarter(p, U.e0, quarter, lane, s4);
         for (uint32_t t = 0; t < U.ntiles; t++) {
             const uint32_t q = q0 + t;
             if (!__all_sync(0xffffffffu, count_wait(R.ecount + q % E, (q / E + 1) * kTileElems, R, p.status)))
@@ -638,7 +645,9 @@ __device__ __forceinline__ void merge_epilogue_role(const GemmParams &p, const R
             if (q >= S && !__all_sync(0xffffffffu, count_wait(R.mma_done, q - S + 1, R, p.status)))
                 return;
             __threadfence_block();
-            merge_quarter(p, R, q, U.e0 + ((uint64_t)t << kTileShift), quarter, lane);
+            merge_quarter(p, R, q, quarter, lane, s4);
+            if (t + 1 < U.ntiles)
+                load_quarter(p, U.e0 + ((uint64_t)(t + 1) << kTileShift), quarter, lane, s4);
             fence_proxy_async();  // the operand tile is read by the tensor core (async proxy)
             __syncwarp();
             if (lane == 0) {
