@@ -375,7 +375,7 @@ __device__ __forceinline__ bool count_wait(const volatile uint32_t *c, uint32_t 
         return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1; i < kSpinLimit; i++) {
-        __nanosleep(200);
+        __nanosleep(1000);
         if (*c >= target)
             return true;
         if ((i & 7u) == 0) {

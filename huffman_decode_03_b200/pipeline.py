@@ -104,6 +104,28 @@ def block_gemms(shapes, x):
     return consume
 
 
+def _timed(fn, reps, inner):
+    """Median over `reps` samples of the device time of one call of `fn`;
+    each sample times `inner` calls back to back between two CUDA events, so
+    that host-side launch gaps between calls (small kernels the host cannot
+    feed fast enough) do not count as device time."""
+    import numpy as np
+    import torch
+
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        e0.record()
+        for _ in range(inner):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / inner)
+    return float(np.median(ts))
+
+
 def _bench(args):
     import numpy as np
     import torch
@@ -129,17 +151,7 @@ def _bench(args):
         sink.append(gemm(w))
 
     def timed(fn, reps):
-        fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for _ in range(reps):
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return float(np.median(ts))
+        return _timed(fn, reps, args.inner)
 
     out = torch.empty_like(pipe.bufs[0])
     st = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -213,17 +225,7 @@ def _bench_gemv(args):
             decompress_gemv(f, shapes, xs, ys, st)
 
     def timed(fn, reps):
-        fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for _ in range(reps):
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return float(np.median(ts))
+        return _timed(fn, reps, args.inner)
 
     nb = args.blocks
     res = {"blocks": nb, "batch": 1, "block": "llama3_8b (q,k,v,o,gate,up,down)",
@@ -287,17 +289,7 @@ def _bench_gemm(args):
             decompress_gemm(f, shapes, xs, ys, st, scratch=scratch)
 
     def timed(fn, reps):
-        fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for _ in range(reps):
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return float(np.median(ts))
+        return _timed(fn, reps, args.inner)
 
     nb = args.blocks
     res = {"blocks": nb, "batch": B, "block": "llama3_8b (q,k,v,o,gate,up,down)",
@@ -331,6 +323,8 @@ def main(argv=None):
     ap.add_argument("--no-check", dest="check", action="store_false")
     ap.add_argument("--gemv", action="store_true",
                     help="batch-1 comparison: decompress + cuBLAS matrix-vector products vs df11_decompress_gemv")
+    ap.add_argument("--inner", type=int, default=4,
+                    help="calls timed back to back per sample (their mean is the sample)")
     ap.add_argument("--gemm", action="store_true",
                     help="batch-B comparison: decompress + cuBLAS GEMMs vs df11_decompress_gemm")
     args = ap.parse_args(argv)
