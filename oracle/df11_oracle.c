@@ -565,12 +565,14 @@ int64_t df11o_decode_range(const uint8_t *stream, uint64_t stream_bits,
  *              owns elements b B + 512 j + 16 l + i (j = 0..J-1, i = 0..15),
  *              decoded in the order (j, i); all lanes step together, step
  *              t = 16 j + i; a lane whose element lies at or past n skips the
- *              step.  After each step the lanes that renormalise read one word
- *              each, in lane order, from the block's word sequence.  The
- *              encoder runs the same steps backwards (t descending, lanes
- *              descending), starting every lane at x = L; its final states are
- *              the decoder's start states, and its words, reversed, the block's
- *              word sequence.
+ *              step.  Each lane has its own word stream: a renormalising lane
+ *              reads the next word of it.  A block's words are lane 0's
+ *              stream, then lane 1's, ..., lane 31's; lane_words[32 b + l]
+ *              counts lane l's words (at most one per step: 16 J <= 240
+ *              words, so J <= 15).  The encoder runs the same steps backwards
+ *              (t descending), starting every lane at x = L; its final states
+ *              are the decoder's start states, and each lane's words,
+ *              reversed, that lane's stream.
  * ======================================================================== */
 
 /* Frequencies: f[s] = max(1, floor(h[s] M / n)) for every symbol present,
@@ -623,15 +625,19 @@ static uint64_t oracle_rans_pos(uint64_t b, int J, int l, int t)
     return b * (uint64_t)(512 * J) + 512u * (uint64_t)(t / 16) + 16u * (uint64_t)l + (uint64_t)(t % 16);
 }
 
-/* rANS encode of n exponents, blocks of 512 J elements.  words receives the
- * 16-bit words of block 0, then block 1, ...; offsets[b] (nblocks + 1
- * entries) the index of block b's first word; states[32 b + l] the start
- * state of lane l of block b.  Returns the number of words, or -1 (capacity,
- * a symbol with frequency 0, or a state outside [L, 2^32)). */
+/* rANS encode of n exponents, blocks of 512 J elements (J <= 15).  words
+ * receives the words of block 0 (lane 0's stream, then lane 1's, ...), then
+ * block 1, ...; offsets[b] (nblocks + 1 entries) the index of block b's
+ * first word; lane_words[32 b + l] the length of lane l's stream in block b;
+ * states[32 b + l] the start state of lane l of block b.  Returns the number
+ * of words, or -1 (J out of range, capacity, a symbol with frequency 0, or a
+ * state outside [L, 2^32)). */
 int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq, int prob_bits, int J,
-                          uint16_t *words, uint64_t cap, uint32_t *states, uint64_t *offsets)
+                          uint16_t *words, uint64_t cap, uint32_t *states, uint64_t *offsets, uint8_t *lane_words)
 {
     const uint64_t L = 1ull << 16, M = 1ull << prob_bits;
+    if (J < 1 || J > 15)
+        return -1;
     const uint64_t B = 512ull * (uint64_t)J;
     const uint64_t nblocks = (n + B - 1) / B;
     uint64_t cum[ORACLE_NSYM];
@@ -642,17 +648,20 @@ int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq,
     }
     if (c != M)
         return -1;
-    uint16_t *stack = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(B ? B : 1));
+    /* one stack per lane: at most one word per step */
+    uint16_t *stack = (uint16_t *)malloc(sizeof(uint16_t) * 32 * 16 * (size_t)J);
     if (!stack)
         return -1;
     uint64_t total = 0;
     for (uint64_t b = 0; b < nblocks; b++) {
         uint64_t x[32];
-        for (int l = 0; l < 32; l++)
+        int depth[32];
+        for (int l = 0; l < 32; l++) {
             x[l] = L;
-        uint64_t depth = 0;
+            depth[l] = 0;
+        }
         for (int t = 16 * J - 1; t >= 0; t--) {
-            for (int l = 31; l >= 0; l--) {
+            for (int l = 0; l < 32; l++) {
                 const uint64_t pos = oracle_rans_pos(b, J, l, t);
                 if (pos >= n)
                     continue;
@@ -663,7 +672,7 @@ int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq,
                     return -1;
                 }
                 if (x[l] >= (1ull << (32 - prob_bits)) * f) {
-                    stack[depth++] = (uint16_t)(x[l] & 0xFFFFu);
+                    stack[16 * J * l + depth[l]++] = (uint16_t)(x[l] & 0xFFFFu);
                     x[l] >>= 16;
                 }
                 x[l] = (x[l] / f) * M + (x[l] % f) + cum[s];
@@ -674,15 +683,17 @@ int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq,
             }
         }
         offsets[b] = total;
-        if (total + depth > cap) {
-            free(stack);
-            return -1;
-        }
-        for (uint64_t k = 0; k < depth; k++)
-            words[total + k] = stack[depth - 1 - k];
-        total += depth;
-        for (int l = 0; l < 32; l++)
+        for (int l = 0; l < 32; l++) {
+            if (total + (uint64_t)depth[l] > cap) {
+                free(stack);
+                return -1;
+            }
+            for (int k = 0; k < depth[l]; k++)
+                words[total + k] = stack[16 * J * l + depth[l] - 1 - k];
+            total += (uint64_t)depth[l];
+            lane_words[32 * b + l] = (uint8_t)depth[l];
             states[32 * b + l] = (uint32_t)x[l];
+        }
     }
     offsets[nblocks] = total;
     free(stack);
@@ -690,13 +701,17 @@ int64_t df11o_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freq,
 }
 
 /* rANS decode back to BF16 bits (exponent from the words, sign and mantissa
- * from sm).  Returns 0, or -1 when the words, states or offsets are
- * inconsistent (a block reads past its words, does not use all of them, or
- * does not end every lane at x = L). */
+ * from sm).  Returns 0, or -1 when the words, states, offsets or lane counts
+ * are inconsistent (the lane counts do not add up to the block's words, a
+ * lane reads past its stream or does not use all of it, or does not end at
+ * x = L). */
 int df11o_rans_decode(const uint16_t *words, const uint32_t *states, const uint64_t *offsets,
-                      const uint32_t *freq, int prob_bits, int J, uint64_t n, const uint8_t *sm, uint16_t *out)
+                      const uint8_t *lane_words, const uint32_t *freq, int prob_bits, int J, uint64_t n,
+                      const uint8_t *sm, uint16_t *out)
 {
     const uint64_t L = 1ull << 16, M = 1ull << prob_bits;
+    if (J < 1 || J > 15)
+        return -1;
     const uint64_t B = 512ull * (uint64_t)J;
     const uint64_t nblocks = (n + B - 1) / B;
     uint64_t cum[ORACLE_NSYM];
@@ -708,10 +723,16 @@ int df11o_rans_decode(const uint16_t *words, const uint32_t *states, const uint6
     if (c != M)
         return -1;
     for (uint64_t b = 0; b < nblocks; b++) {
-        uint64_t x[32];
-        for (int l = 0; l < 32; l++)
+        uint64_t x[32], ptr[32], end[32];
+        uint64_t start = offsets[b];
+        for (int l = 0; l < 32; l++) {
             x[l] = states[32 * b + l];
-        uint64_t ptr = offsets[b];
+            ptr[l] = start;
+            end[l] = start + lane_words[32 * b + l];
+            start = end[l];
+        }
+        if (start != offsets[b + 1])
+            return -1;
         for (int t = 0; t < 16 * J; t++) {
             for (int l = 0; l < 32; l++) {
                 const uint64_t pos = oracle_rans_pos(b, J, l, t);
@@ -728,16 +749,14 @@ int df11o_rans_decode(const uint16_t *words, const uint32_t *states, const uint6
                 const unsigned sign = (sm[pos] >> 7) & 1u, mantissa = sm[pos] & 0x7Fu;
                 out[pos] = (uint16_t)((sign << 15) | ((unsigned)s << 7) | mantissa);
                 if (x[l] < L) {
-                    if (ptr >= offsets[b + 1])
+                    if (ptr[l] >= end[l])
                         return -1;
-                    x[l] = (x[l] << 16) | words[ptr++];
+                    x[l] = (x[l] << 16) | words[ptr[l]++];
                 }
             }
         }
-        if (ptr != offsets[b + 1])
-            return -1;
         for (int l = 0; l < 32; l++)
-            if (x[l] != L)
+            if (ptr[l] != end[l] || x[l] != L)
                 return -1;
     }
     return 0;

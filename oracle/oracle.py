@@ -14,8 +14,9 @@ BlockOffset) and the hierarchical LUTs.
 ``rans_build_format`` / ``rans_decode_format`` are the rANS variant of the
 exponent coder that the page's discussion proposes (range asymmetric numeral
 systems from their published definition: quantised frequencies, one 32-bit
-state per lane, 16-bit words, blocks of 512 J elements decoded by 32 lanes in
-step); sign and mantissa stay verbatim as in DF11.  Pinned in
+state per lane, 16-bit words, each lane its own word stream, blocks of 512 J
+elements decoded by 32 lanes in step); sign and mantissa stay verbatim as in
+DF11.  Pinned in
 ``tests/test_rans_oracle.py``.
 """
 from __future__ import annotations
@@ -87,9 +88,9 @@ def _load():
         lib.df11o_split_all.restype = None
         lib.df11o_rans_freqs.argtypes = [P, ctypes.c_int, P]
         lib.df11o_rans_freqs.restype = ctypes.c_int
-        lib.df11o_rans_encode.argtypes = [P, U64, P, ctypes.c_int, ctypes.c_int, P, U64, P, P]
+        lib.df11o_rans_encode.argtypes = [P, U64, P, ctypes.c_int, ctypes.c_int, P, U64, P, P, P]
         lib.df11o_rans_encode.restype = ctypes.c_int64
-        lib.df11o_rans_decode.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, U64, P, P]
+        lib.df11o_rans_decode.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int, U64, P, P]
         lib.df11o_rans_decode.restype = ctypes.c_int
         lib.df11o_rans_step_encode.argtypes = [U64, ctypes.c_int, P, ctypes.c_int, P, P]
         lib.df11o_rans_step_encode.restype = U64
@@ -292,7 +293,9 @@ def rans_freqs(hist, prob_bits: int = RANS_PROB_BITS) -> np.ndarray:
 
 
 def rans_encode(exps, freq, prob_bits: int = RANS_PROB_BITS, chunks: int = RANS_CHUNKS):
-    """-> (words uint16, states uint32 [nblocks, 32], offsets uint64 [nblocks + 1])"""
+    """-> (words uint16, states uint32 [nblocks, 32], offsets uint64 [nblocks + 1],
+    lane_words uint8 [nblocks, 32]); words of a block: lane 0's stream, then
+    lane 1's, ..."""
     exps = np.ascontiguousarray(exps, dtype=np.uint8)
     freq = np.ascontiguousarray(freq, dtype=np.uint32)
     n = exps.size
@@ -301,15 +304,17 @@ def rans_encode(exps, freq, prob_bits: int = RANS_PROB_BITS, chunks: int = RANS_
     words = np.zeros(max(n, 1), np.uint16)
     states = np.zeros(max(32 * nblocks, 1), np.uint32)
     offsets = np.zeros(nblocks + 1, np.uint64)
+    lane_words = np.zeros(max(32 * nblocks, 1), np.uint8)
     src = exps if n else np.zeros(1, np.uint8)
     got = _load().df11o_rans_encode(_ptr(src), n, _ptr(freq), prob_bits, chunks, _ptr(words), words.size,
-                                    _ptr(states), _ptr(offsets))
+                                    _ptr(states), _ptr(offsets), _ptr(lane_words))
     if got < 0:
         raise ValueError("rANS encode failed")
-    return words[:got].copy(), states[: 32 * nblocks].reshape(nblocks, 32).copy(), offsets
+    return (words[:got].copy(), states[: 32 * nblocks].reshape(nblocks, 32).copy(), offsets,
+            lane_words[: 32 * nblocks].reshape(nblocks, 32).copy())
 
 
-def rans_decode(words, states, offsets, freq, sm, n: int, prob_bits: int = RANS_PROB_BITS,
+def rans_decode(words, states, offsets, lane_words, freq, sm, n: int, prob_bits: int = RANS_PROB_BITS,
                 chunks: int = RANS_CHUNKS) -> np.ndarray:
     words = np.ascontiguousarray(words, dtype=np.uint16)
     if words.size == 0:
@@ -318,13 +323,16 @@ def rans_decode(words, states, offsets, freq, sm, n: int, prob_bits: int = RANS_
     if states.size == 0:
         states = np.zeros(1, np.uint32)
     offsets = np.ascontiguousarray(offsets, dtype=np.uint64)
+    lane_words = np.ascontiguousarray(lane_words, dtype=np.uint8).reshape(-1)
+    if lane_words.size == 0:
+        lane_words = np.zeros(1, np.uint8)
     freq = np.ascontiguousarray(freq, dtype=np.uint32)
     sm = np.ascontiguousarray(sm, dtype=np.uint8)
     if sm.size == 0:
         sm = np.zeros(1, np.uint8)
     out = np.empty(max(n, 1), np.uint16)
-    rc = _load().df11o_rans_decode(_ptr(words), _ptr(states), _ptr(offsets), _ptr(freq), prob_bits, chunks, n,
-                                   _ptr(sm), _ptr(out))
+    rc = _load().df11o_rans_decode(_ptr(words), _ptr(states), _ptr(offsets), _ptr(lane_words), _ptr(freq),
+                                   prob_bits, chunks, n, _ptr(sm), _ptr(out))
     if rc != 0:
         raise ValueError("rANS data inconsistent")
     return out[:n]
@@ -355,14 +363,15 @@ def rans_build_format(w: np.ndarray, prob_bits: int = RANS_PROB_BITS, chunks: in
     exps, sm = split_all(w)
     hist = histogram(exps)
     freq = rans_freqs(hist, prob_bits) if exps.size else np.zeros(256, np.uint32)
-    words, states, offsets = rans_encode(exps, freq, prob_bits, chunks) if exps.size else (
-        np.zeros(0, np.uint16), np.zeros((0, 32), np.uint32), np.zeros(1, np.uint64))
+    words, states, offsets, lane_words = rans_encode(exps, freq, prob_bits, chunks) if exps.size else (
+        np.zeros(0, np.uint16), np.zeros((0, 32), np.uint32), np.zeros(1, np.uint64), np.zeros((0, 32), np.uint8))
     return {"n": int(exps.size), "hist": hist, "freq": freq, "words": words, "states": states,
-            "offsets": offsets, "packed_sign_mantissa": sm, "prob_bits": prob_bits, "chunks": chunks}
+            "offsets": offsets, "lane_words": lane_words, "packed_sign_mantissa": sm, "prob_bits": prob_bits,
+            "chunks": chunks}
 
 
 def rans_decode_format(fmt: dict) -> np.ndarray:
     if fmt["n"] == 0:
         return np.zeros(0, np.uint16)
-    return rans_decode(fmt["words"], fmt["states"], fmt["offsets"], fmt["freq"], fmt["packed_sign_mantissa"],
-                       fmt["n"], fmt["prob_bits"], fmt["chunks"])
+    return rans_decode(fmt["words"], fmt["states"], fmt["offsets"], fmt["lane_words"], fmt["freq"],
+                       fmt["packed_sign_mantissa"], fmt["n"], fmt["prob_bits"], fmt["chunks"])

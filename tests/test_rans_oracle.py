@@ -95,9 +95,12 @@ def test_round_trips(oracle_mod):
     cases.append(allp)
     cases.append(np.full(10_000, 0x3C00, np.uint16))  # one exponent only
     for w in cases:
-        for chunks in (1, 8):
+        for chunks in (1, 8, 15):
             fmt = oracle_mod.rans_build_format(w, 12, chunks)
             assert np.array_equal(oracle_mod.rans_decode_format(fmt), w)
+    # a lane reads at most one word per step and counts them in a byte: 16 J <= 240
+    with pytest.raises(ValueError):
+        oracle_mod.rans_build_format(inputs.gaussian(100, [77]), 12, 16)
 
 
 def test_single_symbol_costs_nothing(oracle_mod):
@@ -109,18 +112,19 @@ def test_single_symbol_costs_nothing(oracle_mod):
 def test_two_equal_symbols_cost_one_bit_each(oracle_mod):
     # f = M/2 for both: every encode step adds exactly one bit to the state,
     # so a lane that codes k symbols from x = 2^16 emits floor(k / 16) words
-    # and ends with a state of 17 + k mod 16 bits
+    # (its stream's length) and ends with a state of 17 + k mod 16 bits
     rng = np.random.default_rng(2)
     for n in (4096, 4096 * 2 + 700, 123):
         exps = rng.integers(0, 2, n).astype(np.uint8)
         freq = np.zeros(256, np.uint32)
         freq[:2] = 2048
-        words, states, offsets = oracle_mod.rans_encode(exps, freq, 12, 8)
+        words, states, offsets, lane_words = oracle_mod.rans_encode(exps, freq, 12, 8)
         for b in range(states.shape[0]):
             for lane in range(32):
                 pos = b * 4096 + np.arange(8)[:, None] * 512 + 16 * lane + np.arange(16)[None, :]
                 k = int((pos < n).sum())
                 assert states[b, lane].item().bit_length() == 17 + k % 16
+                assert int(lane_words[b, lane]) == k // 16
         per_lane = [int(((b * 4096 + np.arange(8)[:, None] * 512 + 16 * l + np.arange(16)[None, :]) < n).sum())
                     for b in range(states.shape[0]) for l in range(32)]
         assert words.size == sum(k // 16 for k in per_lane)
@@ -147,9 +151,52 @@ def test_size_is_the_information_content_of_the_model(oracle_mod):
         assert content <= entropy + 0.02 * n
 
 
+def test_each_lane_stream_decodes_alone(oracle_mod):
+    # every lane's stream, decoded on its own by the decoding rule (written
+    # here independently of the oracle), gives back that lane's exponents in
+    # the layout's order and ends at x = L with the stream used up
+    w = inputs.stress(3 * 4096 + 1000, key=(78, 0))
+    fmt = oracle_mod.rans_build_format(w, 12, 8)
+    exps = ((w >> 7) & 0xFF).astype(np.int64)
+    freq = fmt["freq"].astype(np.int64)
+    cum = np.concatenate([[0], np.cumsum(freq)])
+    n = w.size
+    for b in range(fmt["states"].shape[0]):
+        start = int(fmt["offsets"][b])
+        for lane in range(32):
+            cnt = int(fmt["lane_words"][b, lane])
+            stream = fmt["words"][start: start + cnt]
+            start += cnt
+            x, k = int(fmt["states"][b, lane]), 0
+            for t in range(16 * 8):
+                pos = b * 4096 + 512 * (t // 16) + 16 * lane + t % 16
+                if pos >= n:
+                    continue
+                slot = x % 4096
+                s = int(np.searchsorted(cum, slot, side="right") - 1)
+                assert s == exps[pos]
+                x = int(freq[s]) * (x // 4096) + slot - int(cum[s])
+                if x < L:
+                    x = (x << 16) | int(stream[k])
+                    k += 1
+            assert x == L and k == cnt
+        assert start == int(fmt["offsets"][b + 1])
+
+
 def test_inconsistent_data_is_rejected(oracle_mod):
     w = inputs.gaussian(10_000, [90])
     fmt = oracle_mod.rans_build_format(w)
+    moved = dict(fmt)  # one word moved from lane 3's stream to lane 4's
+    moved["lane_words"] = fmt["lane_words"].copy()
+    moved["lane_words"][0, 3] -= 1
+    moved["lane_words"][0, 4] += 1
+    with pytest.raises(ValueError):
+        oracle_mod.rans_decode_format(moved)
+    uncounted = dict(fmt)  # lane counts that do not add up to the block's words
+    uncounted["lane_words"] = fmt["lane_words"].copy()
+    uncounted["lane_words"][1, 0] += 1
+    with pytest.raises(ValueError):
+        oracle_mod.rans_decode_format(uncounted)
     short = dict(fmt)
     short["words"] = fmt["words"][:-1]
     short["offsets"] = fmt["offsets"].copy()
