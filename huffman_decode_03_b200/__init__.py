@@ -90,6 +90,7 @@ class df11_rans_arrays(ctypes.Structure):
         ("words", ctypes.c_void_p),
         ("states", ctypes.c_void_p),
         ("block_word", ctypes.c_void_p),
+        ("lane_words", ctypes.c_void_p),
         ("freq", ctypes.c_void_p),
         ("packed_sign_mantissa", ctypes.c_void_p),
         ("packed_sign_mantissa_bytes", ctypes.c_uint64),
@@ -588,6 +589,7 @@ class RansFormat:
             "words": self._view(a.words, a.num_words + 8 if a.n else 0, np.uint16),
             "states": self._view(a.states, 32 * a.num_blocks, np.uint32),
             "block_word": self._view(a.block_word, a.num_blocks + 1 if a.n else 0, np.uint32),
+            "lane_words": self._view(a.lane_words, 32 * a.num_blocks, np.uint8),
             "freq": self._view(a.freq, 256 if a.n else 0, np.uint16),
             "packed_sign_mantissa": self._view(a.packed_sign_mantissa, a.packed_sign_mantissa_bytes, np.uint8),
         }
@@ -598,10 +600,11 @@ class RansFormat:
                                                  "max_block_words")}
 
     def compressed_bytes(self) -> int:
-        """Bytes of the stream: words, start states, block offsets, the model
-        and the sign/mantissa bytes (without padding)."""
+        """Bytes of the stream: words, start states, lane counts, block
+        offsets, the model and the sign/mantissa bytes (without padding)."""
         s = self.scalars()
-        return 2 * s["num_words"] + 4 * 32 * s["num_blocks"] + 4 * (s["num_blocks"] + 1) + 2 * 256 + s["n"]
+        return (2 * s["num_words"] + (4 + 1) * 32 * s["num_blocks"] + 4 * (s["num_blocks"] + 1) + 2 * 256
+                + s["n"])
 
 
 def rans_build_format(mats, chunks: int = 8) -> RansFormat:
@@ -638,6 +641,7 @@ class RansDeviceFormat:
         a.words = ts["words"].data_ptr()
         a.states = ts["states"].data_ptr()
         a.block_word = ts["block_word"].data_ptr()
+        a.lane_words = ts["lane_words"].data_ptr()
         a.freq = ts["freq"].data_ptr()
         a.packed_sign_mantissa = ts["packed_sign_mantissa"].data_ptr()
         a.packed_sign_mantissa_bytes = ts["packed_sign_mantissa"].numel()

@@ -113,7 +113,6 @@ __device__ __forceinline__ uint32_t gemv_matrix(const Params &p, uint32_t g)
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(two & 0xFFFF0000u); }
 
 // Sums v over each run of lanes that hold the same key (a run's key is not
 // used by any other lane) and adds the sum to *y from the run's first lane

@@ -12,20 +12,21 @@
 //
 // Per step and lane: one lookup in a 4096-entry table (the slot's exponent,
 // rotated right by one bit for the merge, slot - cum and freq - 1), one
-// multiply-add for the new state, and, when the state falls below 2^16, one
-// 16-bit word: the lanes that need one take consecutive words of the block
-// in lane order (ballot, popcount of the lanes below).  A block's words are
-// read from shared memory: each warp has two buffers, and the next block's
-// words are copied into the other one (cp.async) and its sign/mantissa bytes
-// prefetched into L2 while the current block decodes.  The warps per CTA are
-// as many as the buffers fit (32 for blocks of up to about 1,140 words).
-// Every lane must end the block at x = 2^16 and the block must use exactly
-// its words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped to the
-// padded array and to the buffer.  Full blocks check the word address once
-// per 16 steps (a chunk reads at most 512 words, and each buffer has 512
-// words of slack past the copied ones); the partial last block clamps every
-// read.  So inconsistent data never reads out of bounds; nothing traps and
-// every loop has a fixed trip count.
+// multiply-add for the new state, and, when the state falls below 2^16, the
+// next 16-bit word of the lane's own stream (a predicated load and a pointer
+// increment: the lanes do not coordinate).  A block's streams follow one
+// another; each lane finds its start from the 32 lane counts by one warp
+// scan per block.  A block's words are read from shared memory: each warp
+// has two buffers, and the next block's words are copied into the other one
+// (cp.async) and its sign/mantissa bytes prefetched into L2 while the
+// current block decodes.  The warps per CTA are as many as the buffers fit
+// (32 for blocks of up to about 1,140 words).  Every lane must end the block
+// at x = 2^16 with its stream used up, and the lane counts must add up to
+// the block's words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped
+// to the padded array and to the buffer; a lane's start is clamped to the
+// copied words, and a block reads at most 240 words per lane beyond it,
+// inside the buffer's 512 words of slack.  So inconsistent data never reads
+// out of bounds; nothing traps and every loop has a fixed trip count.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -55,6 +56,7 @@ struct RansParams {
     uint32_t cap;        // words a block may copy into its buffer (multiple of 8, >= max block words + 14)
     uint32_t bufw;       // words of one buffer: cap plus 512 words of slack for one chunk's reads
     uint32_t words_end;  // copies end at or below this word: num_words rounded down to 8, plus the 8 padding words
+    const uint8_t *lane_words;
 };
 
 __device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
@@ -74,41 +76,31 @@ __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
     return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
 }
 
-__device__ __forceinline__ uint32_t lanemask_lt()
-{
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
-// One decode step of one lane (all lanes call it together).  valid: the
-// lane's element exists; acc receives the exponent byte at byte position Q.
+// One decode step of one lane.  valid: the lane's element exists; acc
+// receives the exponent byte at byte position Q; wp: the shared address of
+// the lane's next word.
 template <int Q>
-__device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &base, bool valid, const uint32_t *table,
-                                     const uint16_t *wb, const RansParams &p, uint32_t lt)
+__device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &wp, bool valid, const uint32_t *table)
 {
     if (valid) {
         const uint32_t e = table[x & (kSlots - 1)];
         const uint32_t xh = x >> kProbBits;
         x = (e >> 20) * xh + xh + ((e >> 8) & 0xFFFu);
         acc = __byte_perm(acc, e, (0x3210 & ~(0xF << (4 * Q))) | (4 << (4 * Q)));
+        if (x < kLow) {
+            uint32_t w;
+            asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(wp) : "memory");
+            x = (x << 16) | w;
+            wp += 2u;
+        }
     }
-    const bool need = valid && x < kLow;
-    const uint32_t m = __ballot_sync(0xffffffffu, need);
-    if (need) {
-        uint32_t i = base + __popc(m & lt);  // relative to the buffer's first word
-        i = i < p.cap ? i : p.cap - 1;
-        x = (x << 16) | wb[i];
-    }
-    base += __popc(m);
 }
 
 // 16 steps of the last, partial block: elements past n are skipped.
-__device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, uint64_t pos0, const uint32_t *table,
-                                                  const uint16_t *wb, const RansParams &p, uint32_t lt,
-                                                  uint32_t acc[4])
+__device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &wp, uint64_t pos0, const uint32_t *table,
+                                                  const RansParams &p, uint32_t acc[4])
 {
-#define DF11_STEP(I) step<(I) & 3>(x, acc[(I) >> 2], base, pos0 + (I) < p.n, table, wb, p, lt)
+#define DF11_STEP(I) step<(I) & 3>(x, acc[(I) >> 2], wp, pos0 + (I) < p.n, table)
     DF11_STEP(0); DF11_STEP(1); DF11_STEP(2); DF11_STEP(3);
     DF11_STEP(4); DF11_STEP(5); DF11_STEP(6); DF11_STEP(7);
     DF11_STEP(8); DF11_STEP(9); DF11_STEP(10); DF11_STEP(11);
@@ -117,11 +109,11 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, u
 }
 
 // One step of a full block in PTX, the same arithmetic as step() with the
-// word read predicated instead of branched around.  Operands: %0 the state,
-// %1 the shared address of the warp's next word, A the accumulator that
-// takes the exponent byte at the position SEL selects, %6 the table's
-// shared address, %7 the lanes-below mask.  No clamp: a chunk reads at most
-// 512 words past %1, and the buffer's slack holds them.
+// word read predicated.  Operands: %0 the state, %1 the shared address of
+// the lane's next word, A the accumulator that takes the exponent byte at
+// the position SEL selects, %6 the table's shared address.  No clamp: a lane
+// starts at most cap words into its buffer and reads at most one word per
+// step, 240 per block, and the buffer has 512 words of slack.
 #define DF11_RSTEP(A, SEL)                       \
     "and.b32 ts, %0, 4095;\n\t"                  \
     "shl.b32 ts, ts, 2;\n\t"                     \
@@ -134,25 +126,20 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &base, u
     "add.u32 %0, %0, to;\n\t"                    \
     "prmt.b32 " A ", " A ", te, " SEL ";\n\t"    \
     "setp.lt.u32 tp, %0, 65536;\n\t"             \
-    "vote.sync.ballot.b32 tm, tp, 0xffffffff;\n\t" \
-    "and.b32 tt, tm, %7;\n\t"                    \
-    "popc.b32 tt, tt;\n\t"                       \
-    "mad.lo.u32 ta, tt, 2, %1;\n\t"              \
-    "@tp ld.shared.u16 tw, [ta];\n\t"            \
+    "@tp ld.shared.u16 tw, [%1];\n\t"            \
     "@tp prmt.b32 %0, tw, %0, 0x5410;\n\t"       \
-    "popc.b32 tt, tm;\n\t"                       \
-    "mad.lo.u32 %1, tt, 2, %1;\n\t"
+    "@tp add.u32 %1, %1, 2;\n\t"
 #define DF11_RSTEP4(A) \
     DF11_RSTEP(A, "0x3214") DF11_RSTEP(A, "0x3240") DF11_RSTEP(A, "0x3410") DF11_RSTEP(A, "0x4210")
 
-// 16 steps of a full block (all lanes valid, warp converged).
-__device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wa, uint32_t tbl, uint32_t lt, uint32_t acc[4])
+// 16 steps of a full block (all lanes valid).
+__device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wp, uint32_t tbl, uint32_t acc[4])
 {
-    asm volatile("{\n\t.reg .b32 ts, te, th, tf, to, tt, ta, tw, tm;\n\t.reg .pred tp;\n\t"
+    asm volatile("{\n\t.reg .b32 ts, te, th, tf, to, tw;\n\t.reg .pred tp;\n\t"
                  DF11_RSTEP4("%2") DF11_RSTEP4("%3") DF11_RSTEP4("%4") DF11_RSTEP4("%5")
                  "}"
-                 : "+r"(x), "+r"(wa), "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
-                 : "r"(tbl), "r"(lt)
+                 : "+r"(x), "+r"(wp), "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
+                 : "r"(tbl)
                  : "memory");
 }
 #undef DF11_RSTEP4
@@ -237,19 +224,20 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         return;
     }
 
-    const uint32_t lt = lanemask_lt();
     const uint64_t B = 512ull * p.chunks;
     const uint32_t warps = blockDim.x >> 5, stride = gridDim.x * warps;
     uint16_t *wbuf = wbufs + 2u * p.bufw * warp;
     const uint32_t wbuf_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
     const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(table));
     uint32_t b = blockIdx.x * warps + warp, k = 0;
-    // software pipeline: the next block's state and word offsets, and the
-    // next chunk's sign/mantissa bytes, are loaded one step ahead
-    uint32_t x_n = 0, bw0_n = 0, bw1_n = 0, wfirst = 0;
+    // software pipeline: the next block's state, lane count and word
+    // offsets, and the next chunk's sign/mantissa bytes, are loaded one step
+    // ahead
+    uint32_t x_n = 0, c_n = 0, bw0_n = 0, bw1_n = 0, wfirst = 0;
     uint4 s_n = make_uint4(0u, 0u, 0u, 0u);
     if (b < p.num_blocks) {
         x_n = __ldg(p.states + 32ull * b + lane);
+        c_n = __ldg(p.lane_words + 32ull * b + lane);
         bw0_n = __ldg(p.block_word + b);
         bw1_n = __ldg(p.block_word + b + 1);
         wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s);
@@ -259,16 +247,26 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         // this block's words have landed; the next block's go to the other buffer
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncwarp();
-        const uint16_t *wb = wbuf + k * p.bufw;
         const uint32_t wb_s = wbuf_s + 2u * p.bufw * k;
-        bool bad = false;
         uint32_t x = x_n;
-        uint32_t wa = wb_s + 2u * (bw0_n - wfirst);  // bw0 - wfirst = bw0 mod 8
-        const uint32_t end = bw1_n - wfirst;
+        // the lane's stream: after the streams of the lanes below it
+        uint32_t incl = c_n;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d)
+                incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+        const uint32_t first = (bw0_n - wfirst) + (incl - c_n);  // bw0 - wfirst = bw0 mod 8
+        const uint32_t end = first + c_n;                          // words, from the buffer's start
+        bool bad = total != bw1_n - bw0_n || bw1_n - wfirst > p.cap;
+        uint32_t wp = wb_s + 2u * (first < p.cap ? first : p.cap);  // clamped: inconsistent counts
         const bool full = (b + 1) * B <= p.n;  // warp-uniform
         const uint32_t nb = b + stride;
         if (nb < p.num_blocks) {
             x_n = __ldg(p.states + 32ull * nb + lane);
+            c_n = __ldg(p.lane_words + 32ull * nb + lane);
             bw0_n = __ldg(p.block_word + nb);
             bw1_n = __ldg(p.block_word + nb + 1);
             wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.bufw * (k ^ 1u));
@@ -283,17 +281,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
             const uint4 s4 = s_n;
             s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512 : (uint64_t)nb * B + 16u * (uint32_t)lane);
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
-            if (wa > wb_s + 2u * p.cap) {  // past the copied words: inconsistent data
-                wa = wb_s;
-                bad = true;
-            }
-            if (full) {
-                decode_chunk_full(x, wa, tbl, lt, acc);
-            } else {
-                uint32_t base = (wa - wb_s) >> 1;
-                decode_chunk_tail(x, base, pos0, table, wb, p, lt, acc);
-                wa = wb_s + 2u * base;
-            }
+            if (full)
+                decode_chunk_full(x, wp, tbl, acc);
+            else
+                decode_chunk_tail(x, wp, pos0, table, p, acc);
             // merge with the 16 sign/mantissa bytes and store
             if (pos0 + 16 <= p.n) {
                 uint32_t r[8];
@@ -318,7 +309,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
                         p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
             }
         }
-        bad = bad || x != kLow || wa != wb_s + 2u * end || end > p.cap;
+        bad = bad || x != kLow || wp != wb_s + 2u * end;
         if (__any_sync(0xffffffffu, bad) && lane == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         __syncwarp();  // every lane is done with this buffer before it is refilled
@@ -340,10 +331,10 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     if (a->n == 0)
         return DF11_OK;
     if (!dst || (reinterpret_cast<uintptr_t>(dst) & 15) || !a->words || (reinterpret_cast<uintptr_t>(a->words) & 15) ||
-        !a->states || !a->block_word || !a->freq ||
+        !a->states || !a->block_word || !a->lane_words || !a->freq ||
         !a->packed_sign_mantissa || (reinterpret_cast<uintptr_t>(a->packed_sign_mantissa) & 15))
         return DF11_ERR_INVALID_ARG;
-    if (a->prob_bits != kProbBits || a->chunks < 1 || a->chunks > 64 || a->n >= (1ull << 32))
+    if (a->prob_bits != kProbBits || a->chunks < 1 || a->chunks > 15 || a->n >= (1ull << 32))
         return DF11_ERR_INVALID_ARG;
     const uint64_t B = 512ull * a->chunks;
     if (a->num_blocks != (a->n + B - 1) / B || a->num_words + 8 >= (1ull << 32) ||
@@ -366,6 +357,7 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     p.words = a->words;
     p.states = a->states;
     p.block_word = a->block_word;
+    p.lane_words = a->lane_words;
     p.freq = a->freq;
     p.sm = a->packed_sign_mantissa;
     p.dst = dst;

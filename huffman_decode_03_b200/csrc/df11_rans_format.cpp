@@ -8,10 +8,11 @@
 // renormalisation words, blocks of 512 * chunks elements decoded by 32 lanes
 // in step.  Sign and mantissa stay verbatim, as in DF11 ("Format DFloat11").
 //
-// Encoding runs each block's steps backwards (step descending, lane
-// descending) from x = 2^16 in every lane; the final states are the decoder's
-// start states and the block's words, reversed, the order in which the
-// decoder takes them.  Blocks are independent and encoded in parallel.
+// Encoding runs each block's steps backwards (step descending) from x = 2^16
+// in every lane; the final states are the decoder's start states and each
+// lane's words, reversed, its stream in the order the decoder takes them.
+// A block's words are lane 0's stream, then lane 1's, ...  Blocks are
+// independent and encoded in parallel.
 #include "df11.h"
 
 #include <algorithm>
@@ -25,6 +26,7 @@ struct df11_rans_format {
     df11_rans_arrays a;
     std::vector<uint16_t> words;
     std::vector<uint32_t> states, block_word;
+    std::vector<uint8_t> lane_words;
     std::vector<uint16_t> freq;
     std::vector<uint8_t> sm;
 };
@@ -98,7 +100,7 @@ extern "C" df11_status df11_rans_build(const uint16_t *const *mats, const uint64
         return DF11_ERR_INVALID_ARG;
     if (chunks == 0)
         chunks = 8;
-    if (chunks > 64)
+    if (chunks > 15)  // a lane's words per block (at most one per step) are counted in a byte
         return DF11_ERR_INVALID_ARG;
     uint64_t n = 0;
     std::vector<uint64_t> first(num_mats + 1, 0);
@@ -146,31 +148,34 @@ extern "C" df11_status df11_rans_build(const uint16_t *const *mats, const uint64
             throw std::bad_alloc();
         std::vector<std::vector<uint16_t>> blk(nblocks);
         f->states.assign(32 * nblocks, 0);
+        f->lane_words.assign(32 * nblocks, 0);
         for_each_index(nblocks, [&](uint64_t b) {
             uint64_t x[32];
             std::fill(x, x + 32, kLow);
-            std::vector<uint16_t> &st = blk[b];
-            st.reserve(B / 4);
+            std::vector<uint16_t> lane[32];
             const uint64_t b0 = b * B;
             for (int t = (int)(16 * chunks) - 1; t >= 0; t--) {
                 const uint64_t row = b0 + 512ull * (uint64_t)(t >> 4) + (uint64_t)(t & 15);
-                for (int l = 31; l >= 0; l--) {
+                for (int l = 0; l < 32; l++) {
                     const uint64_t pos = row + 16ull * (uint64_t)l;
                     if (pos >= n)
                         continue;
                     const uint32_t s = exps[pos];
                     const uint64_t fs = f->freq[s];
                     if (x[l] >= (fs << (32 - kProbBits))) {
-                        st.push_back((uint16_t)x[l]);
+                        lane[l].push_back((uint16_t)x[l]);
                         x[l] >>= 16;
                     }
                     const uint64_t q = x[l] / fs;
                     x[l] = (q << kProbBits) + (x[l] - q * fs) + cum[s];
                 }
             }
-            std::reverse(st.begin(), st.end());
-            for (int l = 0; l < 32; l++)
+            std::vector<uint16_t> &st = blk[b];
+            for (int l = 0; l < 32; l++) {
+                st.insert(st.end(), lane[l].rbegin(), lane[l].rend());
+                f->lane_words[32 * b + l] = (uint8_t)lane[l].size();
                 f->states[32 * b + l] = (uint32_t)x[l];
+            }
         });
         f->block_word.assign(nblocks + 1, 0);
         uint64_t total = 0;
@@ -197,6 +202,7 @@ extern "C" df11_status df11_rans_build(const uint16_t *const *mats, const uint64
         a.words = f->words.data();
         a.states = f->states.data();
         a.block_word = f->block_word.data();
+        a.lane_words = f->lane_words.data();
         a.freq = f->freq.data();
         a.packed_sign_mantissa = f->sm.data();
         a.packed_sign_mantissa_bytes = f->sm.size();

@@ -421,14 +421,17 @@ df11_status df11_device_encode_static(const df11_format *plan, const uint16_t *w
  *     the exponent s whose range [cum[s], cum[s] + freq[s]) holds it, and
  *     x = freq[s] (x >> prob_bits) + slot - cum[s]; below 2^16 the state
  *     takes the next 16-bit word: x = (x << 16) | word.
- *   - blocks of 512 * chunks elements; lane l (0..31) of block b owns
- *     elements b 512 chunks + 512 j + 16 l + i (j < chunks, i < 16), decoded
- *     in the order (j, i), all lanes stepping together; after a step the
- *     lanes whose state fell below 2^16 take one word each, in lane order,
- *     from the block's words; a lane skips steps whose element lies at or
- *     past n.  Every lane ends the block at x = 2^16.
+ *   - blocks of 512 * chunks elements (chunks <= 15); lane l (0..31) of
+ *     block b owns elements b 512 chunks + 512 j + 16 l + i (j < chunks,
+ *     i < 16), decoded in the order (j, i), all lanes stepping together;
+ *     each lane has its own stream of words, and a lane whose state fell
+ *     below 2^16 after a step takes the next word of it; a lane skips steps
+ *     whose element lies at or past n.  Every lane ends the block at
+ *     x = 2^16 with its stream used up.
  *   - states[32 b + l] is lane l's start state in block b; the words of
- *     block b are words[block_word[b] .. block_word[b + 1]).
+ *     block b are words[block_word[b] .. block_word[b + 1]): lane 0's stream,
+ *     then lane 1's, ..., lane 31's, lane_words[32 b + l] words each (at most
+ *     one per step: 16 chunks <= 240).
  */
 typedef struct df11_rans_format df11_rans_format;
 
@@ -436,12 +439,13 @@ typedef struct df11_rans_arrays {
     uint64_t n;                          /* BF16 elements */
     uint64_t num_words;                  /* 16-bit words of all blocks */
     uint32_t prob_bits;                  /* 12 */
-    uint32_t chunks;                     /* 16-element chunks per lane and block, 1..64 */
+    uint32_t chunks;                     /* 16-element chunks per lane and block, 1..15 */
     uint32_t num_blocks;                 /* ceil(n / (512 chunks)) */
     uint32_t max_block_words;            /* largest block_word[b + 1] - block_word[b] */
     const uint16_t *words;               /* num_words + 8 (zero padding) */
     const uint32_t *states;              /* 32 * num_blocks */
     const uint32_t *block_word;          /* num_blocks + 1 */
+    const uint8_t *lane_words;           /* 32 * num_blocks: words of each lane's stream */
     const uint16_t *freq;                /* 256, summing to 2^prob_bits (0 when n = 0) */
     const uint8_t *packed_sign_mantissa; /* round_up(n, 16) + 16 bytes, 16-B aligned */
     uint64_t packed_sign_mantissa_bytes;
@@ -452,7 +456,7 @@ typedef struct df11_rans_arrays {
  * df11_build_format; matrices concatenated) with the rANS exponent coder.
  *   chunks: 16-element chunks per lane and block (0 = 8: 4096-element blocks).
  * On success *out owns every array (host memory); DF11_ERR_TOO_LARGE for
- * n >= 2^32, DF11_ERR_INVALID_ARG for bad pointers or chunks > 64.
+ * n >= 2^32, DF11_ERR_INVALID_ARG for bad pointers or chunks > 15.
  */
 df11_status df11_rans_build(const uint16_t *const *mats, const uint64_t *counts, int num_mats, uint32_t chunks,
                             df11_rans_format **out);
@@ -470,9 +474,11 @@ void df11_rans_free(df11_rans_format *f);
  * into dst_dev (16-byte aligned, n elements), asynchronously on `stream`.
  * One warp decodes one block; the exponents of a lane's 16 elements are
  * merged with their sign/mantissa bytes and stored with one 32-byte store.
- * Inconsistent words, states or offsets set DF11_ERR_CORRUPT in
- * *status_dev (caller-zeroed) and leave that block's outputs unspecified;
- * nothing traps.  Argument errors return DF11_ERR_INVALID_ARG synchronously.
+ * Inconsistent words, states, offsets or lane counts set DF11_ERR_CORRUPT
+ * in *status_dev (caller-zeroed) and leave that block's outputs
+ * unspecified; nothing traps or reads out of bounds.  Argument errors
+ * (including words not 16-byte aligned) return DF11_ERR_INVALID_ARG
+ * synchronously.
  */
 df11_status df11_rans_decompress(const df11_rans_arrays *dev, uint16_t *dst_dev, uint32_t *status_dev,
                                  void *stream);

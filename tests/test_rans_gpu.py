@@ -35,7 +35,7 @@ def test_round_trip_against_the_oracle(oracle_mod, n):
     assert np.array_equal(got, ref)
 
 
-@pytest.mark.parametrize("chunks", [1, 2, 16, 64])
+@pytest.mark.parametrize("chunks", [1, 2, 15])
 def test_chunks(chunks):
     w = inputs.stress(300_007, key=(101, chunks))
     assert np.array_equal(gpu_decode(w, chunks), w)
@@ -84,10 +84,11 @@ def test_corruption_is_reported():
 
 
 def test_inconsistent_offsets_and_states_stay_in_bounds():
-    # offsets far past the word array or going backwards, and states of 0
-    # (every step then takes a word): the copies are clamped to the array and
-    # the buffer, the word address is checked every 16 steps against the
-    # buffer's slack, and the launch reports the block as corrupt
+    # offsets far past the word array or going backwards, states of 0 (every
+    # step then takes a word), lane counts that do not match the streams: the
+    # copies are clamped to the array and the buffer, each lane's start to the
+    # copied words (a block reads at most 240 more words per lane, inside the
+    # buffer's slack), and the launch reports the block as corrupt
     torch = torch_cuda()
     w = inputs.gaussian(20 * 4096 + 77, [106])
     fmt = df11.rans_build_format(w)
@@ -102,7 +103,12 @@ def test_inconsistent_offsets_and_states_stay_in_bounds():
         t.view(torch.int32)[64:96] = 0
         t.view(torch.int32)[-32:] = 0  # the partial last block too
 
-    for name, edit in (("block_word", far), ("block_word", backwards), ("states", zero_states)):
+    def lane_counts_off(t):
+        t[64] = 255  # lane 0 of block 2: a stream that runs past the block's words
+        t[97] = 0  # lane 1 of block 3: a stream cut short
+
+    for name, edit in (("block_word", far), ("block_word", backwards), ("states", zero_states),
+                       ("lane_words", lane_counts_off)):
         dev = df11.RansDeviceFormat(fmt, "cuda")
         edit(dev.tensors[name])
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
