@@ -607,7 +607,7 @@ class RansFormat:
                 + s["n"])
 
 
-def rans_build_format(mats, chunks: int = 8) -> RansFormat:
+def rans_build_format(mats, chunks: int = 10) -> RansFormat:
     """Compresses BF16 bit patterns (uint16 arrays) into one stream of the
     rANS variant (df11_rans_build); matrices are concatenated in order."""
     lib = load_library()

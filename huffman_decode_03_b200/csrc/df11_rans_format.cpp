@@ -99,7 +99,7 @@ extern "C" df11_status df11_rans_build(const uint16_t *const *mats, const uint64
     if (num_mats < 0 || (num_mats > 0 && (!mats || !counts)))
         return DF11_ERR_INVALID_ARG;
     if (chunks == 0)
-        chunks = 8;
+        chunks = 10;
     if (chunks > 15)  // a lane's words per block (at most one per step) are counted in a byte
         return DF11_ERR_INVALID_ARG;
     uint64_t n = 0;

@@ -454,7 +454,7 @@ typedef struct df11_rans_arrays {
 /*
  * df11_rans_build -- host: compress num_mats BF16 matrices (as
  * df11_build_format; matrices concatenated) with the rANS exponent coder.
- *   chunks: 16-element chunks per lane and block (0 = 8: 4096-element blocks).
+ *   chunks: 16-element chunks per lane and block (0 = 10: 5120-element blocks).
  * On success *out owns every array (host memory); DF11_ERR_TOO_LARGE for
  * n >= 2^32, DF11_ERR_INVALID_ARG for bad pointers or chunks > 15.
  */

@@ -280,7 +280,7 @@ def decode_format(fmt: dict) -> np.ndarray:
 # as the SIMD-friendlier entropy coder); the C side states the model and the
 # layout.
 RANS_PROB_BITS = 12
-RANS_CHUNKS = 8  # J: chunks of 16 elements per lane and block (4096 elements per block)
+RANS_CHUNKS = 10  # J: chunks of 16 elements per lane and block (5120 elements per block)
 RANS_L = 1 << 16
 
 
