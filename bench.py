@@ -59,7 +59,7 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between timed steps")
-    ap.add_argument("--rans", default="2,3",
+    ap.add_argument("--rans", default="2,3,4",
                     help="workloads on which the rANS variant of the exponent coder is measured at N=1 and "
                          "reported in the line's rans object (comma-separated ids, or 'none')")
     ap.add_argument("--per-workload", default="4,3,1",
