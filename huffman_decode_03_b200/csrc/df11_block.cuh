@@ -47,7 +47,8 @@ struct Smem {
     static constexpr uint32_t luts = sym + kIdxEntries * 4;  // 17 * 256
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
     static constexpr uint32_t zq = cl + 256;                 // uint8[16]
-    static constexpr uint32_t bufs = zq + 16;
+    static constexpr uint32_t ctr = zq + 16;                 // uint32 block counter (decoder), 16 B
+    static constexpr uint32_t bufs = ctr + 16;
     __host__ __device__ static constexpr uint32_t per_warp(uint32_t cap, uint32_t stride)
     {
         return cap + slot_bytes(stride);

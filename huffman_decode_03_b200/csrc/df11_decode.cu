@@ -19,7 +19,9 @@
 //     two lookups in flight per thread): a block's prefix sum is five warp
 //     shuffles and its buffers are private to the warp, so warps never wait
 //     for one another -- no block-wide barrier after set-up.  One persistent
-//     CTA per SM; every warp walks its own sequence of blocks;
+//     CTA per SM takes a contiguous range of blocks, and its warps take them
+//     one at a time from a counter in shared memory, so that they finish
+//     within about one block of each other;
 //   * decode once, not twice: the page counts the codes of every segment in
 //     a first pass and decodes them again in a second.  Here every chain
 //     decodes once into a private staging slot in shared memory (slots 68
@@ -374,11 +376,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     uint8_t *slots = exp_s + p.cap;
     const uint32_t nbuf = static_cast<uint32_t>(__cvta_generic_to_shared(slots + slot_bytes(SLOT)));
 
+    // the CTA's blocks are a contiguous range; each warp takes its first one
+    // here and every next one from a counter in shared memory, so that the
+    // CTA's warps all finish within about one block of each other
+    uint32_t &next_block = *reinterpret_cast<uint32_t *>(smem + Smem::ctr);
+    const uint32_t b_end = (uint32_t)(((uint64_t)p.nblocks * (blockIdx.x + 1)) / gridDim.x);
+    uint32_t b = (uint32_t)(((uint64_t)p.nblocks * blockIdx.x) / gridDim.x) + (uint32_t)warp;
+    if (tid == 0)
+        next_block = b + kWarps;  // published by the barriers in build_tables
+    auto take_next = [&]() -> uint32_t {
+        uint32_t v = 0;
+        if (lane == 0)
+            v = atomicAdd(&next_block, 1u);
+        return __shfl_sync(0xffffffffu, v, 0);
+    };
     // with long slots the first block's registers load while the tables are built
-    const uint32_t stride = gridDim.x * kWarps;
-    uint32_t b = blockIdx.x * kWarps + warp;
     BlockRegs<C> cur, nxt;
-    if (!kCopy && b < p.nblocks)
+    if (!kCopy && b < b_end)
         load_block<C>(p, b, lane, cur);
 
     build_tables(p.luts, p.cl, p.num_luts, smem, (uint32_t)tid, (uint32_t)kThreads);
@@ -395,21 +409,22 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     }
     // with short slots the first block's metadata is copied only now: the
     // table set-up used the start of the per-warp buffers as scratch
-    if (kCopy && b < p.nblocks)
+    if (kCopy && b < b_end)
         prefetch_block<C>(p, b, lane, nbuf);
 
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * SLOT;
 
-    // ---- each warp walks its own blocks; no block-wide barrier from here on
-    for (; b < p.nblocks; b += stride) {
+    // ---- each warp decodes the blocks it takes; no block-wide barrier from here on
+    for (uint32_t nb; b < b_end; b = nb) {
+        nb = take_next();
         if (kCopy) {
             read_block<C>(nbuf, lane, cur);
-            if (b + stride < p.nblocks)
-                prefetch_block<C>(p, b + stride, lane, nbuf);
-        } else if (b + stride < p.nblocks) {
-            load_block<C>(p, b + stride, lane, nxt);
+            if (nb < b_end)
+                prefetch_block<C>(p, nb, lane, nbuf);
+        } else if (nb < b_end) {
+            load_block<C>(p, nb, lane, nxt);
         }
         BlockOut bo;
         if (decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
