@@ -76,6 +76,7 @@ class df11_arrays(ctypes.Structure):
         ("block_offset", ctypes.c_void_p),
         ("luts", ctypes.c_void_p),
         ("code_lengths", ctypes.c_void_p),
+        ("symbol_table", ctypes.c_void_p),
     ]
 
 
@@ -118,6 +119,7 @@ EXPORTS = (
     "df11_gemm_scratch_bytes", "df11_tile_major", "df11_decompress_host", "df11_read_status", "df11_device_histogram", "df11_plan_from_histogram",
     "df11_device_encode_scratch_words", "df11_device_encode", "df11_device_encode_static",
     "df11_rans_build", "df11_rans_format_arrays", "df11_rans_free", "df11_rans_decompress",
+    "df11_symbol_table",
 )
 
 _lib = None
@@ -157,6 +159,8 @@ def load_library(path: str | None = None):
     lib.df11_gemm_scratch_bytes.argtypes = [ctypes.POINTER(df11_gemm_matrix), ctypes.c_uint32, ctypes.c_uint32]
     lib.df11_gemm_scratch_bytes.restype = ctypes.c_uint64
     lib.df11_tile_major.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32, P]
+    lib.df11_symbol_table.argtypes = [P, P, ctypes.c_uint32, P]
+    lib.df11_symbol_table.restype = ctypes.c_int
     lib.df11_tile_major.restype = ctypes.c_int
     lib.df11_decompress_host.argtypes = [
         ctypes.POINTER(df11_arrays), ctypes.POINTER(df11_arrays), P, P, P, P]
@@ -241,6 +245,8 @@ class Format:
             "block_offset": self._view(a.block_offset, a.num_blocks + 1, np.uint32),
             "luts": self._view(a.luts, a.num_luts * 256, np.uint8).reshape(a.num_luts, 256),
             "code_lengths": self._view(a.code_lengths, 256, np.uint8),
+            # the decoders' derived table (not part of the compressed bytes)
+            "symbol_table": self._view(a.symbol_table, 4096 if a.symbol_table else 0, np.uint32),
         }
 
     def info(self) -> dict:
@@ -298,6 +304,8 @@ class DeviceFormat:
         self.tensors = {}
         self.host_tensors = {}
         for name, arr in arrs.items():
+            if arr.size == 0 and name == "symbol_table":
+                continue
             t = torch.from_numpy(np.ascontiguousarray(arr).reshape(-1).view(np.uint8))
             if pin_host:
                 t = t.pin_memory()
@@ -334,6 +342,8 @@ class DeviceFormat:
         a.block_offset = ts["block_offset"].data_ptr()
         a.luts = ts["luts"].data_ptr()
         a.code_lengths = ts["code_lengths"].data_ptr()
+        if "symbol_table" in ts:
+            a.symbol_table = ts["symbol_table"].data_ptr()
         return a
 
     @property
@@ -546,6 +556,9 @@ def encode_device(w, threads_per_block: int = 64, stream=None, static_scratch: b
         raise Df11Error(6, f"df11_device_encode: the elements do not match their histogram (status word {st})")
     scalars = plan.scalars()
     scalars["max_block_elems"] = int(maxb.item())
+    table = plan.arrays()["symbol_table"]
+    if table.size:  # the decoders' derived table, from the plan's code
+        tensors["symbol_table"] = torch.from_numpy(table.view(np.uint8).copy()).to(dev)
     return DeviceFormat.from_tensors(scalars, tensors, dev), plan
 
 

@@ -10,11 +10,13 @@
 // memory, a dot product, a tensor-core operand tile) is up to the kernel.
 //
 // A kernel's parameter struct P provides: stream, sm, gaps (uint32 halves of
-// the Gaps words), offs, luts, cl, status, n, total_bits, nseg, nblocks,
-// num_luts, min_code_len and cap (bytes of one warp's exponent buffer).
+// the Gaps words), offs, luts, cl, sym_table (optional stored symbol table),
+// status, n, total_bits, nseg, nblocks, num_luts, min_code_len and cap
+// (bytes of one warp's exponent buffer).
 #pragma once
 
 #include "df11.h"
+#include "df11_symtab.h"
 
 #include <cuda_runtime.h>
 
@@ -64,32 +66,11 @@ static_assert(slot_bytes(kSlotShort) % 16 == 0 && slot_bytes(kSlotLong) % 16 == 
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-__device__ __forceinline__ uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
-
-// The page's hierarchical lookup: LUT 0 on the first 8 bits of the window,
-// pointer value 256 - j continues in LUT j on the next 8 bits.  Returns
-// symbol | length << 8; *bad on a dangling pointer.
-__device__ __forceinline__ uint32_t lut_decode(uint32_t win, const uint8_t *luts, const uint8_t *cl,
-                                               uint32_t num_luts, bool *bad)
-{
-    uint32_t e = luts[win >> 24];
-#pragma unroll
-    for (int lvl = 1; lvl <= 3; lvl++) {
-        if (e < kPointerBase)
-            break;
-        uint32_t j = 256u - e;
-        if (j >= num_luts) {
-            *bad = true;
-            return 32u << 8;
-        }
-        e = luts[j * 256u + ((win >> (24 - 8 * lvl)) & 0xFFu)];
-    }
-    if (e >= kPointerBase) {
-        *bad = true;
-        return 32u << 8;
-    }
-    return e | ((uint32_t)cl[e] << 8);
-}
+// ror8 (exponents stored rotated right by one bit) and the page's
+// hierarchical LUT lookup, shared with the host's copy of the derived table
+using df11_symtab::lut_decode;
+using df11_symtab::ror8;
+static_assert(df11_symtab::kIdxBits == kIdxBits && df11_symtab::kPointerBase == kPointerBase, "one definition");
 
 // 96-bit window h:m:l shifted left by c bits (0 <= c <= 32).
 __device__ __forceinline__ void shift_window(uint32_t &h, uint32_t &m, uint32_t &l, uint32_t c)
@@ -370,8 +351,11 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
 // Once per CTA, called by all its nthreads threads (tid = thread index): the
 // page's LUTs and CodeLengths into shared memory and the tables derived from
 // them.  Uses the first 8 KB after Smem::bufs as scratch.
-__device__ __forceinline__ void build_tables(const uint8_t *luts_g, const uint8_t *cl_g, uint32_t num_luts,
-                                             uint8_t *smem, uint32_t tid, uint32_t nthreads)
+// Returns false (every thread alike) when a stored table has an entry no
+// code can produce (more than 3 codes, more than 12 bits, or fewer bits
+// than codes): the decode loop relies on every code taking at least one bit.
+__device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_t *cl_g, uint32_t num_luts,
+                                             const uint32_t *sym_g, uint8_t *smem, uint32_t tid, uint32_t nthreads)
 {
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
     uint8_t *luts = smem + Smem::luts;
@@ -382,36 +366,32 @@ __device__ __forceinline__ void build_tables(const uint8_t *luts_g, const uint8_
         luts[i] = luts_g[i];
     for (uint32_t i = tid; i < 256; i += nthreads)
         cl[i] = cl_g[i];
-    __syncthreads();
-    // first_code[i]: the first code of the 12-bit window i (bits past 12 taken
-    // as zeros): symbol | length << 8, or 0 when that code is longer than 12
-    // bits.  A code found in a zero-filled window is genuine when it ends
-    // inside the window (prefix property).  Scratch in the per-warp buffers,
-    // which are free until the blocks start.
-    uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
-    for (uint32_t i = tid; i < kIdxEntries; i += nthreads) {
+    if (sym_g) {
+        // the stream carries the derived table (df11_build_format): copied
+        // and checked
         bool bad = false;
-        const uint32_t e = lut_decode(i << (32 - kIdxBits), luts, cl, num_luts, &bad);
-        const uint32_t len = e >> 8;
-        first_code[i] = (!bad && len >= 1 && len <= kIdxBits) ? (uint16_t)e : (uint16_t)0;
-    }
-    __syncthreads();
-    // Symbol table: the first three codes of each window, by three dependent
-    // first_code lookups.
-    for (uint32_t i = tid; i < kIdxEntries; i += nthreads) {
-        uint32_t syms = 0, bits = 0, n = 0;
+        for (uint32_t i = tid; i < kIdxEntries / 4; i += nthreads) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(sym_g) + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < 3; j++) {
-            const uint32_t fc = first_code[(i << bits) & (kIdxEntries - 1)];
-            const uint32_t len = fc >> 8;
-            if (len != 0 && len + bits <= kIdxBits && n == (uint32_t)j) {
-                syms |= ror8(fc & 0xFFu) << (8 * j);
-                bits += len;
-                n++;
+            for (int k = 0; k < 4; k++) {
+                const uint32_t n = w[k] >> 29, bits = (w[k] >> 24) & 31u;
+                bad |= n > 3u || bits > (uint32_t)kIdxBits || bits < n || (n == 0 && bits != 0);
             }
+            reinterpret_cast<uint4 *>(sym_tab)[i] = v;
         }
-        // exponents in bytes 0..2, total length in bits 24..28, count in 29..30
-        sym_tab[i] = syms | (bits << 24) | (n << 29);
+        if (__syncthreads_or(bad))
+            return false;
+    } else {
+        __syncthreads();
+        // the first code of each 12-bit window (df11_symtab::first_code), in
+        // scratch in the per-warp buffers, which are free until the blocks start
+        uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
+        for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
+            first_code[i] = df11_symtab::first_code(i, luts, cl, num_luts);
+        __syncthreads();
+        for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
+            sym_tab[i] = df11_symtab::table_entry(i, first_code);
     }
     if (tid < 16) {
         // codes formed by d trailing zero bits, d = 0..15: the all-zero code
@@ -423,6 +403,7 @@ __device__ __forceinline__ void build_tables(const uint8_t *luts_g, const uint8_
         zq[tid] = (lmin >= 1 && !bad) ? (uint8_t)((d / lmin) | ((d % lmin == 0) << 7)) : (uint8_t)0;
     }
     __syncthreads();
+    return true;
 }
 
 // Outputs of one decoded block: stream elements [g0 + lo_off, g0 + hi) have
@@ -608,7 +589,7 @@ df11_status stream_params(const df11_arrays *a, uint32_t *status_dev, P &prm)
         !a->code_lengths)
         return DF11_ERR_INVALID_ARG;
     if (!aligned(a->encoded_exponent, 16) || !aligned(a->packed_sign_mantissa, 16) || !aligned(a->gaps, 8) ||
-        !aligned(a->block_offset, 4))
+        !aligned(a->block_offset, 4) || !aligned(a->symbol_table, 16))
         return DF11_ERR_INVALID_ARG;
     if (a->num_luts < 1 || a->num_luts > DF11_MAX_LUTS || a->n >= (1ull << 32))
         return DF11_ERR_INVALID_ARG;
@@ -627,6 +608,7 @@ df11_status stream_params(const df11_arrays *a, uint32_t *status_dev, P &prm)
     prm.offs = a->block_offset;
     prm.luts = a->luts;
     prm.cl = a->code_lengths;
+    prm.sym_table = a->symbol_table;  // optional: null derives it in each CTA
     prm.status = status_dev;
     prm.n = a->n;
     prm.total_bits = a->total_bits;

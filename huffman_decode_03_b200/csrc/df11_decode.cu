@@ -90,6 +90,7 @@ struct Params {
     const uint32_t *offs;
     const uint8_t *luts;
     const uint8_t *cl;
+    const uint32_t *sym_table;  // optional stored symbol table (null: derived per CTA)
     uint16_t *dst;
     uint32_t *status;
     uint64_t n;
@@ -395,7 +396,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (!kCopy && b < b_end)
         load_block<C>(p, b, lane, cur);
 
-    build_tables(p.luts, p.cl, p.num_luts, smem, (uint32_t)tid, (uint32_t)kThreads);
+    if (!build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads)) {
+        if (tid == 0)
+            atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+        return;
+    }
     if (SLOT < kSlotLong) {
         // short slots hold a segment's codes only when no code is 1 bit long
         // (the all-zero code is the shortest: canonical codes)
@@ -670,6 +675,9 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
     dev.block_offset = d->block_offset;
     dev.luts = d->luts;
     dev.code_lengths = d->code_lengths;
+    // the derived table travels with the other small arrays when both sides
+    // have one; otherwise every CTA derives it
+    dev.symbol_table = h->symbol_table && d->symbol_table ? d->symbol_table : nullptr;
     {
         Params check;  // the whole stream's arguments, before anything is queued
         const df11_status st = stream_params(&dev, status_dev, check);
@@ -731,6 +739,9 @@ extern "C" df11_status df11_decompress_host(const df11_arrays *h, const df11_arr
                                up) == cudaSuccess;
     ok = ok && cudaMemcpyAsync(const_cast<uint8_t *>(d->code_lengths), h->code_lengths, 256, cudaMemcpyHostToDevice,
                                up) == cudaSuccess;
+    ok = ok && (!dev.symbol_table ||
+                cudaMemcpyAsync(const_cast<uint32_t *>(d->symbol_table), h->symbol_table, 4096 * 4,
+                                cudaMemcpyHostToDevice, up) == cudaSuccess);
     if (!ok)
         return cleanup(DF11_ERR_CUDA);
     for (uint32_t k = 0; k < pieces; k++) {

@@ -17,6 +17,7 @@
 // The byte layout is specified in include/df11.h.  Steps 1, 3 and 4 run in
 // parallel over element chunks; everything is exact integer work.
 #include "df11.h"
+#include "df11_symtab.h"
 
 #include <algorithm>
 #include <array>
@@ -272,7 +273,27 @@ df11_status build_luts(const uint8_t *len, const uint32_t *code, std::vector<uin
     return DF11_OK;
 }
 
+// The decoders' derived 12-bit table (df11_symtab.h) from a code's LUTs and
+// CodeLengths: the same functions the kernels run when a stream has none.
+void derive_symbol_table(const uint8_t *luts, const uint8_t *cl, uint32_t num_luts, uint32_t *out)
+{
+    std::vector<uint16_t> fc(df11_symtab::kIdxEntries);
+    for (uint32_t i = 0; i < (uint32_t)df11_symtab::kIdxEntries; i++)
+        fc[i] = df11_symtab::first_code(i, luts, cl, num_luts);
+    for (uint32_t i = 0; i < (uint32_t)df11_symtab::kIdxEntries; i++)
+        out[i] = df11_symtab::table_entry(i, fc.data());
+}
+
 }  // namespace
+
+extern "C" df11_status df11_symbol_table(const uint8_t *luts, const uint8_t *code_lengths, uint32_t num_luts,
+                                         uint32_t *out)
+{
+    if (!luts || !code_lengths || !out || num_luts < 1 || num_luts > DF11_MAX_LUTS)
+        return DF11_ERR_INVALID_ARG;
+    derive_symbol_table(luts, code_lengths, num_luts, out);
+    return DF11_OK;
+}
 
 // ------------------------------------------------------------------ handle
 struct df11_format {
@@ -280,6 +301,7 @@ struct df11_format {
     std::vector<uint8_t> stream, sm, luts;
     std::vector<uint64_t> gaps;
     std::vector<uint32_t> offsets;
+    std::vector<uint32_t> symbol_table;  // the decoders' derived table (df11_symtab.h)
     uint8_t code_lengths[kSymbols];
     uint32_t codes[kSymbols];
     uint64_t hist[kSymbols];
@@ -494,6 +516,9 @@ extern "C" df11_status df11_build_format(const uint16_t *const *mats, const uint
         a.block_offset = f->offsets.data();
         a.luts = f->luts.data();
         a.code_lengths = f->code_lengths;
+        f->symbol_table.assign(df11_symtab::kIdxEntries, 0);
+        derive_symbol_table(f->luts.data(), f->code_lengths, a.num_luts, f->symbol_table.data());
+        a.symbol_table = f->symbol_table.data();
     } catch (const std::bad_alloc &) {
         delete f;
         return DF11_ERR_NO_MEMORY;
@@ -570,6 +595,9 @@ extern "C" df11_status df11_plan_from_histogram(const uint64_t *hist, uint32_t T
         a.block_offset = nullptr;
         a.luts = f->luts.data();
         a.code_lengths = f->code_lengths;
+        f->symbol_table.assign(df11_symtab::kIdxEntries, 0);
+        derive_symbol_table(f->luts.data(), f->code_lengths, a.num_luts, f->symbol_table.data());
+        a.symbol_table = f->symbol_table.data();
         f->plan_only = true;
     } catch (const std::bad_alloc &) {
         delete f;

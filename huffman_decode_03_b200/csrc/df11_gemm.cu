@@ -106,6 +106,7 @@ struct GemmParams {
     const uint32_t *offs;
     const uint8_t *luts;
     const uint8_t *cl;
+    const uint32_t *sym_table;  // optional stored symbol table (null: derived per CTA)
     uint32_t *status;
     uint64_t n;
     uint64_t total_bits;
@@ -709,15 +710,17 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     }
     // the tables (the barriers, flags and tensor-memory address above are
     // published by its __syncthreads)
-    build_tables(p.luts, p.cl, p.num_luts, smem, tid, gemm_threads(DW));
+    const bool tables_ok = build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW));
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
     // short staging slots hold a segment's codes only when no code is 1 bit
     // long (the all-zero code is the shortest): otherwise no role runs, the
     // stream is reported and the tensor memory is released below
-    bool slots_ok = true;
-    if (SLOT < kSlotLong) {
+    bool slots_ok = tables_ok;  // a stored table with an impossible entry: reported below
+    if (!tables_ok && tid == 0)
+        atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+    if (tables_ok && SLOT < kSlotLong) {
         bool bad = false;
         const uint32_t lmin = lut_decode(0u, smem + Smem::luts, smem + Smem::cl, p.num_luts, &bad) >> 8;
         slots_ok = !bad && lmin >= 2;

@@ -122,6 +122,10 @@ typedef struct df11_arrays {
     const uint32_t *block_offset;        /* num_blocks + 1 entries */
     const uint8_t *luts;                 /* num_luts * 256 bytes */
     const uint8_t *code_lengths;         /* 256 bytes, indexed by exponent */
+    const uint32_t *symbol_table;        /* optional, 16-B aligned: the decoders' derived table,
+                                            4096 entries (df11_build_format fills it; see
+                                            df11_symbol_table); NULL: each CTA derives it from
+                                            luts and code_lengths */
 } df11_arrays;
 
 /* Statistics of a built stream ("Ruang kompresi": exponent entropy and the
@@ -286,6 +290,20 @@ uint64_t df11_gemm_scratch_bytes(const df11_gemm_matrix *mats, uint32_t num_mats
  * multiple of 128 and cols of 64.
  */
 df11_status df11_tile_major(const uint16_t *src, uint32_t rows, uint32_t cols, uint16_t *dst);
+
+/*
+ * df11_symbol_table -- host: the decoders' derived 12-bit table of a code
+ * ("Decoding berbasis LUT hierarkis": the page's LUTs answer one code per
+ * lookup chain; the table answers, for each 12-bit window, the first up to
+ * three whole codes inside it: exponents rotated right by one bit in bytes
+ * 0..2, their total length in bits 24..28, their count in bits 29..30).
+ * luts: num_luts * 256 bytes; code_lengths: 256 bytes; out: 4096 entries.
+ * df11_build_format and df11_plan_from_histogram store it with a stream
+ * (df11_arrays.symbol_table); a caller that uploads it spares every CTA of
+ * every launch its derivation.  DF11_ERR_INVALID_ARG for null pointers or
+ * num_luts outside 1..17.
+ */
+df11_status df11_symbol_table(const uint8_t *luts, const uint8_t *code_lengths, uint32_t num_luts, uint32_t *out);
 
 /*
  * df11_decompress_host -- the same decode, starting and ending in host

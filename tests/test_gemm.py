@@ -252,3 +252,27 @@ def test_gemm_reports_a_corrupt_block():
     torch.cuda.synchronize()
     word = int(status.item()) & 0xFFFFFFFF
     assert word != 0 and not (word & 0x80000000), hex(word)
+
+
+@pytest.mark.gpu
+def test_gemm_refuses_an_impossible_symbol_table():
+    # a stored table entry no code can produce (one code of 0 bits) is
+    # refused before any role runs: reported, no timeout, tensor memory freed
+    torch = _torch()
+    shapes = [(256, 1024)]
+    mats = [df11.tile_major(inputs.gaussian(256 * 1024, [78]), 256, 1024)]
+    dev = df11.DeviceFormat(df11.build_format(mats), "cuda")
+    dev.tensors["symbol_table"].view(torch.int32)[300] = 1 << 29
+    xs = [torch.ones(16, 1024, dtype=torch.bfloat16, device="cuda")]
+    ys = [torch.zeros(16, 256, dtype=torch.float32, device="cuda")]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress_gemm(dev, shapes, xs, ys, status)
+    torch.cuda.synchronize()
+    word = int(status.item()) & 0xFFFFFFFF
+    assert word == df11.DF11_ERR_CORRUPT, hex(word)
+    # the next launch on the same context works
+    dev2 = df11.DeviceFormat(df11.build_format(mats), "cuda")
+    status.zero_()
+    df11.decompress_gemm(dev2, shapes, xs, ys, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0

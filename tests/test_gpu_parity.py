@@ -253,7 +253,20 @@ def test_dangling_lut_pointer_is_reported():
 
     def mutate(dev, torch):
         dev.tensors["luts"][ptr_idx] = 240  # child 16, beyond num_luts
+        # without the stored table every code is looked up through the LUTs
+        # (a stored table answers codes of up to 12 bits without them)
+        dev.c_arrays.symbol_table = None
     assert _corrupt_run(w, mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_impossible_symbol_table_entry_is_reported():
+    # a stored table entry no code can produce (one code of 0 bits; 13 bits;
+    # 4 codes) is refused before any block is decoded: the decode loop relies
+    # on every code taking at least one bit
+    for entry in (1 << 29, (1 << 29) | (13 << 24), (4 << 29) | (12 << 24)):
+        def mutate(dev, torch, entry=entry):
+            dev.tensors["symbol_table"].view(torch.int32)[77] = entry - (1 << 32 if entry >= 1 << 31 else 0)
+        assert _corrupt_run(inputs.gaussian(200_000, [32]), mutate) == df11.DF11_ERR_CORRUPT
 
 
 def test_understated_capacity_is_reported():
@@ -356,3 +369,19 @@ def test_workload_stream_of_32_blocks():
             assert torch.equal(out.view(torch.int16), ref), f"block {b}"
             del dev, ref
     assert df11.read_status(status) == 0
+
+
+@pytest.mark.gpu
+def test_stream_without_symbol_table_derives_it():
+    # a stream whose arrays carry no derived table (symbol_table NULL): each
+    # CTA derives it from the LUTs and CodeLengths, with the same result
+    torch = torch_cuda()
+    for w in (inputs.gaussian(3_000_017, [130]), inputs.stress(1_000_003, key=(131, 0))):
+        dev = df11.DeviceFormat(df11.build_format(w), "cuda")
+        assert dev.c_arrays.symbol_table
+        dev.c_arrays.symbol_table = None
+        out = torch.empty(w.size, dtype=torch.int16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.decompress(dev, out, status)
+        assert df11.read_status(status) == 0
+        assert np.array_equal(out.cpu().numpy().view(np.uint16), w)

@@ -147,3 +147,50 @@ def test_null_arguments():
     assert lib.df11_build_format(None, None, 0, 256, None) == 1
     assert lib.df11_format_arrays(None, None) == 1
     lib.df11_free(None)
+
+
+@pytest.mark.parametrize("case", ["gauss", "stress", "one_symbol", "two_symbols"])
+def test_symbol_table_against_the_oracle_code(oracle_mod, case):
+    # the decoders' derived table that df11_build_format stores with a stream:
+    # for every 12-bit window, the first up to three whole codes inside it
+    # (exponents rotated right by one bit), their count and total length --
+    # checked by prefix matching against the oracle's canonical code
+    w = {"gauss": lambda: inputs.gaussian(200_000, [120]),
+         "stress": lambda: inputs.stress(200_000, key=(121, 0)),
+         "one_symbol": lambda: np.full(5000, 0x3F80, np.uint16),
+         "two_symbols": lambda: np.array([0x3F80, 0x4000] * 2500, np.uint16)}[case]()
+    fmt = df11.build_format(w)
+    a = fmt.arrays()
+    tab = a["symbol_table"]
+    assert tab.size == 4096
+    lens = a["code_lengths"].astype(np.int64)
+    codes = oracle_mod.canonical_codes(a["code_lengths"]).astype(np.int64)
+    syms = [s for s in range(256) if lens[s]]
+    complete = sum(2.0 ** -lens[s] for s in syms) == 1.0
+    for i in range(4096):
+        if not complete and i != 0:
+            # an incomplete code (one exponent: the code 0, Kraft sum 1/2):
+            # a valid stream is all zeros; the unused LUT entries repeat the
+            # symbol, so other windows are never decoded
+            continue
+        bits, found = 0, []
+        while len(found) < 3:
+            hit = [s for s in syms if bits + lens[s] <= 12
+                   and (i >> (12 - bits - lens[s])) & ((1 << lens[s]) - 1) == codes[s]]
+            if not hit:
+                break
+            assert len(hit) == 1  # prefix code
+            found.append(hit[0])
+            bits += lens[hit[0]]
+        e = int(tab[i])
+        assert e >> 29 == len(found) and (e >> 24) & 31 == bits, i
+        for j, s in enumerate(found):
+            assert (e >> (8 * j)) & 0xFF == ((s >> 1) | (s << 7)) & 0xFF, (i, j)
+        assert e & (0xFFFFFF >> (8 * (3 - len(found)))) == e & 0xFFFFFF  # unused bytes are zero
+    # the exported function gives the same table
+    out = np.zeros(4096, np.uint32)
+    lib = df11.load_library()
+    assert lib.df11_symbol_table(a["luts"].ctypes.data, a["code_lengths"].ctypes.data,
+                                 fmt.scalars()["num_luts"], out.ctypes.data) == 0
+    assert np.array_equal(out, tab)
+    assert lib.df11_symbol_table(None, a["code_lengths"].ctypes.data, 1, out.ctypes.data) == 1
