@@ -332,6 +332,9 @@ __device__ __forceinline__ uint32_t block_of(const uint32_t *offs, uint32_t nblo
 // the operand image of each K chunk, and finds each unit's blocks.
 __global__ void gemm_prep_kernel(const GemmParams p)
 {
+    // the GEMM kernel may launch now and do its set-up beside this one; it
+    // waits (griddepcontrol.wait) before it reads what this kernel writes
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t g = blockIdx.x * blockDim.x + threadIdx.x;
     if (g < p.num_pieces) {
         uint32_t m = 0;
@@ -713,6 +716,10 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     const bool tables_ok = build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW));
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    // the prep kernel's packed activations and unit ranges are complete and
+    // visible from here on (a launch without a programmatic dependency
+    // passes at once)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // short staging slots hold a segment's codes only when no code is 1 bit
     // long (the all-zero code is the shortest): otherwise no role runs, the
@@ -901,7 +908,20 @@ extern "C" df11_status df11_decompress_gemm(const df11_arrays *a, const df11_gem
     if (cudaGetLastError() != cudaSuccess)
         return DF11_ERR_CUDA;
     const uint32_t grid = (uint32_t)f->sms < prm.num_units ? (uint32_t)f->sms : prm.num_units;
-    kern<<<grid, gemm_threads(dw), smem, s>>>(prm);
+    // programmatic dependent launch: the GEMM kernel's set-up (tensor memory,
+    // barriers, tables) overlaps the prep kernel's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(gemm_threads(dw));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, prm) != cudaSuccess)
+        return DF11_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
 
