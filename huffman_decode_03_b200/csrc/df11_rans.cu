@@ -24,9 +24,12 @@
 // at x = 2^16 with its stream used up, and the lane counts must add up to
 // the block's words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped
 // to the padded array and to the buffer; a lane's start is clamped to the
-// copied words, and a block reads at most 240 words per lane beyond it,
-// inside the buffer's 512 words of slack.  So inconsistent data never reads
-// out of bounds; nothing traps and every loop has a fixed trip count.
+// copied words, and a block reads at most 16 words per chunk and lane beyond
+// it, inside the buffer's slack of 16 chunks + 8 words.  So inconsistent
+// data never reads out of bounds; nothing traps and every loop has a fixed
+// trip count.  Blocks go to warps by striding over the stream when its last
+// round is nearly full, else as contiguous ranges per CTA handed to its
+// warps by a shared-memory counter.
 #include "df11.h"
 
 #include <cuda_runtime.h>
@@ -54,7 +57,7 @@ struct RansParams {
     uint32_t chunks;
     uint32_t wide;  // dst is 32-byte aligned: 32-byte stores
     uint32_t cap;        // words a block may copy into its buffer (multiple of 8, >= max block words + 14)
-    uint32_t bufw;       // words of one buffer: cap plus 512 words of slack for one chunk's reads
+    uint32_t bufw;       // words of one buffer: cap plus the slack a block's reads need past a clamped start
     uint32_t words_end;  // copies end at or below this word: num_words rounded down to 8, plus the 8 padding words
     const uint8_t *lane_words;
 };
@@ -113,7 +116,7 @@ __device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &wp, uin
 // the lane's next word, A the accumulator that takes the exponent byte at
 // the position SEL selects, %6 the table's shared address.  No clamp: a lane
 // starts at most cap words into its buffer and reads at most one word per
-// step, 240 per block, and the buffer has 512 words of slack.
+// step, 16 per chunk, and the buffer has that much slack.
 #define DF11_RSTEP(A, SEL)                       \
     "and.b32 ts, %0, 4095;\n\t"                  \
     "shl.b32 ts, ts, 2;\n\t"                     \
@@ -170,14 +173,21 @@ __device__ __forceinline__ uint4 load_sm(const RansParams &p, uint64_t pos)
     return pos < p.n ? __ldg(reinterpret_cast<const uint4 *>(p.sm + pos)) : make_uint4(0u, 0u, 0u, 0u);
 }
 
+// DYN: blocks as contiguous ranges per CTA handed out by a shared-memory
+// counter; otherwise strided over the stream (balanced when the last round
+// is nearly full).
+template <bool DYN>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const RansParams p)
 {
     __shared__ uint32_t table[kSlots];
     __shared__ uint32_t cum[257];
+    __shared__ uint32_t next_block;
     extern __shared__ __align__(16) uint16_t wbufs[];  // per warp: two buffers of cap words
     const uint32_t tid = threadIdx.x, warp = tid >> 5;
     const int lane = (int)(tid & 31u);
 
+    if (DYN && tid == 0)  // published by the barriers below
+        next_block = (uint32_t)(((uint64_t)p.num_blocks * blockIdx.x) / gridDim.x) + (blockDim.x >> 5);
     // cumulative frequencies (one warp: 8 per lane, shuffle scan)
     if (warp == 0) {
         uint32_t f[8], s = 0;
@@ -225,17 +235,33 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
     }
 
     const uint64_t B = 512ull * p.chunks;
-    const uint32_t warps = blockDim.x >> 5, stride = gridDim.x * warps;
+    const uint32_t warps = blockDim.x >> 5;
     uint16_t *wbuf = wbufs + 2u * p.bufw * warp;
     const uint32_t wbuf_s = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
     const uint32_t tbl = static_cast<uint32_t>(__cvta_generic_to_shared(table));
-    uint32_t b = blockIdx.x * warps + warp, k = 0;
+    // with DYN the CTA's blocks are a contiguous range, and each warp takes
+    // its first one here and every next one from a counter in shared memory;
+    // otherwise the warps stride over the whole stream (when that leaves the
+    // last round nearly full it is as balanced, and neighbouring warps read
+    // neighbouring blocks)
+    const uint32_t stride = gridDim.x * warps;
+    const uint32_t b_end = DYN ? (uint32_t)(((uint64_t)p.num_blocks * (blockIdx.x + 1)) / gridDim.x) : p.num_blocks;
+    uint32_t b = (DYN ? (uint32_t)(((uint64_t)p.num_blocks * blockIdx.x) / gridDim.x) : blockIdx.x * warps) + warp,
+             k = 0;
+    auto take_next = [&]() -> uint32_t {
+        if (!DYN)
+            return b + stride;
+        uint32_t v = 0;
+        if (lane == 0)
+            v = atomicAdd(&next_block, 1u);
+        return __shfl_sync(0xffffffffu, v, 0);
+    };
     // software pipeline: the next block's state, lane count and word
     // offsets, and the next chunk's sign/mantissa bytes, are loaded one step
     // ahead
     uint32_t x_n = 0, c_n = 0, bw0_n = 0, bw1_n = 0, wfirst = 0;
     uint4 s_n = make_uint4(0u, 0u, 0u, 0u);
-    if (b < p.num_blocks) {
+    if (b < b_end) {
         x_n = __ldg(p.states + 32ull * b + lane);
         c_n = __ldg(p.lane_words + 32ull * b + lane);
         bw0_n = __ldg(p.block_word + b);
@@ -243,7 +269,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s);
         s_n = load_sm(p, b * B + 16u * (uint32_t)lane);
     }
-    for (; b < p.num_blocks; b += stride, k ^= 1u) {
+    uint32_t nb = 0;
+    for (; b < b_end; b = nb, k ^= 1u) {
         // this block's words have landed; the next block's go to the other buffer
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncwarp();
@@ -263,8 +290,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         bool bad = total != bw1_n - bw0_n || bw1_n - wfirst > p.cap;
         uint32_t wp = wb_s + 2u * (first < p.cap ? first : p.cap);  // clamped: inconsistent counts
         const bool full = (b + 1) * B <= p.n;  // warp-uniform
-        const uint32_t nb = b + stride;
-        if (nb < p.num_blocks) {
+        nb = take_next();
+        if (nb < b_end) {
             x_n = __ldg(p.states + 32ull * nb + lane);
             c_n = __ldg(p.lane_words + 32ull * nb + lane);
             bw0_n = __ldg(p.block_word + nb);
@@ -279,7 +306,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         for (uint32_t j = 0; j < p.chunks; j++) {
             const uint64_t pos0 = b * B + 512ull * j + 16u * (uint32_t)lane;
             const uint4 s4 = s_n;
-            s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512 : (uint64_t)nb * B + 16u * (uint32_t)lane);
+            s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512
+                                              : (!DYN || nb < b_end ? (uint64_t)nb * B + 16u * (uint32_t)lane : p.n));
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
             if (full)
                 decode_chunk_full(x, wp, tbl, acc);
@@ -319,7 +347,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
 std::mutex g_rans_mu;
 int g_rans_sms[64] = {0};
 int g_rans_optin[64] = {0};
-uint32_t g_rans_granted[64] = {0};
+uint32_t g_rans_granted[2][64] = {};
 
 }  // namespace
 
@@ -369,24 +397,27 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     p.cap = ((a->max_block_words + 16u) + 7u) & ~7u;
     p.words_end = (uint32_t)((a->num_words & ~7ull) + 8);
     // two buffers of cap words per warp; as many warps as shared memory holds
-    p.bufw = p.cap + 512u;
+    p.bufw = p.cap + 16u * p.chunks + 8u;  // a lane reads at most 16 words per chunk past its clamped start
     const uint64_t per_warp = 4ull * p.bufw, room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
     const uint64_t warps = room / per_warp < (uint64_t)kMaxWarps ? room / per_warp : (uint64_t)kMaxWarps;
     if (warps == 0)
         return DF11_ERR_INVALID_ARG;  // cannot happen for chunks <= 64 (at most 24,576 words per block)
     const uint64_t dyn = per_warp * warps;
-    {
-        std::lock_guard<std::mutex> lock(g_rans_mu);
-        if (dyn > g_rans_granted[dev]) {
-            if (cudaFuncSetAttribute(rans_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) !=
-                cudaSuccess)
-                return DF11_ERR_CUDA;
-            g_rans_granted[dev] = (uint32_t)dyn;
-        }
-    }
     uint32_t grid = (uint32_t)((a->num_blocks + warps - 1) / warps);
     if (grid > (uint32_t)sms)
         grid = (uint32_t)sms;
-    rans_decode_kernel<<<grid, (uint32_t)(warps * 32), (size_t)dyn, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    // striding when its last round is at least 85 % full, else ranges per CTA
+    const uint64_t W = (uint64_t)grid * warps, rem = a->num_blocks % W;
+    const int di = (rem != 0 && rem * 100 < W * 85) ? 1 : 0;
+    auto kern = di ? rans_decode_kernel<true> : rans_decode_kernel<false>;
+    {
+        std::lock_guard<std::mutex> lock(g_rans_mu);
+        if (dyn > g_rans_granted[di][dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
+                return DF11_ERR_CUDA;
+            g_rans_granted[di][dev] = (uint32_t)dyn;
+        }
+    }
+    kern<<<grid, (uint32_t)(warps * 32), (size_t)dyn, reinterpret_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? DF11_OK : DF11_ERR_CUDA;
 }
