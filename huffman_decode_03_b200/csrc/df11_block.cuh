@@ -30,14 +30,17 @@ constexpr int kIdxEntries = 1 << kIdxBits;
 constexpr int kLutBytes = DF11_MAX_LUTS * 256;
 constexpr uint32_t kPointerBase = 240;
 // bytes per lane's staging slot: codes start at most every lmin bits of a
-// 64-bit segment, plus two zero-fill codes and the two bytes the decode
-// loop's last 3-byte store may write past its codes: 36 when the shortest
-// code has >= 2 bits, 68 otherwise (both odd word counts, so the 32 lanes'
-// slots start in 32 distinct banks)
+// 64-bit segment, plus two zero-fill codes, stored as whole words (the last
+// word may hold up to three bytes past the codes): 36 when the shortest code
+// has >= 2 bits, 68 otherwise (both odd word counts, so the 32 lanes' slots
+// start in 32 distinct banks)
 constexpr uint32_t kSlotShort = 36, kSlotLong = 68;
 // per warp: two chains x 32 lanes, plus 32 bytes so that a chain of
-// inconsistent data stays inside the warp's own slots; such a block is
-// reported and writes nothing
+// inconsistent data stays inside the warp's own slots (such a block is
+// reported and writes nothing): a chain reads at most 95 bits before its last
+// lookup, each code of >= 2 bits (short slots) or >= 1 bit (long slots, and
+// long codes >= 13), so it holds at most 47 + 3 or 94 + 3 codes, whose words
+// end by byte 52 or 100 of its slot
 __host__ __device__ constexpr uint32_t slot_bytes(uint32_t stride) { return 2 * 32 * stride + 32; }
 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
@@ -123,73 +126,111 @@ __device__ __forceinline__ void st_u32(uint32_t addr, uint32_t v)
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v));
 }
 
-// Decode loop for two chains (A, B) of one lane, in PTX.  Symbol-table
-// entry: up to three rotated exponents in bytes 0..2, their total length in
-// bits 24..28, their number in bits 29..30 (0 = a code longer than 12 bits).
-// A chain is active while pos < pend and its last entry was not 0; the bits
-// of its window past pend are zeros.  Per lookup: the three exponent bytes go
-// to the chain's staging slot at q unconditionally (bytes past the codes
-// found are overwritten by the next lookup or never read), q advances by the
-// count, the window and pos by the length.  (entry >> 24) serves as the
-// funnel-shift amount directly: wrap mode reads only its low five bits.  An
-// entry of 0 changes nothing and stops its chain: the caller resolves that
-// long code, resets the chain's entry to non-zero and calls again.
-__device__ __forceinline__ void decode_bulk2(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA, int &posA,
-                                             uint32_t &eA, uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
-                                             int &posB, uint32_t &eB, int pendA, int pendB, uint32_t sym_base)
+// Bytes of shared memory by 32-bit address, for lut_decode: keeps the
+// tables' addresses in one register each instead of generic pointers.
+struct SharedBytes {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t operator[](uint32_t i) const { return ld_u8(base + i); }
+};
+
+// Decode loop for two chains (A, B) of one lane, in PTX.  Shared-memory
+// table entry (table_word): number of codes in bits 0..1, their total length
+// in bits 2..6, their rotated exponents in bits 8..31 (bytes past the count
+// zero); 0 = a code longer than 12 bits.  A chain is active while rem (its
+// bits left before pend) is > 0 and its last entry was not 0; the bits of its
+// window past pend are zeros.  Per lookup the window advances and rem drops
+// by the length ((entry >> 2) serves as the funnel-shift amount directly:
+// wrap mode reads only its low five bits) and the exponents are added to the
+// chain's pending word w at byte n, where mul = 2^(8 n); mul rotates left by
+// 8 x count bits.  When the pending word fills (the rotation wraps, mul
+// decreases) it is stored at the slot address qa, qa advances one word and w
+// keeps the bytes that spilled past it.  An entry of 0 changes nothing and
+// stops its chain: the caller resolves that long code and calls again.
+struct Chain {
+    uint32_t h, m, l;  // 96-bit window, next bit at the top of h
+    int rem;           // pend - bits consumed
+    uint32_t qa;       // slot word that w goes to
+    uint32_t w;        // pending exponents, bytes 0..n-1
+    uint32_t mul;      // 2^(8 n)
+};
+
+__device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_base)
 {
     asm volatile(
         "{\n\t"
-        ".reg .pred pa, pb, pz;\n\t"
-        ".reg .u32 ca, cb, t;\n\t"
+        ".reg .pred pa, pb, ka, kb, pz, po;\n\t"
+        ".reg .u32 ea, eb, ca, t;\n\t"
+        "setp.eq.u32 ka, 0, 0;\n\t"
+        "setp.eq.u32 kb, 0, 0;\n\t"
         "DB_TOP:\n\t"
-        "setp.lt.s32 pa, %4, %12;\n\t"
-        "setp.lt.s32 pb, %10, %13;\n\t"
-        "setp.ne.and.u32 pa, %5, 0, pa;\n\t"
-        "setp.ne.and.u32 pb, %11, 0, pb;\n\t"
+        "setp.gt.and.s32 pa, %3, 0, ka;\n\t"
+        "setp.gt.and.s32 pb, %10, 0, kb;\n\t"
         "or.pred pz, pa, pb;\n\t"
         "@!pz bra DB_END;\n\t"
-        "@pa shr.u32 %5, %0, 20;\n\t"
-        "@pb shr.u32 %11, %6, 20;\n\t"
-        "@pa mad.lo.u32 %5, %5, 4, %14;\n\t"
-        "@pb mad.lo.u32 %11, %11, 4, %14;\n\t"
-        "@pa ld.shared.u32 %5, [%5];\n\t"
-        "@pb ld.shared.u32 %11, [%11];\n\t"
+        "@pa shr.u32 ea, %0, 20;\n\t"
+        "@pb shr.u32 eb, %7, 20;\n\t"
+        "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"
+        "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"
+        "@pa ld.shared.u32 ea, [ea];\n\t"
+        "@pb ld.shared.u32 eb, [eb];\n\t"
         // chain A
-        "@pa st.shared.u8 [%3], %5;\n\t"
-        "@pa mul.hi.u32 t, %5, 16777216;\n\t"
-        "@pa st.shared.u8 [%3+1], t;\n\t"
-        "@pa mul.hi.u32 t, %5, 65536;\n\t"
-        "@pa st.shared.u8 [%3+2], t;\n\t"
-        "@pa shr.u32 ca, %5, 24;\n\t"
-        "@pa mul.hi.u32 t, %5, 8;\n\t"
-        "@pa add.u32 %3, %3, t;\n\t"
+        "@pa shr.u32 ca, ea, 2;\n\t"
         "@pa and.b32 t, ca, 31;\n\t"
-        "@pa add.s32 %4, %4, t;\n\t"
+        "@pa sub.s32 %3, %3, t;\n\t"
         "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
+        "@pa setp.ne.u32 ka, ea, 0;\n\t"
+        "@pa shr.u32 t, ea, 8;\n\t"
+        "@pa mul.hi.u32 ca, t, %6;\n\t"
+        "@pa mad.lo.u32 t, t, %6, %5;\n\t"
+        "@pa shl.b32 %5, ea, 3;\n\t"
+        "@pa shf.l.wrap.b32 %5, %6, %6, %5;\n\t"
+        "setp.lt.and.u32 po, %5, %6, pa;\n\t"
+        "@pa mov.b32 %6, %5;\n\t"
+        "@po st.shared.u32 [%4], t;\n\t"
+        "@po add.u32 %4, %4, 4;\n\t"
+        "@pa selp.b32 %5, ca, t, po;\n\t"
         // chain B
-        "@pb st.shared.u8 [%9], %11;\n\t"
-        "@pb mul.hi.u32 t, %11, 16777216;\n\t"
-        "@pb st.shared.u8 [%9+1], t;\n\t"
-        "@pb mul.hi.u32 t, %11, 65536;\n\t"
-        "@pb st.shared.u8 [%9+2], t;\n\t"
-        "@pb shr.u32 cb, %11, 24;\n\t"
-        "@pb mul.hi.u32 t, %11, 8;\n\t"
-        "@pb add.u32 %9, %9, t;\n\t"
-        "@pb and.b32 t, cb, 31;\n\t"
-        "@pb add.s32 %10, %10, t;\n\t"
-        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
-        "@pb shf.l.wrap.b32 %7, %8, %7, cb;\n\t"
-        "@pb shf.l.wrap.b32 %8, 0, %8, cb;\n\t"
+        "@pb shr.u32 ca, eb, 2;\n\t"
+        "@pb and.b32 t, ca, 31;\n\t"
+        "@pb sub.s32 %10, %10, t;\n\t"
+        "@pb shf.l.wrap.b32 %7, %8, %7, ca;\n\t"
+        "@pb shf.l.wrap.b32 %8, %9, %8, ca;\n\t"
+        "@pb shf.l.wrap.b32 %9, 0, %9, ca;\n\t"
+        "@pb setp.ne.u32 kb, eb, 0;\n\t"
+        "@pb shr.u32 t, eb, 8;\n\t"
+        "@pb mul.hi.u32 ca, t, %13;\n\t"
+        "@pb mad.lo.u32 t, t, %13, %12;\n\t"
+        "@pb shl.b32 %12, eb, 3;\n\t"
+        "@pb shf.l.wrap.b32 %12, %13, %13, %12;\n\t"
+        "setp.lt.and.u32 po, %12, %13, pb;\n\t"
+        "@pb mov.b32 %13, %12;\n\t"
+        "@po st.shared.u32 [%11], t;\n\t"
+        "@po add.u32 %11, %11, 4;\n\t"
+        "@pb selp.b32 %12, ca, t, po;\n\t"
         "bra DB_TOP;\n\t"
         "DB_END:\n\t"
         "}"
-        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(eA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB),
-          "+r"(posB), "+r"(eB)
-        : "r"(pendA), "r"(pendB), "r"(sym_base)
+        : "+r"(A.h), "+r"(A.m), "+r"(A.l), "+r"(A.rem), "+r"(A.qa), "+r"(A.w), "+r"(A.mul), "+r"(B.h), "+r"(B.m),
+          "+r"(B.l), "+r"(B.rem), "+r"(B.qa), "+r"(B.w), "+r"(B.mul)
+        : "r"(sym_base)
         : "memory");
+}
+
+// Adds one exponent (rotated) to a chain's pending word; the long-code path.
+__device__ __forceinline__ void chain_put1(Chain &c, uint32_t sym)
+{
+    const uint32_t lo = sym * c.mul + c.w;
+    const uint32_t nm = __funnelshift_l(c.mul, c.mul, 8);
+    if (nm < c.mul) {
+        st_u32(c.qa, lo);
+        c.qa += 4;
+        c.w = 0;
+    } else {
+        c.w = lo;
+    }
+    c.mul = nm;
 }
 
 // Registers one lane holds for one block: per chain its 12 stream bytes and
@@ -348,14 +389,31 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
         : "memory");
 }
 
+// A symbol-table entry (df11_symtab::table_entry: exponents in bytes 0..2,
+// total length in bits 24..28, count in bits 29..30) in the decode loop's
+// shared-memory form: count in bits 0..1, length in bits 2..6, the count's
+// exponents from bit 8 on, the bytes past them zero.  *bad when no code set
+// with codes of >= min_bits bits each produces the entry (more than 3
+// codes, more than 12 bits, fewer than min_bits x count bits, or a length
+// without codes).
+__device__ __forceinline__ uint32_t table_word(uint32_t e, uint32_t min_bits, bool &bad)
+{
+    const uint32_t n = e >> 29, bits = (e >> 24) & 31u;
+    bad |= n > 3u || bits > (uint32_t)kIdxBits || bits < n * min_bits || (n == 0 && bits != 0);
+    const uint32_t syms = n >= 3u ? e & 0xFFFFFFu : e & ((1u << (8u * n)) - 1u);
+    return (n & 3u) | ((bits & 31u) << 2) | (syms << 8);
+}
+
 // Once per CTA, called by all its nthreads threads (tid = thread index): the
 // page's LUTs and CodeLengths into shared memory and the tables derived from
-// them.  Uses the first 8 KB after Smem::bufs as scratch.
-// Returns false (every thread alike) when a stored table has an entry no
-// code can produce (more than 3 codes, more than 12 bits, or fewer bits
-// than codes): the decode loop relies on every code taking at least one bit.
+// them.  Uses the first 8 KB after Smem::bufs as scratch.  min_bits: the
+// shortest code the staging slots allow (2 for short slots, else 1).
+// Returns false (every thread alike) when the symbol table, stored or
+// derived, has an entry no such code set produces (table_word): the decode
+// loop's slot bound relies on every code taking at least min_bits bits.
 __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_t *cl_g, uint32_t num_luts,
-                                             const uint32_t *sym_g, uint8_t *smem, uint32_t tid, uint32_t nthreads)
+                                             const uint32_t *sym_g, uint8_t *smem, uint32_t tid, uint32_t nthreads,
+                                             uint32_t min_bits)
 {
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
     uint8_t *luts = smem + Smem::luts;
@@ -366,22 +424,15 @@ __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_
         luts[i] = luts_g[i];
     for (uint32_t i = tid; i < 256; i += nthreads)
         cl[i] = cl_g[i];
+    bool bad = false;
     if (sym_g) {
         // the stream carries the derived table (df11_build_format): copied
         // and checked
-        bool bad = false;
         for (uint32_t i = tid; i < kIdxEntries / 4; i += nthreads) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(sym_g) + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                const uint32_t n = w[k] >> 29, bits = (w[k] >> 24) & 31u;
-                bad |= n > 3u || bits > (uint32_t)kIdxBits || bits < n || (n == 0 && bits != 0);
-            }
-            reinterpret_cast<uint4 *>(sym_tab)[i] = v;
+            reinterpret_cast<uint4 *>(sym_tab)[i] = make_uint4(table_word(v.x, min_bits, bad), table_word(v.y, min_bits, bad),
+                                                             table_word(v.z, min_bits, bad), table_word(v.w, min_bits, bad));
         }
-        if (__syncthreads_or(bad))
-            return false;
     } else {
         __syncthreads();
         // the first code of each 12-bit window (df11_symtab::first_code), in
@@ -391,8 +442,10 @@ __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_
             first_code[i] = df11_symtab::first_code(i, luts, cl, num_luts);
         __syncthreads();
         for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
-            sym_tab[i] = df11_symtab::table_entry(i, first_code);
+            sym_tab[i] = table_word(df11_symtab::table_entry(i, first_code), min_bits, bad);
     }
+    if (__syncthreads_or(bad))
+        return false;
     if (tid < 16) {
         // codes formed by d trailing zero bits, d = 0..15: the all-zero code
         // (the canonical first code, of length lmin) repeated d / lmin times;
@@ -417,16 +470,19 @@ struct BlockOut {
 
 // Decodes format block b (its registers in cur, loaded by load_block) into
 // the warp's write buffer at shared address exp_base, through the lane's
-// staging slots at slot_base; luts, cl and zq are the shared copies,
-// sym_base the symbol table's shared address.  Asks L2 for the block's
+// staging slots at slot_base; sym_base: the shared address of the symbol
+// table (and of the tables after it).  Asks L2 for the block's
 // sign/mantissa bytes first.  Returns false, after setting DF11_ERR_CORRUPT
 // in *p.status, when the block is inconsistent (nothing placed).  Called by
 // all 32 lanes of the warp.
 template <int C, uint32_t SLOT, class P>
 __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, const BlockRegs<C> &cur,
-                                             const uint8_t *luts, const uint8_t *cl, const uint8_t *zq,
                                              uint32_t sym_base, uint32_t exp_base, uint32_t slot_base, BlockOut &out)
 {
+    // the LUTs, CodeLengths and zero-code table lie at fixed offsets from the
+    // symbol table (Smem)
+    const SharedBytes luts{sym_base + (Smem::luts - Smem::sym)}, cl{sym_base + (Smem::cl - Smem::sym)};
+    const uint32_t zq = sym_base + (Smem::zq - Smem::sym);
     constexpr uint32_t T = 32 * C;
     const uint32_t o0 = cur.o0, o1 = cur.o1;
     const uint32_t lo_off = o0 & 15u;
@@ -482,29 +538,32 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
     // (< 12) and the count by overshoot / lmin.
     uint32_t cnt[2];
     {
-        uint32_t q[2], q0[2], e[2] = {1u, 1u};
-        int pos[2];
+        Chain ch[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
-            q0[k] = slot_base + k * (32 * SLOT);
-            q[k] = q0[k];
-            pos[k] = pos0[k];
+            ch[k].h = h[k];
+            ch[k].m = m[k];
+            ch[k].l = l[k];
+            ch[k].rem = pend[k] - pos0[k];
+            ch[k].qa = slot_base + k * (32 * SLOT);
+            ch[k].w = 0u;
+            ch[k].mul = 1u;
         }
         for (;;) {  // each pass resolves >= 1 code or ends both chains
-            decode_bulk2(h[0], m[0], l[0], q[0], pos[0], e[0], h[1], m[1], l[1], q[1], pos[1], e[1], pend[0],
-                         pend[1], sym_base);
+            decode_bulk2(ch[0], ch[1], sym_base);
             bool any_long = false;
 #pragma unroll
             for (int k = 0; k < 2; k++) {
-                if (pos[k] < pend[k]) {
+                if (ch[k].rem > 0) {
                     // stopped on a code longer than 12 bits: the page's LUTs
-                    const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
-                    const uint32_t len = (d >> 8) ? (d >> 8) : 1u;
-                    st_u8(q[k], ror8(d & 0xFFu));
-                    q[k] += 1;
-                    pos[k] += (int)len;
-                    shift_window(h[k], m[k], l[k], len);
-                    e[k] = 1u;
+                    // (a code the table leaves to them has >= 13 bits)
+                    const uint32_t d = lut_decode(ch[k].h, luts, cl, p.num_luts, &bad);
+                    uint32_t len = d >> 8;
+                    bad |= len <= (uint32_t)kIdxBits;
+                    len = len > (uint32_t)kIdxBits ? len : (uint32_t)kIdxBits + 1u;
+                    chain_put1(ch[k], ror8(d & 0xFFu));
+                    ch[k].rem -= (int)len;
+                    shift_window(ch[k].h, ch[k].m, ch[k].l, len);
                     any_long = true;
                 }
             }
@@ -513,10 +572,13 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
         }
 #pragma unroll
         for (int k = 0; k < 2; k++) {
-            const uint32_t d = (uint32_t)(pos[k] - pend[k]);  // >= 0
-            const uint32_t z = zq[d & 15u];
+            st_u32(ch[k].qa, ch[k].w);  // the pending bytes
+            const uint32_t q0 = slot_base + k * (32 * SLOT);
+            const uint32_t bytes = ch[k].qa - q0 + ((uint32_t)(__ffs((int)ch[k].mul) - 1) >> 3);
+            const uint32_t d = (uint32_t)(-ch[k].rem);  // overshoot past pend, >= 0
+            const uint32_t z = ld_u8(zq + (d & 15u));
             bad |= d > 15u || !(z & 0x80u);
-            cnt[k] = q[k] - q0[k] - (z & 0x7Fu);
+            cnt[k] = bytes - (z & 0x7Fu);
         }
     }
 

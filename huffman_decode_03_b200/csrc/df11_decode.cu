@@ -369,9 +369,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
     constexpr bool kCopy = SLOT == kSlotShort;  // metadata by cp.async
     extern __shared__ __align__(128) uint8_t smem[];
-    const uint8_t *luts = smem + Smem::luts;
-    const uint8_t *cl = smem + Smem::cl;
-    const uint8_t *zq = smem + Smem::zq;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *exp_s = smem + Smem::bufs + warp * warp_bytes<C, SLOT>(p.cap);
     uint8_t *slots = exp_s + p.cap;
@@ -396,7 +393,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (!kCopy && b < b_end)
         load_block<C>(p, b, lane, cur);
 
-    if (!build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads)) {
+    if (!build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
+                      SLOT < kSlotLong ? 2u : 1u)) {
         if (tid == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         return;
@@ -405,7 +403,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         // short slots hold a segment's codes only when no code is 1 bit long
         // (the all-zero code is the shortest: canonical codes)
         bool bad = false;
-        const uint32_t lmin = lut_decode(0u, luts, cl, p.num_luts, &bad) >> 8;
+        const uint32_t lmin = lut_decode(0u, smem + Smem::luts, smem + Smem::cl, p.num_luts, &bad) >> 8;
         if (bad || lmin < 2) {
             if (tid == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
@@ -432,7 +430,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             load_block<C>(p, nb, lane, nxt);
         }
         BlockOut bo;
-        if (decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo)) {
+        if (decode_block<C, SLOT>(p, b, lane, cur, sym_base, exp_base, slot_base, bo)) {
             // ---- merge with sign/mantissa (from L2)
             const uint64_t g0 = bo.g0;
             const uint32_t lo_off = bo.lo_off, hi = bo.hi;
@@ -471,7 +469,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
                 const uint32_t l = head ? lane : 16 * c_end + (lane - 16);
                 const bool want = head ? (lo_off != 0 || hi < 16) : (c_end > 0 && (hi & 15u) != 0);
                 if (want && l >= lo_off && l < hi)
-                    p.dst[g0 + l] = merge1(__ldg(smg + l), exp_s[l]);
+                    p.dst[g0 + l] = merge1(__ldg(smg + l), ld_u8(exp_base + l));
             } else {
                 // 8 elements per lane and step, one 16-byte store: a warp's
                 // stores cover 512 contiguous bytes
@@ -493,7 +491,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
                 const uint32_t l = lane < 16 ? (uint32_t)lane : tail0 + (lane - 16);
                 const bool want = lane < 16 ? (l >= lo_off && l < head_end) : (lane < 24 && l < hi);
                 if (want)
-                    p.dst[g0 + l] = merge1(__ldg(smg + l), exp_s[l]);
+                    p.dst[g0 + l] = merge1(__ldg(smg + l), ld_u8(exp_base + l));
             }
             __syncwarp();
         }

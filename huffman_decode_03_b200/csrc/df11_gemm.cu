@@ -452,9 +452,6 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
 {
     const uint32_t E = p.etiles;
     uint8_t *exp_s = smem + Smem::bufs + warp * Smem::per_warp(p.cap, SLOT);
-    const uint8_t *luts = smem + Smem::luts;
-    const uint8_t *cl = smem + Smem::cl;
-    const uint8_t *zq = smem + Smem::zq;
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base =
@@ -487,7 +484,7 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
             const uint64_t o0 = cur.o0, o1 = cur.o1 > cur.o0 ? cur.o1 : cur.o0;
             const uint64_t r0 = o0 > e0 ? o0 : e0, r1 = o1 < e1 ? o1 : e1;
             BlockOut bo;
-            const bool dok = decode_block<C, SLOT>(p, b, lane, cur, luts, cl, zq, sym_base, exp_base, slot_base, bo);
+            const bool dok = decode_block<C, SLOT>(p, b, lane, cur, sym_base, exp_base, slot_base, bo);
             if (r0 < r1) {
                 const uint32_t t_first = (uint32_t)((r0 - e0) >> kTileShift);
                 const uint32_t t_last = (uint32_t)((r1 - 1 - e0) >> kTileShift);
@@ -713,7 +710,8 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     }
     // the tables (the barriers, flags and tensor-memory address above are
     // published by its __syncthreads)
-    const bool tables_ok = build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW));
+    const bool tables_ok = build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW),
+                                        SLOT < kSlotLong ? 2u : 1u);
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
     // the prep kernel's packed activations and unit ranges are complete and

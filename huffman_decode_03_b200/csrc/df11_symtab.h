@@ -28,8 +28,10 @@ constexpr uint32_t kPointerBase = 240;
 DF11_HD uint32_t ror8(uint32_t s) { return ((s >> 1) | (s << 7)) & 0xFFu; }
 
 // The page's hierarchical lookup of the code at the top of win: symbol |
-// length << 8; *bad on a dangling pointer.
-DF11_HD uint32_t lut_decode(uint32_t win, const uint8_t *luts, const uint8_t *cl, uint32_t num_luts, bool *bad)
+// length << 8; *bad on a dangling pointer.  Bytes: anything indexable by a
+// byte offset (a pointer, or a device accessor of shared memory).
+template <class Bytes>
+DF11_HD uint32_t lut_decode(uint32_t win, const Bytes &luts, const Bytes &cl, uint32_t num_luts, bool *bad)
 {
     uint32_t e = luts[win >> 24];
 #if defined(__CUDA_ARCH__)

@@ -269,6 +269,50 @@ def test_impossible_symbol_table_entry_is_reported():
         assert _corrupt_run(inputs.gaussian(200_000, [32]), mutate) == df11.DF11_ERR_CORRUPT
 
 
+def _entry_i32(v):
+    return v - (1 << 32) if v >= 1 << 31 else v
+
+
+def test_symbol_table_entry_of_codes_shorter_than_the_slots_allow_is_reported():
+    # a stream whose shortest code has 2 bits decodes through short staging
+    # slots; a stored entry of two 1-bit codes would overrun them, so the
+    # table is refused before any block is decoded
+    w = inputs.gaussian(200_000, [32])
+    assert df11.build_format(w).scalars()["min_code_len"] >= 2
+
+    def mutate(dev, torch):
+        dev.tensors["symbol_table"].view(torch.int32)[77] = _entry_i32((2 << 29) | (2 << 24) | 0x0101)
+    assert _corrupt_run(w, mutate) == df11.DF11_ERR_CORRUPT
+
+
+def test_symbol_table_bytes_past_the_count_are_ignored():
+    # an entry's exponent bytes past its count carry no meaning: filled with
+    # ones, the stream still decodes exactly
+    torch = torch_cuda()
+    w = inputs.gaussian(300_000, [30])
+    fmt = df11.build_format(w)
+    dev = df11.DeviceFormat(fmt, "cuda")
+    t = dev.tensors["symbol_table"].view(torch.int32).cpu().numpy().view(np.uint32).copy()
+    n = t >> 29
+    keep = np.where(n >= 3, 0xFFFFFF, (np.uint32(1) << (8 * n).astype(np.uint32)) - 1).astype(np.uint32)
+    filled = t | (np.uint32(0xFFFFFF) & ~keep)
+    assert (filled != t).any()
+    dev.tensors["symbol_table"].view(torch.int32).copy_(torch.from_numpy(filled.view(np.int32)))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(dev.n, dtype=torch.bfloat16, device="cuda")
+    df11.decompress(dev, out, status)
+    assert df11.read_status(status) == 0
+    assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), w)
+
+
+def test_symbol_table_that_leaves_short_codes_to_the_luts_is_reported():
+    # an entry of 0 sends its window to the page's LUTs as a code longer than
+    # 12 bits; the LUTs finding a shorter one there marks the table wrong
+    def mutate(dev, torch):
+        dev.tensors["symbol_table"].zero_()
+    assert _corrupt_run(inputs.gaussian(200_000, [31]), mutate) == df11.DF11_ERR_CORRUPT
+
+
 def test_understated_capacity_is_reported():
     def mutate(dev, torch):
         dev.c_arrays.max_block_elems = 100
