@@ -125,7 +125,12 @@ typedef struct df11_arrays {
     const uint32_t *symbol_table;        /* optional, 16-B aligned: the decoders' derived table,
                                             4096 entries (df11_build_format fills it; see
                                             df11_symbol_table); NULL: each CTA derives it from
-                                            luts and code_lengths */
+                                            luts and code_lengths.  Exponent bytes past an
+                                            entry's count are ignored; an entry of more than
+                                            3 codes or 12 bits, of fewer bits than codes (or
+                                            than 2 per code when min_code_len >= 2), or a 0
+                                            entry where the LUTs hold a code of <= 12 bits,
+                                            is reported as DF11_ERR_CORRUPT */
 } df11_arrays;
 
 /* Statistics of a built stream ("Ruang kompresi": exponent entropy and the
