@@ -19,8 +19,11 @@
 // scan per block.  A block's words are read from shared memory: each warp
 // has two buffers, and the next block's words are copied into the other one
 // (cp.async) and its sign/mantissa bytes prefetched into L2 while the
-// current block decodes.  The warps per CTA are as many as the buffers fit
-// (32 for blocks of up to about 1,140 words).  Every lane must end the block
+// current block decodes.  The buffers are sized for the stream's largest
+// block while 32 warps per CTA still fit (blocks of up to about 1,500 words);
+// the few blocks of a stream that exceed that read their words straight from
+// global memory (asked into L2 one block ahead), each load clamped to the
+// word array.  Every lane must end the block
 // at x = 2^16 with its stream used up, and the lane counts must add up to
 // the block's words; otherwise DF11_ERR_CORRUPT is set.  Copies are clamped
 // to the padded array and to the buffer; a lane's start is clamped to the
@@ -56,7 +59,8 @@ struct RansParams {
     uint32_t num_blocks;
     uint32_t chunks;
     uint32_t wide;  // dst is 32-byte aligned: 32-byte stores
-    uint32_t cap;        // words a block may copy into its buffer (multiple of 8, >= max block words + 14)
+    uint32_t cap;        // words a block may copy into its buffer (multiple of 8); a block spanning more
+                         // reads its words from global memory
     uint32_t bufw;       // words of one buffer: cap plus the slack a block's reads need past a clamped start
     uint32_t words_end;  // copies end at or below this word: num_words rounded down to 8, plus the 8 padding words
     const uint8_t *lane_words;
@@ -79,31 +83,51 @@ __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e_rot)
     return (uint16_t)((((s & 0x80u) | (e_rot & 0x7Fu)) << 8) | (e_rot & 0x80u) | (s & 0x7Fu));
 }
 
+// The lane's next word: from its block's buffer in shared memory (a 32-bit
+// shared address) or, for a block too large for the buffer, from global
+// memory (a 64-bit address); the address advances past it.
+__device__ __forceinline__ uint32_t next_word(uint32_t &wp)
+{
+    uint32_t w;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(wp) : "memory");
+    wp += 2u;
+    return w;
+}
+struct GlobalWords {
+    uint64_t p;     // address of the lane's next word
+    uint64_t last;  // the word array's last word: loads are clamped to it
+};
+__device__ __forceinline__ uint32_t next_word(GlobalWords &g)
+{
+    uint32_t w;
+    const uint64_t a = g.p < g.last ? g.p : g.last;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=r"(w) : "l"(a) : "memory");
+    g.p += 2u;
+    return w;
+}
+
 // One decode step of one lane.  valid: the lane's element exists; acc
-// receives the exponent byte at byte position Q; wp: the shared address of
-// the lane's next word.
-template <int Q>
-__device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, uint32_t &wp, bool valid, const uint32_t *table)
+// receives the exponent byte at byte position Q; wp: the address of the
+// lane's next word (next_word).
+template <int Q, class W>
+__device__ __forceinline__ void step(uint32_t &x, uint32_t &acc, W &wp, bool valid, const uint32_t *table)
 {
     if (valid) {
         const uint32_t e = table[x & (kSlots - 1)];
         const uint32_t xh = x >> kProbBits;
         x = (e >> 20) * xh + xh + ((e >> 8) & 0xFFFu);
         acc = __byte_perm(acc, e, (0x3210 & ~(0xF << (4 * Q))) | (4 << (4 * Q)));
-        if (x < kLow) {
-            uint32_t w;
-            asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(wp) : "memory");
-            x = (x << 16) | w;
-            wp += 2u;
-        }
+        if (x < kLow)
+            x = (x << 16) | next_word(wp);
     }
 }
 
 // 16 steps of the last, partial block: elements past n are skipped.
-__device__ __forceinline__ void decode_chunk_tail(uint32_t &x, uint32_t &wp, uint64_t pos0, const uint32_t *table,
+template <class W>
+__device__ __forceinline__ void decode_chunk_tail(uint32_t &x, W &wp, uint64_t pos0, const uint32_t *table,
                                                   const RansParams &p, uint32_t acc[4])
 {
-#define DF11_STEP(I) step<(I) & 3>(x, acc[(I) >> 2], wp, pos0 + (I) < p.n, table)
+#define DF11_STEP(I) step<(I) & 3, W>(x, acc[(I) >> 2], wp, pos0 + (I) < p.n, table)
     DF11_STEP(0); DF11_STEP(1); DF11_STEP(2); DF11_STEP(3);
     DF11_STEP(4); DF11_STEP(5); DF11_STEP(6); DF11_STEP(7);
     DF11_STEP(8); DF11_STEP(9); DF11_STEP(10); DF11_STEP(11);
@@ -145,24 +169,68 @@ __device__ __forceinline__ void decode_chunk_full(uint32_t &x, uint32_t &wp, uin
                  : "r"(tbl)
                  : "memory");
 }
+// The same 16 steps for a block whose words stay in global memory (the word
+// load through the read-only path, its address clamped to the array's last
+// word: a lane of inconsistent data may read up to 16 words per chunk past
+// its stream, and global memory has no slack).
+#define DF11_RSTEP_G(A, SEL)                     \
+    "and.b32 ts, %0, 4095;\n\t"                  \
+    "shl.b32 ts, ts, 2;\n\t"                     \
+    "add.u32 ts, ts, %6;\n\t"                    \
+    "ld.shared.u32 te, [ts];\n\t"                \
+    "shr.u32 th, %0, 12;\n\t"                    \
+    "shr.u32 tf, te, 20;\n\t"                    \
+    "bfe.u32 to, te, 8, 12;\n\t"                 \
+    "mad.lo.u32 %0, tf, th, th;\n\t"             \
+    "add.u32 %0, %0, to;\n\t"                    \
+    "prmt.b32 " A ", " A ", te, " SEL ";\n\t"    \
+    "setp.lt.u32 tp, %0, 65536;\n\t"             \
+    "@tp min.u64 ta, %1, %7;\n\t"                \
+    "@tp ld.global.nc.u16 tw, [ta];\n\t"         \
+    "@tp prmt.b32 %0, tw, %0, 0x5410;\n\t"       \
+    "@tp add.u64 %1, %1, 2;\n\t"
+#define DF11_RSTEP4_G(A) \
+    DF11_RSTEP_G(A, "0x3214") DF11_RSTEP_G(A, "0x3240") DF11_RSTEP_G(A, "0x3410") DF11_RSTEP_G(A, "0x4210")
+
+__device__ __forceinline__ void decode_chunk_full(uint32_t &x, GlobalWords &g, uint32_t tbl, uint32_t acc[4])
+{
+    asm volatile("{\n\t.reg .b32 ts, te, th, tf, to, tw;\n\t.reg .b64 ta;\n\t.reg .pred tp;\n\t"
+                 DF11_RSTEP4_G("%2") DF11_RSTEP4_G("%3") DF11_RSTEP4_G("%4") DF11_RSTEP4_G("%5")
+                 "}"
+                 : "+r"(x), "+l"(g.p), "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
+                 : "r"(tbl), "l"(g.last)
+                 : "memory");
+}
+#undef DF11_RSTEP4_G
+#undef DF11_RSTEP_G
 #undef DF11_RSTEP4
 #undef DF11_RSTEP
 
 // Asynchronous copy (cp.async) of a block's words [bw0, bw1) into a warp
 // buffer at shared address buf: from the 16-byte boundary at or below bw0 to
 // the one at or above bw1 (inside the array's 8-word padding), one commit
-// group.  Returns the index of the buffer's first word.
+// group.  A block spanning more than cap words from that boundary (big(), and
+// inconsistent offsets) is not copied: its words are asked into L2 and read
+// from global memory.  Returns the index of the buffer's first word.
+__device__ __forceinline__ bool big_block(const RansParams &p, uint32_t bw1, uint32_t w0) { return bw1 - w0 > p.cap; }
+
+template <bool BIG>
 __device__ __forceinline__ uint32_t copy_words(const RansParams &p, uint32_t bw0, uint32_t bw1, int lane,
                                                uint32_t buf)
 {
     const uint32_t w0 = bw0 & ~7u;
     uint32_t w1 = (bw1 + 7u) & ~7u;
-    // inconsistent offsets: copy what fits the buffer and the array
     w1 = w1 < p.words_end ? w1 : p.words_end;
-    const uint32_t w1c = w1 <= w0 ? w0 : (w1 - w0 <= p.cap ? w1 : w0 + p.cap);
-    for (uint32_t o = 8u * (uint32_t)lane; w0 + o < w1c; o += 256u)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(buf + 2u * o), "l"(p.words + w0 + o)
-                     : "memory");
+    if (!BIG || !big_block(p, bw1, w0)) {
+        // (without BIG, inconsistent offsets: what fits the buffer)
+        const uint32_t w1c = w1 <= w0 ? w0 : (w1 - w0 <= p.cap ? w1 : w0 + p.cap);
+        for (uint32_t o = 8u * (uint32_t)lane; w0 + o < w1c; o += 256u)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(buf + 2u * o), "l"(p.words + w0 + o)
+                         : "memory");
+    } else if (lane == 0 && w1 > w0) {
+        const uint32_t bytes = w1 - w0 < 32768u ? 2u * (w1 - w0) : 65536u;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.words + w0), "r"(bytes) : "memory");
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
     return w0;
 }
@@ -175,8 +243,10 @@ __device__ __forceinline__ uint4 load_sm(const RansParams &p, uint64_t pos)
 
 // DYN: blocks as contiguous ranges per CTA handed out by a shared-memory
 // counter; otherwise strided over the stream (balanced when the last round
-// is nearly full).
-template <bool DYN>
+// is nearly full).  BIG: the stream has blocks larger than the warp buffers
+// (they read their words from global memory); without it such a block is
+// inconsistent data.
+template <bool DYN, bool BIG>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const RansParams p)
 {
     __shared__ uint32_t table[kSlots];
@@ -266,7 +336,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         c_n = __ldg(p.lane_words + 32ull * b + lane);
         bw0_n = __ldg(p.block_word + b);
         bw1_n = __ldg(p.block_word + b + 1);
-        wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s);
+        wfirst = copy_words<BIG>(p, bw0_n, bw1_n, lane, wbuf_s);
         s_n = load_sm(p, b * B + 16u * (uint32_t)lane);
     }
     uint32_t nb = 0;
@@ -287,8 +357,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
         const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
         const uint32_t first = (bw0_n - wfirst) + (incl - c_n);  // bw0 - wfirst = bw0 mod 8
         const uint32_t end = first + c_n;                          // words, from the buffer's start
-        bool bad = total != bw1_n - bw0_n || bw1_n - wfirst > p.cap;
+        const bool big = BIG && big_block(p, bw1_n, wfirst);  // warp-uniform: words in global memory
+        bool bad = total != bw1_n - bw0_n || (!BIG && big_block(p, bw1_n, wfirst));
         uint32_t wp = wb_s + 2u * (first < p.cap ? first : p.cap);  // clamped: inconsistent counts
+        // big block: the lane's stream in global memory (every load clamped
+        // to the array, next_word)
+        const uint64_t gfirst = (uint64_t)wfirst + first, wbase = reinterpret_cast<uint64_t>(p.words);
+        GlobalWords wg{wbase + 2u * (gfirst < p.words_end ? gfirst : p.words_end), wbase + 2u * (p.words_end - 1u)};
+        const uint64_t wg_end = wbase + 2u * ((uint64_t)wfirst + end);
         const bool full = (b + 1) * B <= p.n;  // warp-uniform
         nb = take_next();
         if (nb < b_end) {
@@ -296,7 +372,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
             c_n = __ldg(p.lane_words + 32ull * nb + lane);
             bw0_n = __ldg(p.block_word + nb);
             bw1_n = __ldg(p.block_word + nb + 1);
-            wfirst = copy_words(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.bufw * (k ^ 1u));
+            wfirst = copy_words<BIG>(p, bw0_n, bw1_n, lane, wbuf_s + 2u * p.bufw * (k ^ 1u));
             const uint64_t s0 = nb * B, s1 = s0 + B < p.n ? s0 + B : p.n;
             if (lane == 0)
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.sm + s0),
@@ -309,10 +385,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
             s_n = load_sm(p, j + 1 < p.chunks ? pos0 + 512
                                               : (!DYN || nb < b_end ? (uint64_t)nb * B + 16u * (uint32_t)lane : p.n));
             uint32_t acc[4] = {0u, 0u, 0u, 0u};
-            if (full)
-                decode_chunk_full(x, wp, tbl, acc);
-            else
-                decode_chunk_tail(x, wp, pos0, table, p, acc);
+            if (!BIG || !big) {
+                if (full)
+                    decode_chunk_full(x, wp, tbl, acc);
+                else
+                    decode_chunk_tail(x, wp, pos0, table, p, acc);
+            } else {
+                if (full)
+                    decode_chunk_full(x, wg, tbl, acc);
+                else
+                    decode_chunk_tail(x, wg, pos0, table, p, acc);
+            }
             // merge with the 16 sign/mantissa bytes and store
             if (pos0 + 16 <= p.n) {
                 uint32_t r[8];
@@ -337,7 +420,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
                         p.dst[pos0 + i] = merge1(p.sm[pos0 + i], (acc[i >> 2] >> (8 * (i & 3))) & 0xFFu);
             }
         }
-        bad = bad || x != kLow || wp != wb_s + 2u * end;
+        bad = bad || x != kLow || (big ? wg.p != wg_end : wp != wb_s + 2u * end);
         if (__any_sync(0xffffffffu, bad) && lane == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
         __syncwarp();  // every lane is done with this buffer before it is refilled
@@ -347,7 +430,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rans_decode_kernel(const Ra
 std::mutex g_rans_mu;
 int g_rans_sms[64] = {0};
 int g_rans_optin[64] = {0};
-uint32_t g_rans_granted[2][64] = {};
+uint32_t g_rans_granted[4][64] = {};  // [DYN + 2 BIG][device]
 
 }  // namespace
 
@@ -394,11 +477,18 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     p.num_blocks = a->num_blocks;
     p.chunks = a->chunks;
     p.wide = (reinterpret_cast<uintptr_t>(dst) & 31) == 0;
-    p.cap = ((a->max_block_words + 16u) + 7u) & ~7u;
     p.words_end = (uint32_t)((a->num_words & ~7ull) + 8);
-    // two buffers of cap words per warp; as many warps as shared memory holds
-    p.bufw = p.cap + 16u * p.chunks + 8u;  // a lane reads at most 16 words per chunk past its clamped start
-    const uint64_t per_warp = 4ull * p.bufw, room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
+    // two buffers per warp of cap words plus the slack a lane's reads past
+    // its clamped start need (16 words per chunk); cap holds the largest
+    // block unless that leaves room for fewer than 32 warps: then the few
+    // larger blocks read their words from global memory
+    const uint32_t slack = 16u * p.chunks + 8u;
+    const uint64_t room = (uint64_t)optin - sizeof(uint32_t) * (kSlots + 257) - 1024;
+    const uint64_t cap_all = ((uint64_t)a->max_block_words + 16u + 7u) & ~7ull;
+    const uint64_t cap_32 = room / (4ull * kMaxWarps) > slack + 256u ? (room / (4ull * kMaxWarps) - slack) & ~7ull : 256u;
+    p.cap = (uint32_t)(cap_all < cap_32 ? cap_all : cap_32);
+    p.bufw = p.cap + slack;
+    const uint64_t per_warp = 4ull * p.bufw;
     const uint64_t warps = room / per_warp < (uint64_t)kMaxWarps ? room / per_warp : (uint64_t)kMaxWarps;
     if (warps == 0)
         return DF11_ERR_INVALID_ARG;  // cannot happen for chunks <= 64 (at most 24,576 words per block)
@@ -409,13 +499,17 @@ extern "C" df11_status df11_rans_decompress(const df11_rans_arrays *a, uint16_t 
     // striding when its last round is at least 85 % full, else ranges per CTA
     const uint64_t W = (uint64_t)grid * warps, rem = a->num_blocks % W;
     const int di = (rem != 0 && rem * 100 < W * 85) ? 1 : 0;
-    auto kern = di ? rans_decode_kernel<true> : rans_decode_kernel<false>;
+    const bool big = cap_all > p.cap;
+    static void (*const kernels[4])(RansParams) = {rans_decode_kernel<false, false>, rans_decode_kernel<true, false>,
+                                                   rans_decode_kernel<false, true>, rans_decode_kernel<true, true>};
+    const int ki = di + (big ? 2 : 0);
+    auto kern = kernels[ki];
     {
         std::lock_guard<std::mutex> lock(g_rans_mu);
-        if (dyn > g_rans_granted[di][dev]) {
+        if (dyn > g_rans_granted[ki][dev]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
                 return DF11_ERR_CUDA;
-            g_rans_granted[di][dev] = (uint32_t)dyn;
+            g_rans_granted[ki][dev] = (uint32_t)dyn;
         }
     }
     kern<<<grid, (uint32_t)(warps * 32), (size_t)dyn, reinterpret_cast<cudaStream_t>(stream)>>>(p);

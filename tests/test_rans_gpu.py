@@ -120,6 +120,54 @@ def test_inconsistent_offsets_and_states_stay_in_bounds():
         assert np.array_equal(got[:2 * 4096], w[:2 * 4096])
 
 
+def _with_high_entropy_runs(seed):
+    # Gaussian weights with runs of uniformly random bit patterns (every
+    # exponent about equally likely, ~8 bits each): blocks of those runs need
+    # ~2,600 words, more than a warp buffer holds at 32 warps per CTA, and
+    # take the decoder's global-memory path; the stream ends inside such a run
+    rng = np.random.default_rng(seed)
+    parts = [inputs.gaussian(100_000, [seed, 1]), rng.integers(0, 1 << 16, 30_000, dtype=np.uint32).astype(np.uint16),
+             inputs.gaussian(50_000, [seed, 2]), rng.integers(0, 1 << 16, 7_001, dtype=np.uint32).astype(np.uint16)]
+    return np.concatenate(parts)
+
+
+def test_blocks_larger_than_the_word_buffer():
+    w = _with_high_entropy_runs(107)
+    fmt = df11.rans_build_format(w)
+    assert fmt.scalars()["max_block_words"] > 2400
+    assert np.array_equal(gpu_decode(w), w)
+
+
+def test_inconsistent_large_blocks_stay_in_bounds():
+    # lane counts that do not match, on blocks read from global memory: each
+    # lane's start is clamped so that its reads stay inside the word array,
+    # and the launch reports the block as corrupt
+    torch = torch_cuda()
+    w = _with_high_entropy_runs(108)
+    fmt = df11.rans_build_format(w)
+    bw = np.diff(fmt.arrays()["block_word"].astype(np.int64))
+    big = int(np.argmax(bw))
+    assert bw[big] > 2400
+
+    def lane_counts_off(t):
+        t[32 * big] = 255
+        t[32 * big + 1] = 0
+
+    def states_off(t):
+        t.view(torch.int32)[32 * big: 32 * big + 32] = 0
+
+    for name, edit in (("lane_words", lane_counts_off), ("states", states_off)):
+        dev = df11.RansDeviceFormat(fmt, "cuda")
+        edit(dev.tensors[name])
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = df11.rans_decompress(dev, None, status)
+        torch.cuda.synchronize()
+        assert df11.read_status(status) != 0, name
+        got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+        B = 5120
+        assert np.array_equal(got[:B * big], w[:B * big])
+
+
 def test_repeated_launches_are_identical():
     torch = torch_cuda()
     w = inputs.gaussian(1 << 20, [105])
