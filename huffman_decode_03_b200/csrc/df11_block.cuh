@@ -218,6 +218,77 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         : "memory");
 }
 
+// The byte-store form of the decode loop (the fused matrix-vector and GEMM
+// kernels, whose other work keeps the ALU busier than the L1): symbol-table
+// entry as stored (table_entry): up to three rotated exponents in bytes
+// 0..2, their total length in bits 24..28, their number in bits 29..30
+// (0 = a code longer than 12 bits).
+// A chain is active while pos < pend and its last entry was not 0; the bits
+// of its window past pend are zeros.  Per lookup: the three exponent bytes go
+// to the chain's staging slot at q unconditionally (bytes past the codes
+// found are overwritten by the next lookup or never read), q advances by the
+// count, the window and pos by the length.  (entry >> 24) serves as the
+// funnel-shift amount directly: wrap mode reads only its low five bits.  An
+// entry of 0 changes nothing and stops its chain: the caller resolves that
+// long code, resets the chain's entry to non-zero and calls again.
+__device__ __forceinline__ void decode_bulk2_bytes(uint32_t &hA, uint32_t &mA, uint32_t &lA, uint32_t &qA, int &posA,
+                                             uint32_t &eA, uint32_t &hB, uint32_t &mB, uint32_t &lB, uint32_t &qB,
+                                             int &posB, uint32_t &eB, int pendA, int pendB, uint32_t sym_base)
+{
+    asm volatile(
+        "{\n\t"
+        ".reg .pred pa, pb, pz;\n\t"
+        ".reg .u32 ca, cb, t;\n\t"
+        "DC_TOP:\n\t"
+        "setp.lt.s32 pa, %4, %12;\n\t"
+        "setp.lt.s32 pb, %10, %13;\n\t"
+        "setp.ne.and.u32 pa, %5, 0, pa;\n\t"
+        "setp.ne.and.u32 pb, %11, 0, pb;\n\t"
+        "or.pred pz, pa, pb;\n\t"
+        "@!pz bra DC_END;\n\t"
+        "@pa shr.u32 %5, %0, 20;\n\t"
+        "@pb shr.u32 %11, %6, 20;\n\t"
+        "@pa mad.lo.u32 %5, %5, 4, %14;\n\t"
+        "@pb mad.lo.u32 %11, %11, 4, %14;\n\t"
+        "@pa ld.shared.u32 %5, [%5];\n\t"
+        "@pb ld.shared.u32 %11, [%11];\n\t"
+        // chain A
+        "@pa st.shared.u8 [%3], %5;\n\t"
+        "@pa mul.hi.u32 t, %5, 16777216;\n\t"
+        "@pa st.shared.u8 [%3+1], t;\n\t"
+        "@pa mul.hi.u32 t, %5, 65536;\n\t"
+        "@pa st.shared.u8 [%3+2], t;\n\t"
+        "@pa shr.u32 ca, %5, 24;\n\t"
+        "@pa mul.hi.u32 t, %5, 8;\n\t"
+        "@pa add.u32 %3, %3, t;\n\t"
+        "@pa and.b32 t, ca, 31;\n\t"
+        "@pa add.s32 %4, %4, t;\n\t"
+        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
+        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
+        "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
+        // chain B
+        "@pb st.shared.u8 [%9], %11;\n\t"
+        "@pb mul.hi.u32 t, %11, 16777216;\n\t"
+        "@pb st.shared.u8 [%9+1], t;\n\t"
+        "@pb mul.hi.u32 t, %11, 65536;\n\t"
+        "@pb st.shared.u8 [%9+2], t;\n\t"
+        "@pb shr.u32 cb, %11, 24;\n\t"
+        "@pb mul.hi.u32 t, %11, 8;\n\t"
+        "@pb add.u32 %9, %9, t;\n\t"
+        "@pb and.b32 t, cb, 31;\n\t"
+        "@pb add.s32 %10, %10, t;\n\t"
+        "@pb shf.l.wrap.b32 %6, %7, %6, cb;\n\t"
+        "@pb shf.l.wrap.b32 %7, %8, %7, cb;\n\t"
+        "@pb shf.l.wrap.b32 %8, 0, %8, cb;\n\t"
+        "bra DC_TOP;\n\t"
+        "DC_END:\n\t"
+        "}"
+        : "+r"(hA), "+r"(mA), "+r"(lA), "+r"(qA), "+r"(posA), "+r"(eA), "+r"(hB), "+r"(mB), "+r"(lB), "+r"(qB),
+          "+r"(posB), "+r"(eB)
+        : "r"(pendA), "r"(pendB), "r"(sym_base)
+        : "memory");
+}
+
 // Adds one exponent (rotated) to a chain's pending word; the long-code path.
 __device__ __forceinline__ void chain_put1(Chain &c, uint32_t sym)
 {
@@ -391,17 +462,19 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
 
 // A symbol-table entry (df11_symtab::table_entry: exponents in bytes 0..2,
 // total length in bits 24..28, count in bits 29..30) in the decode loop's
-// shared-memory form: count in bits 0..1, length in bits 2..6, the count's
-// exponents from bit 8 on, the bytes past them zero.  *bad when no code set
+// shared-memory form, the bytes past the count's exponents zero: with WORDS
+// (the pending-word loop) count in bits 0..1, length in bits 2..6, the
+// exponents from bit 8 on; else as stored.  *bad when no code set
 // with codes of >= min_bits bits each produces the entry (more than 3
 // codes, more than 12 bits, fewer than min_bits x count bits, or a length
 // without codes).
+template <bool WORDS>
 __device__ __forceinline__ uint32_t table_word(uint32_t e, uint32_t min_bits, bool &bad)
 {
     const uint32_t n = e >> 29, bits = (e >> 24) & 31u;
     bad |= n > 3u || bits > (uint32_t)kIdxBits || bits < n * min_bits || (n == 0 && bits != 0);
     const uint32_t syms = n >= 3u ? e & 0xFFFFFFu : e & ((1u << (8u * n)) - 1u);
-    return (n & 3u) | ((bits & 31u) << 2) | (syms << 8);
+    return WORDS ? (n & 3u) | ((bits & 31u) << 2) | (syms << 8) : syms | (bits << 24) | (n << 29);
 }
 
 // Once per CTA, called by all its nthreads threads (tid = thread index): the
@@ -411,6 +484,7 @@ __device__ __forceinline__ uint32_t table_word(uint32_t e, uint32_t min_bits, bo
 // Returns false (every thread alike) when the symbol table, stored or
 // derived, has an entry no such code set produces (table_word): the decode
 // loop's slot bound relies on every code taking at least min_bits bits.
+template <bool WORDS>
 __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_t *cl_g, uint32_t num_luts,
                                              const uint32_t *sym_g, uint8_t *smem, uint32_t tid, uint32_t nthreads,
                                              uint32_t min_bits)
@@ -430,8 +504,9 @@ __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_
         // and checked
         for (uint32_t i = tid; i < kIdxEntries / 4; i += nthreads) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(sym_g) + i);
-            reinterpret_cast<uint4 *>(sym_tab)[i] = make_uint4(table_word(v.x, min_bits, bad), table_word(v.y, min_bits, bad),
-                                                             table_word(v.z, min_bits, bad), table_word(v.w, min_bits, bad));
+            reinterpret_cast<uint4 *>(sym_tab)[i] =
+                make_uint4(table_word<WORDS>(v.x, min_bits, bad), table_word<WORDS>(v.y, min_bits, bad),
+                           table_word<WORDS>(v.z, min_bits, bad), table_word<WORDS>(v.w, min_bits, bad));
         }
     } else {
         __syncthreads();
@@ -442,7 +517,7 @@ __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_
             first_code[i] = df11_symtab::first_code(i, luts, cl, num_luts);
         __syncthreads();
         for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
-            sym_tab[i] = table_word(df11_symtab::table_entry(i, first_code), min_bits, bad);
+            sym_tab[i] = table_word<WORDS>(df11_symtab::table_entry(i, first_code), min_bits, bad);
     }
     if (__syncthreads_or(bad))
         return false;
@@ -471,11 +546,13 @@ struct BlockOut {
 // Decodes format block b (its registers in cur, loaded by load_block) into
 // the warp's write buffer at shared address exp_base, through the lane's
 // staging slots at slot_base; sym_base: the shared address of the symbol
-// table (and of the tables after it).  Asks L2 for the block's
+// table (and of the tables after it), in the form build_tables<WORDS> made.
+// WORDS: the pending-word loop (decode_bulk2), else the byte-store loop
+// (decode_bulk2_bytes).  Asks L2 for the block's
 // sign/mantissa bytes first.  Returns false, after setting DF11_ERR_CORRUPT
 // in *p.status, when the block is inconsistent (nothing placed).  Called by
 // all 32 lanes of the warp.
-template <int C, uint32_t SLOT, class P>
+template <int C, uint32_t SLOT, bool WORDS, class P>
 __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, const BlockRegs<C> &cur,
                                              uint32_t sym_base, uint32_t exp_base, uint32_t slot_base, BlockOut &out)
 {
@@ -537,7 +614,7 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
     // are such zero codes: pos overshoots pend by a multiple of lmin
     // (< 12) and the count by overshoot / lmin.
     uint32_t cnt[2];
-    {
+    if constexpr (WORDS) {
         Chain ch[2];
 #pragma unroll
         for (int k = 0; k < 2; k++) {
@@ -579,6 +656,44 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
             const uint32_t z = ld_u8(zq + (d & 15u));
             bad |= d > 15u || !(z & 0x80u);
             cnt[k] = bytes - (z & 0x7Fu);
+        }
+    } else {
+        uint32_t q[2], q0[2], e[2] = {1u, 1u};
+        int pos[2];
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            q0[k] = slot_base + k * (32 * SLOT);
+            q[k] = q0[k];
+            pos[k] = pos0[k];
+        }
+        for (;;) {  // each pass resolves >= 1 code or ends both chains
+            decode_bulk2_bytes(h[0], m[0], l[0], q[0], pos[0], e[0], h[1], m[1], l[1], q[1], pos[1], e[1], pend[0],
+                               pend[1], sym_base);
+            bool any_long = false;
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                if (pos[k] < pend[k]) {
+                    const uint32_t d = lut_decode(h[k], luts, cl, p.num_luts, &bad);
+                    uint32_t len = d >> 8;
+                    bad |= len <= (uint32_t)kIdxBits;
+                    len = len > (uint32_t)kIdxBits ? len : (uint32_t)kIdxBits + 1u;
+                    st_u8(q[k], ror8(d & 0xFFu));
+                    q[k] += 1;
+                    pos[k] += (int)len;
+                    shift_window(h[k], m[k], l[k], len);
+                    e[k] = 1u;
+                    any_long = true;
+                }
+            }
+            if (!any_long)
+                break;
+        }
+#pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const uint32_t d = (uint32_t)(pos[k] - pend[k]);  // >= 0
+            const uint32_t z = ld_u8(zq + (d & 15u));
+            bad |= d > 15u || !(z & 0x80u);
+            cnt[k] = q[k] - q0[k] - (z & 0x7Fu);
         }
     }
 

@@ -368,6 +368,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     static_assert(C == 1 || C == 2, "one or two chains per lane");
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
     constexpr bool kCopy = SLOT == kSlotShort;  // metadata by cp.async
+    // the pending-word decode loop where the L1 is the busier unit (the
+    // rebuild to memory), the byte-store loop where the ALU is (the fused
+    // matrix-vector product)
+    constexpr bool kWords = MODE == 0;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *exp_s = smem + Smem::bufs + warp * warp_bytes<C, SLOT>(p.cap);
@@ -393,7 +397,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (!kCopy && b < b_end)
         load_block<C>(p, b, lane, cur);
 
-    if (!build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
+    if (!build_tables<kWords>(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
                       SLOT < kSlotLong ? 2u : 1u)) {
         if (tid == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             load_block<C>(p, nb, lane, nxt);
         }
         BlockOut bo;
-        if (decode_block<C, SLOT>(p, b, lane, cur, sym_base, exp_base, slot_base, bo)) {
+        if (decode_block<C, SLOT, kWords>(p, b, lane, cur, sym_base, exp_base, slot_base, bo)) {
             // ---- merge with sign/mantissa (from L2)
             const uint64_t g0 = bo.g0;
             const uint32_t lo_off = bo.lo_off, hi = bo.hi;

@@ -484,7 +484,7 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
             const uint64_t o0 = cur.o0, o1 = cur.o1 > cur.o0 ? cur.o1 : cur.o0;
             const uint64_t r0 = o0 > e0 ? o0 : e0, r1 = o1 < e1 ? o1 : e1;
             BlockOut bo;
-            const bool dok = decode_block<C, SLOT>(p, b, lane, cur, sym_base, exp_base, slot_base, bo);
+            const bool dok = decode_block<C, SLOT, false>(p, b, lane, cur, sym_base, exp_base, slot_base, bo);
             if (r0 < r1) {
                 const uint32_t t_first = (uint32_t)((r0 - e0) >> kTileShift);
                 const uint32_t t_last = (uint32_t)((r1 - 1 - e0) >> kTileShift);
@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(gemm_threads(DW), 1) df11_gemm_kernel(const Ge
     }
     // the tables (the barriers, flags and tensor-memory address above are
     // published by its __syncthreads)
-    const bool tables_ok = build_tables(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW),
+    const bool tables_ok = build_tables<false>(p.luts, p.cl, p.num_luts, p.sym_table, smem, tid, gemm_threads(DW),
                                         SLOT < kSlotLong ? 2u : 1u);
     tc_fence_after();
     R.tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
