@@ -337,46 +337,26 @@ __device__ __forceinline__ void load_block(const P &p, uint32_t b, int lane, Blo
 // aligned, len[k] bytes) to the write buffer at shared address dst[k]: the up
 // to three bytes before dst's first word boundary and after its last one
 // singly (those words are shared with neighbouring chains), the words in
-// between as 32-bit stores assembled by funnel shifts; both chains step
-// through one loop.
-__device__ __forceinline__ void copy_slots2(const uint32_t dst0[2], const uint32_t src0[2], const uint32_t len0[2])
+// between as 32-bit stores assembled by funnel shifts.  The path of blocks
+// with a chain of fewer than 3 codes, so the chains go one after the other
+// (few registers) rather than fast.
+__device__ __noinline__ void copy_slots2(const uint32_t dst0[2], const uint32_t src0[2], const uint32_t len0[2])
 {
-    uint32_t dst[2], src[2], nw[2], sh[2], sa[2], cur[2], tail[2];
-#pragma unroll
     for (int k = 0; k < 2; k++) {
         uint32_t head = (4u - (dst0[k] & 3u)) & 3u;
         head = head < len0[k] ? head : len0[k];
-#pragma unroll
-        for (uint32_t i = 0; i < 3; i++)
-            if (i < head)
-                st_u8(dst0[k] + i, ld_u8(src0[k] + i));
-        dst[k] = dst0[k] + head;
-        src[k] = src0[k] + head;
-        const uint32_t len = len0[k] - head;
-        nw[k] = len >> 2;
-        tail[k] = len & 3u;
-        sh[k] = 8u * (src[k] & 3u);
-        sa[k] = src[k] & ~3u;
-        cur[k] = ld_u32(sa[k]);
-    }
-    const uint32_t nmax = nw[0] > nw[1] ? nw[0] : nw[1];
-    for (uint32_t w = 0; w < nmax; w++) {
-#pragma unroll
-        for (int k = 0; k < 2; k++) {
-            if (w < nw[k]) {
-                const uint32_t nxt = ld_u32(sa[k] + 4 * w + 4);
-                st_u32(dst[k] + 4 * w, __funnelshift_r(cur[k], nxt, sh[k]));
-                cur[k] = nxt;
-            }
+        for (uint32_t i = 0; i < head; i++)
+            st_u8(dst0[k] + i, ld_u8(src0[k] + i));
+        const uint32_t dst = dst0[k] + head, src = src0[k] + head, len = len0[k] - head;
+        const uint32_t nw = len >> 2, sh = 8u * (src & 3u), sa = src & ~3u;
+        uint32_t cur = ld_u32(sa);
+        for (uint32_t w = 0; w < nw; w++) {
+            const uint32_t nxt = ld_u32(sa + 4 * w + 4);
+            st_u32(dst + 4 * w, __funnelshift_r(cur, nxt, sh));
+            cur = nxt;
         }
-    }
-#pragma unroll
-    for (int k = 0; k < 2; k++) {
-        const uint32_t o = 4 * nw[k];
-#pragma unroll
-        for (uint32_t i = 0; i < 3; i++)
-            if (i < tail[k])
-                st_u8(dst[k] + o + i, ld_u8(src[k] + o + i));
+        for (uint32_t i = 4 * nw; i < len; i++)
+            st_u8(dst + i, ld_u8(src + i));
     }
 }
 
