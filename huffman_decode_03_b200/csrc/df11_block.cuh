@@ -340,8 +340,11 @@ __device__ __forceinline__ void load_block(const P &p, uint32_t b, int lane, Blo
 // between as 32-bit stores assembled by funnel shifts.  The path of blocks
 // with a chain of fewer than 3 codes, so the chains go one after the other
 // (few registers) rather than fast.
-__device__ __noinline__ void copy_slots2(const uint32_t dst0[2], const uint32_t src0[2], const uint32_t len0[2])
+__device__ __noinline__ void copy_slots2(uint32_t dA, uint32_t dB, uint32_t sA, uint32_t sB, uint32_t nA, uint32_t nB)
 {
+    // scalar arguments: arrays would be passed through local memory
+    const uint32_t dst0[2] = {dA, dB}, src0[2] = {sA, sB}, len0[2] = {nA, nB};
+#pragma unroll
     for (int k = 0; k < 2; k++) {
         uint32_t head = (4u - (dst0[k] & 3u)) & 3u;
         head = head < len0[k] ? head : len0[k];
@@ -718,8 +721,7 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
             const uint32_t offs2[2] = {lo_off + first[0], lo_off + first[1]};
             place_words<C, SLOT>(exp_base, offs2, srcs, cnt, lane);
         } else {
-            const uint32_t dsts[2] = {exp_base + lo_off + first[0], exp_base + lo_off + first[1]};
-            copy_slots2(dsts, srcs, cnt);
+            copy_slots2(exp_base + lo_off + first[0], exp_base + lo_off + first[1], srcs[0], srcs[1], cnt[0], cnt[1]);
         }
     }
     __syncwarp();
