@@ -158,15 +158,13 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
 {
     asm volatile(
         "{\n\t"
-        ".reg .pred pa, pb, ka, kb, pz, po;\n\t"
+        ".reg .pred pa, pb, pz, po;\n\t"
         ".reg .u32 ea, eb, ca, t;\n\t"
-        "setp.eq.u32 ka, 0, 0;\n\t"
-        "setp.eq.u32 kb, 0, 0;\n\t"
-        "DB_TOP:\n\t"
-        "setp.gt.and.s32 pa, %3, 0, ka;\n\t"
-        "setp.gt.and.s32 pb, %10, 0, kb;\n\t"
+        "setp.gt.s32 pa, %3, 0;\n\t"
+        "setp.gt.s32 pb, %10, 0;\n\t"
         "or.pred pz, pa, pb;\n\t"
         "@!pz bra DB_END;\n\t"
+        "DB_TOP:\n\t"
         "@pa shr.u32 ea, %0, 20;\n\t"
         "@pb shr.u32 eb, %7, 20;\n\t"
         "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"
@@ -180,7 +178,6 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
-        "@pa setp.ne.u32 ka, ea, 0;\n\t"
         "@pa shr.u32 t, ea, 8;\n\t"
         "@pa mul.hi.u32 ca, t, %6;\n\t"
         "@pa mad.lo.u32 t, t, %6, %5;\n\t"
@@ -198,7 +195,6 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@pb shf.l.wrap.b32 %7, %8, %7, ca;\n\t"
         "@pb shf.l.wrap.b32 %8, %9, %8, ca;\n\t"
         "@pb shf.l.wrap.b32 %9, 0, %9, ca;\n\t"
-        "@pb setp.ne.u32 kb, eb, 0;\n\t"
         "@pb shr.u32 t, eb, 8;\n\t"
         "@pb mul.hi.u32 ca, t, %13;\n\t"
         "@pb mad.lo.u32 t, t, %13, %12;\n\t"
@@ -209,7 +205,14 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@po st.shared.u32 [%11], t;\n\t"
         "@po add.u32 %11, %11, 4;\n\t"
         "@pb selp.b32 %12, ca, t, po;\n\t"
-        "bra DB_TOP;\n\t"
+        // a chain stays active while bits are left and its entry was not 0
+        // (a stopped chain keeps its 0 entry: no load refreshes it)
+        "setp.gt.s32 pa, %3, 0;\n\t"
+        "setp.ne.and.u32 pa, ea, 0, pa;\n\t"
+        "setp.gt.s32 pb, %10, 0;\n\t"
+        "setp.ne.and.u32 pb, eb, 0, pb;\n\t"
+        "or.pred pz, pa, pb;\n\t"
+        "@pz bra DB_TOP;\n\t"
         "DB_END:\n\t"
         "}"
         : "+r"(A.h), "+r"(A.m), "+r"(A.l), "+r"(A.rem), "+r"(A.qa), "+r"(A.w), "+r"(A.mul), "+r"(B.h), "+r"(B.m),
