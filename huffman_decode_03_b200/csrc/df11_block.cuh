@@ -135,17 +135,19 @@ struct SharedBytes {
 
 // Decode loop for two chains (A, B) of one lane, in PTX.  Shared-memory
 // table entry (table_word): number of codes in bits 0..1, their total length
-// in bits 2..6, their rotated exponents in bits 8..31 (bytes past the count
-// zero); 0 = a code longer than 12 bits.  A chain is active while rem (its
-// bits left before pend) is > 0 and its last entry was not 0; the bits of its
-// window past pend are zeros.  Per lookup the window advances and rem drops
-// by the length ((entry >> 2) serves as the funnel-shift amount directly:
-// wrap mode reads only its low five bits) and the exponents are added to the
+// in bits 2..6, their rotated exponents in bits 7..30 (bytes past the count
+// zero); 2^31 = a code longer than 12 bits.  A chain is active while rem
+// (its bits left before pend) is > 0; the bits of its window past pend are
+// zeros.  Per lookup the window advances and rem drops by the length
+// ((entry >> 2) serves as the funnel-shift amount directly: wrap mode reads
+// only its low five bits; masked with bit 31 kept, the long-code entry takes
+// 2^31 from rem, which ends the chain) and the exponents are added to the
 // chain's pending word w at byte n, where mul = 2^(8 n); mul rotates left by
 // 8 x count bits.  When the pending word fills (the rotation wraps, mul
 // decreases) it is stored at the slot address qa, qa advances one word and w
-// keeps the bytes that spilled past it.  An entry of 0 changes nothing and
-// stops its chain: the caller resolves that long code and calls again.
+// keeps the bytes that spilled past it.  The long-code entry moves nothing
+// but adds 2^24 x mul to w; the caller undoes both, resolves that code and
+// calls again.
 struct Chain {
     uint32_t h, m, l;  // 96-bit window, next bit at the top of h
     int rem;           // pend - bits consumed
@@ -172,13 +174,13 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@pa ld.shared.u32 ea, [ea];\n\t"
         "@pb ld.shared.u32 eb, [eb];\n\t"
         // chain A
-        "@pa shr.u32 ca, ea, 2;\n\t"
-        "@pa and.b32 t, ca, 31;\n\t"
+        "@pa shr.s32 ca, ea, 2;\n\t"
+        "@pa and.b32 t, ca, 0x8000001F;\n\t"
         "@pa sub.s32 %3, %3, t;\n\t"
         "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
         "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
         "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
-        "@pa shr.u32 t, ea, 8;\n\t"
+        "@pa shr.u32 t, ea, 7;\n\t"
         "@pa mul.hi.u32 ca, t, %6;\n\t"
         "@pa mad.lo.u32 t, t, %6, %5;\n\t"
         "@pa shl.b32 %5, ea, 3;\n\t"
@@ -189,13 +191,13 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@po add.u32 %4, %4, 4;\n\t"
         "@pa selp.b32 %5, ca, t, po;\n\t"
         // chain B
-        "@pb shr.u32 ca, eb, 2;\n\t"
-        "@pb and.b32 t, ca, 31;\n\t"
+        "@pb shr.s32 ca, eb, 2;\n\t"
+        "@pb and.b32 t, ca, 0x8000001F;\n\t"
         "@pb sub.s32 %10, %10, t;\n\t"
         "@pb shf.l.wrap.b32 %7, %8, %7, ca;\n\t"
         "@pb shf.l.wrap.b32 %8, %9, %8, ca;\n\t"
         "@pb shf.l.wrap.b32 %9, 0, %9, ca;\n\t"
-        "@pb shr.u32 t, eb, 8;\n\t"
+        "@pb shr.u32 t, eb, 7;\n\t"
         "@pb mul.hi.u32 ca, t, %13;\n\t"
         "@pb mad.lo.u32 t, t, %13, %12;\n\t"
         "@pb shl.b32 %12, eb, 3;\n\t"
@@ -205,12 +207,10 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "@po st.shared.u32 [%11], t;\n\t"
         "@po add.u32 %11, %11, 4;\n\t"
         "@pb selp.b32 %12, ca, t, po;\n\t"
-        // a chain stays active while bits are left and its entry was not 0
-        // (a stopped chain keeps its 0 entry: no load refreshes it)
+        // a chain stays active while bits are left (a long-code entry took
+        // 2^31 from them)
         "setp.gt.s32 pa, %3, 0;\n\t"
-        "setp.ne.and.u32 pa, ea, 0, pa;\n\t"
         "setp.gt.s32 pb, %10, 0;\n\t"
-        "setp.ne.and.u32 pb, eb, 0, pb;\n\t"
         "or.pred pz, pa, pb;\n\t"
         "@pz bra DB_TOP;\n\t"
         "DB_END:\n\t"
@@ -450,7 +450,8 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
 // total length in bits 24..28, count in bits 29..30) in the decode loop's
 // shared-memory form, the bytes past the count's exponents zero: with WORDS
 // (the pending-word loop) count in bits 0..1, length in bits 2..6, the
-// exponents from bit 8 on; else as stored.  *bad when no code set
+// exponents in bits 7..30, and 2^31 for a code longer than 12 bits; else as
+// stored.  *bad when no code set
 // with codes of >= min_bits bits each produces the entry (more than 3
 // codes, more than 12 bits, fewer than min_bits x count bits, or a length
 // without codes).
@@ -460,7 +461,9 @@ __device__ __forceinline__ uint32_t table_word(uint32_t e, uint32_t min_bits, bo
     const uint32_t n = e >> 29, bits = (e >> 24) & 31u;
     bad |= n > 3u || bits > (uint32_t)kIdxBits || bits < n * min_bits || (n == 0 && bits != 0);
     const uint32_t syms = n >= 3u ? e & 0xFFFFFFu : e & ((1u << (8u * n)) - 1u);
-    return WORDS ? (n & 3u) | ((bits & 31u) << 2) | (syms << 8) : syms | (bits << 24) | (n << 29);
+    if (!WORDS)
+        return syms | (bits << 24) | (n << 29);
+    return n == 0 ? 0x80000000u : (n & 3u) | ((bits & 31u) << 2) | (syms << 7);
 }
 
 // Once per CTA, called by all its nthreads threads (tid = thread index): the
@@ -617,9 +620,13 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
             bool any_long = false;
 #pragma unroll
             for (int k = 0; k < 2; k++) {
-                if (ch[k].rem > 0) {
-                    // stopped on a code longer than 12 bits: the page's LUTs
-                    // (a code the table leaves to them has >= 13 bits)
+                if (ch[k].rem < -(1 << 30)) {
+                    // stopped on a code longer than 12 bits: undo the entry's
+                    // 2^31 and the 2^24 x mul its flag bit added to the
+                    // pending word, then the page's LUTs (a code the table
+                    // leaves to them has >= 13 bits)
+                    ch[k].rem = (int)((uint32_t)ch[k].rem ^ 0x80000000u);
+                    ch[k].w -= 0x01000000u * ch[k].mul;
                     const uint32_t d = lut_decode(ch[k].h, luts, cl, p.num_luts, &bad);
                     uint32_t len = d >> 8;
                     bad |= len <= (uint32_t)kIdxBits;
