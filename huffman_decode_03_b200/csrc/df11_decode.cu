@@ -392,15 +392,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             v = atomicAdd(&next_block, 1u);
         return __shfl_sync(0xffffffffu, v, 0);
     };
-    // with long slots the first block's registers load while the tables are built
+    // the first block's metadata arrives while the tables are set up: with
+    // long slots into registers; with short slots copied into the warp's
+    // buffer, unless the table is derived (its scratch overlaps the buffers)
     BlockRegs<C> cur, nxt;
     if (!kCopy && b < b_end)
         load_block<C>(p, b, lane, cur);
+    const bool early = kCopy && p.sym_table != nullptr;  // uniform
+    if (early && b < b_end)
+        prefetch_block<C>(p, b, lane, nbuf);
 
     if (!build_tables<kWords>(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
                       SLOT < kSlotLong ? 2u : 1u)) {
         if (tid == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+        asm volatile("cp.async.wait_all;" ::: "memory");  // no copy outlives the CTA
         return;
     }
     if (SLOT < kSlotLong) {
@@ -411,12 +417,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         if (bad || lmin < 2) {
             if (tid == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
+            asm volatile("cp.async.wait_all;" ::: "memory");
             return;
         }
     }
-    // with short slots the first block's metadata is copied only now: the
-    // table set-up used the start of the per-warp buffers as scratch
-    if (kCopy && b < b_end)
+    // a derived table used the start of the per-warp buffers as scratch:
+    // the first block's metadata is copied only now
+    if (kCopy && !early && b < b_end)
         prefetch_block<C>(p, b, lane, nbuf);
 
     const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
