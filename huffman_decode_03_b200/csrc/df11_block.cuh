@@ -409,41 +409,50 @@ __device__ __forceinline__ void place_words(uint32_t exp_base, const uint32_t s[
     // predicated per chain and word, no divergent branch inside
     const int nw1m[2] = {(int)nw[0] - 1, (int)nw[1] - 1};
     uint32_t sa = src[0], i = 0;
+    // Two passes per loop trip, the second with the roles of the previous
+    // and last words' registers exchanged, so no word is moved between
+    // passes; the trip count is tested after each pass.
+#define DF11_PW_PASS(PA, PB, DA, DB)                      \
+    "setp.lt.s32 r0, %5, %11;\n\t"                      \
+    "setp.lt.s32 r1, %5, %12;\n\t"                      \
+    "@p0 ld.shared.u32 c0, [%4];\n\t"                   \
+    "@p1 ld.shared.u32 c1, [%4+%10];\n\t"               \
+    "@r0 ld.shared.u32 " DA ", [%4+4];\n\t"             \
+    "@r1 ld.shared.u32 " DB ", [%4+%10+4];\n\t"         \
+    "@p0 shf.l.clamp.b32 w0, " PA ", c0, %8;\n\t"       \
+    "@p1 shf.l.clamp.b32 w1, " PB ", c1, %9;\n\t"       \
+    "@p0 st.shared.u32 [%2], w0;\n\t"                   \
+    "@p1 st.shared.u32 [%3], w1;\n\t"                   \
+    "@r0 shf.l.clamp.b32 w0, c0, " DA ", %8;\n\t"       \
+    "@r1 shf.l.clamp.b32 w1, c1, " DB ", %9;\n\t"       \
+    "@r0 st.shared.u32 [%2+4], w0;\n\t"                 \
+    "@r1 st.shared.u32 [%3+4], w1;\n\t"                 \
+    "add.u32 %4, %4, 8;\n\t"                            \
+    "add.u32 %2, %2, 8;\n\t"                            \
+    "add.u32 %3, %3, 8;\n\t"                            \
+    "add.u32 %5, %5, 2;\n\t"                            \
+    "setp.lt.u32 p0, %5, %6;\n\t"                       \
+    "setp.lt.u32 p1, %5, %7;\n\t"                       \
+    "or.pred pz, p0, p1;\n\t"
     asm volatile(
         "{\n\t"
         ".reg .pred p0, p1, r0, r1, pz;\n\t"
         ".reg .u32 c0, c1, d0, d1, w0, w1;\n\t"
-        "PW_TOP:\n\t"
         "setp.lt.u32 p0, %5, %6;\n\t"
         "setp.lt.u32 p1, %5, %7;\n\t"
         "or.pred pz, p0, p1;\n\t"
         "@!pz bra PW_END;\n\t"
-        "setp.lt.s32 r0, %5, %11;\n\t"
-        "setp.lt.s32 r1, %5, %12;\n\t"
-        "@p0 ld.shared.u32 c0, [%4];\n\t"
-        "@p1 ld.shared.u32 c1, [%4+%10];\n\t"
-        "@r0 ld.shared.u32 d0, [%4+4];\n\t"
-        "@r1 ld.shared.u32 d1, [%4+%10+4];\n\t"
-        "@p0 shf.l.clamp.b32 w0, %0, c0, %8;\n\t"
-        "@p1 shf.l.clamp.b32 w1, %1, c1, %9;\n\t"
-        "@p0 st.shared.u32 [%2], w0;\n\t"
-        "@p1 st.shared.u32 [%3], w1;\n\t"
-        "@r0 shf.l.clamp.b32 w0, c0, d0, %8;\n\t"
-        "@r1 shf.l.clamp.b32 w1, c1, d1, %9;\n\t"
-        "@r0 st.shared.u32 [%2+4], w0;\n\t"
-        "@r1 st.shared.u32 [%3+4], w1;\n\t"
-        "mov.b32 %0, d0;\n\t"
-        "mov.b32 %1, d1;\n\t"
-        "add.u32 %4, %4, 8;\n\t"
-        "add.u32 %2, %2, 8;\n\t"
-        "add.u32 %3, %3, 8;\n\t"
-        "add.u32 %5, %5, 2;\n\t"
-        "bra PW_TOP;\n\t"
+        "PW_TOP:\n\t"
+        DF11_PW_PASS("%0", "%1", "d0", "d1")
+        "@!pz bra PW_END;\n\t"
+        DF11_PW_PASS("d0", "d1", "%0", "%1")
+        "@pz bra PW_TOP;\n\t"
         "PW_END:\n\t"
         "}"
         : "+r"(prev[0]), "+r"(prev[1]), "+r"(dst[0]), "+r"(dst[1]), "+r"(sa), "+r"(i)
         : "r"(nw[0]), "r"(nw[1]), "r"(sh[0]), "r"(sh[1]), "n"(32 * SLOT), "r"(nw1m[0]), "r"(nw1m[1])
         : "memory");
+#undef DF11_PW_PASS
 }
 
 // A symbol-table entry (df11_symtab::table_entry: exponents in bytes 0..2,
