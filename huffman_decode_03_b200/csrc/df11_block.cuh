@@ -140,14 +140,14 @@ struct SharedBytes {
 // (its bits left before pend) is > 0; the bits of its window past pend are
 // zeros.  Per lookup the window advances and rem drops by the length
 // ((entry >> 2) serves as the funnel-shift amount directly: wrap mode reads
-// only its low five bits; masked with bit 31 kept, the long-code entry takes
-// 2^31 from rem, which ends the chain) and the exponents are added to the
-// chain's pending word w at byte n, where mul = 2^(8 n); mul rotates left by
-// 8 x count bits.  When the pending word fills (the rotation wraps, mul
-// decreases) it is stored at the slot address qa, qa advances one word and w
-// keeps the bytes that spilled past it.  The long-code entry moves nothing
-// but adds 2^24 x mul to w; the caller undoes both, resolves that code and
-// calls again.
+// only its low five bits; masked with its sign bits kept, the long-code
+// entry takes 2^31 or 2^30 from rem, which ends the chain) and the exponents
+// are added to the chain's pending word w at byte n, where mul = 2^(8 n); mul
+// rotates left by 8 x count bits.  When the pending word fills (the rotation
+// wraps, mul decreases) it is stored at the slot address qa, qa advances one
+// word and w keeps the bytes that spilled past it.  The long-code entry moves
+// nothing but adds 2^24 x mul to w; chain_roles undoes both, and the caller
+// resolves that code and calls again.
 struct Chain {
     uint32_t h, m, l;  // 96-bit window, next bit at the top of h
     int rem;           // pend - bits consumed
@@ -156,6 +156,63 @@ struct Chain {
     uint32_t mul;      // 2^(8 n)
 };
 
+// One pass of the loop for both chains.  The pending word and mul trade
+// registers every pass: a pass reads mul from MA (MB) and w from WA (WB) and
+// leaves the new mul in WA (WB) and the new w in MA (MB), so no value is
+// moved; the next pass is written with the roles exchanged.
+#define DF11_DB_CHAIN(P, E, H, M, L, REM, QA, MUL, W, MASK)        \
+    "@" P " shr.s32 ca, " E ", 2;\n\t"                            \
+    "@" P " and.b32 t, ca, " MASK ";\n\t"                         \
+    "@" P " sub.s32 " REM ", " REM ", t;\n\t"                      \
+    "@" P " shf.l.wrap.b32 " H ", " M ", " H ", ca;\n\t"          \
+    "@" P " shf.l.wrap.b32 " M ", " L ", " M ", ca;\n\t"          \
+    "@" P " shf.l.wrap.b32 " L ", 0, " L ", ca;\n\t"              \
+    "@" P " shr.u32 t, " E ", 7;\n\t"                             \
+    "@" P " mul.hi.u32 ca, t, " MUL ";\n\t"                       \
+    "@" P " mad.lo.u32 t, t, " MUL ", " W ";\n\t"                 \
+    "@" P " shl.b32 " W ", " E ", 3;\n\t"                         \
+    "@" P " shf.l.wrap.b32 " W ", " MUL ", " MUL ", " W ";\n\t"   \
+    "setp.lt.and.u32 po, " W ", " MUL ", " P ";\n\t"              \
+    "@po st.shared.u32 [" QA "], t;\n\t"                          \
+    "@po add.u32 " QA ", " QA ", 4;\n\t"                          \
+    "@" P " selp.b32 " MUL ", ca, t, po;\n\t"
+#define DF11_DB_PASS(MA, WA, MB, WB, MASK)                                         \
+    "@pa shr.u32 ea, %0, 20;\n\t"                                                 \
+    "@pb shr.u32 eb, %7, 20;\n\t"                                                 \
+    "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"                                          \
+    "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"                                          \
+    "@pa ld.shared.u32 ea, [ea];\n\t"                                             \
+    "@pb ld.shared.u32 eb, [eb];\n\t"                                             \
+    DF11_DB_CHAIN("pa", "ea", "%0", "%1", "%2", "%3", "%4", MA, WA, MASK)          \
+    DF11_DB_CHAIN("pb", "eb", "%7", "%8", "%9", "%10", "%11", MB, WB, MASK)        \
+    /* a chain stays active while bits are left (a long-code entry took */        \
+    /* 2^31 or 2^30 from them) */                                                  \
+    "setp.gt.s32 pa, %3, 0;\n\t"                                                  \
+    "setp.gt.s32 pb, %10, 0;\n\t"                                                 \
+    "or.pred pz, pa, pb;\n\t"
+
+// A chain's mul and w after decode_bulk2 (w and mul name its two registers):
+// a chain that ran out of bits has them in either order, the larger being
+// mul (w holds only the n bytes below mul = 2^(8 n)).  A chain stopped on a
+// code longer than 12 bits took 2^31 from rem in a first pass of the loop,
+// 2^30 in a second, which also tells the order, and its pending word holds
+// 2^24 x mul more: both are undone, leaving rem > 0 for the caller.
+__device__ __forceinline__ void chain_roles(Chain &c)
+{
+    const uint32_t r0 = c.w, r1 = c.mul;
+    if (c.rem < -(1 << 29)) {
+        const bool first = c.rem < -(3 << 29);  // 2^31 taken: a first pass
+        c.mul = first ? r0 : r1;
+        c.w = (first ? r1 : r0) - 0x01000000u * c.mul;
+        c.rem = (int)((uint32_t)c.rem + (first ? 0x80000000u : 0x40000000u));
+    } else {
+        c.mul = r0 > r1 ? r0 : r1;
+        c.w = r0 > r1 ? r1 : r0;
+    }
+}
+
+// The loop, two passes per trip (mul and w exchanged between them); each
+// chain's values are sorted out afterwards by chain_roles.
 __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_base)
 {
     asm volatile(
@@ -167,51 +224,9 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "or.pred pz, pa, pb;\n\t"
         "@!pz bra DB_END;\n\t"
         "DB_TOP:\n\t"
-        "@pa shr.u32 ea, %0, 20;\n\t"
-        "@pb shr.u32 eb, %7, 20;\n\t"
-        "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"
-        "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"
-        "@pa ld.shared.u32 ea, [ea];\n\t"
-        "@pb ld.shared.u32 eb, [eb];\n\t"
-        // chain A
-        "@pa shr.s32 ca, ea, 2;\n\t"
-        "@pa and.b32 t, ca, 0x8000001F;\n\t"
-        "@pa sub.s32 %3, %3, t;\n\t"
-        "@pa shf.l.wrap.b32 %0, %1, %0, ca;\n\t"
-        "@pa shf.l.wrap.b32 %1, %2, %1, ca;\n\t"
-        "@pa shf.l.wrap.b32 %2, 0, %2, ca;\n\t"
-        "@pa shr.u32 t, ea, 7;\n\t"
-        "@pa mul.hi.u32 ca, t, %6;\n\t"
-        "@pa mad.lo.u32 t, t, %6, %5;\n\t"
-        "@pa shl.b32 %5, ea, 3;\n\t"
-        "@pa shf.l.wrap.b32 %5, %6, %6, %5;\n\t"
-        "setp.lt.and.u32 po, %5, %6, pa;\n\t"
-        "@pa mov.b32 %6, %5;\n\t"
-        "@po st.shared.u32 [%4], t;\n\t"
-        "@po add.u32 %4, %4, 4;\n\t"
-        "@pa selp.b32 %5, ca, t, po;\n\t"
-        // chain B
-        "@pb shr.s32 ca, eb, 2;\n\t"
-        "@pb and.b32 t, ca, 0x8000001F;\n\t"
-        "@pb sub.s32 %10, %10, t;\n\t"
-        "@pb shf.l.wrap.b32 %7, %8, %7, ca;\n\t"
-        "@pb shf.l.wrap.b32 %8, %9, %8, ca;\n\t"
-        "@pb shf.l.wrap.b32 %9, 0, %9, ca;\n\t"
-        "@pb shr.u32 t, eb, 7;\n\t"
-        "@pb mul.hi.u32 ca, t, %13;\n\t"
-        "@pb mad.lo.u32 t, t, %13, %12;\n\t"
-        "@pb shl.b32 %12, eb, 3;\n\t"
-        "@pb shf.l.wrap.b32 %12, %13, %13, %12;\n\t"
-        "setp.lt.and.u32 po, %12, %13, pb;\n\t"
-        "@pb mov.b32 %13, %12;\n\t"
-        "@po st.shared.u32 [%11], t;\n\t"
-        "@po add.u32 %11, %11, 4;\n\t"
-        "@pb selp.b32 %12, ca, t, po;\n\t"
-        // a chain stays active while bits are left (a long-code entry took
-        // 2^31 from them)
-        "setp.gt.s32 pa, %3, 0;\n\t"
-        "setp.gt.s32 pb, %10, 0;\n\t"
-        "or.pred pz, pa, pb;\n\t"
+        DF11_DB_PASS("%6", "%5", "%13", "%12", "0x8000001F")
+        "@!pz bra DB_END;\n\t"
+        DF11_DB_PASS("%5", "%6", "%12", "%13", "0x4000001F")
         "@pz bra DB_TOP;\n\t"
         "DB_END:\n\t"
         "}"
@@ -219,7 +234,11 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
           "+r"(B.l), "+r"(B.rem), "+r"(B.qa), "+r"(B.w), "+r"(B.mul)
         : "r"(sym_base)
         : "memory");
+    chain_roles(A);
+    chain_roles(B);
 }
+#undef DF11_DB_PASS
+#undef DF11_DB_CHAIN
 
 // The byte-store form of the decode loop (the fused matrix-vector and GEMM
 // kernels, whose other work keeps the ALU busier than the L1): symbol-table
@@ -629,13 +648,9 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
             bool any_long = false;
 #pragma unroll
             for (int k = 0; k < 2; k++) {
-                if (ch[k].rem < -(1 << 30)) {
-                    // stopped on a code longer than 12 bits: undo the entry's
-                    // 2^31 and the 2^24 x mul its flag bit added to the
-                    // pending word, then the page's LUTs (a code the table
-                    // leaves to them has >= 13 bits)
-                    ch[k].rem = (int)((uint32_t)ch[k].rem ^ 0x80000000u);
-                    ch[k].w -= 0x01000000u * ch[k].mul;
+                if (ch[k].rem > 0) {
+                    // stopped on a code longer than 12 bits: the page's LUTs
+                    // (a code the table leaves to them has >= 13 bits)
                     const uint32_t d = lut_decode(ch[k].h, luts, cl, p.num_luts, &bad);
                     uint32_t len = d >> 8;
                     bad |= len <= (uint32_t)kIdxBits;
