@@ -46,10 +46,14 @@ __host__ __device__ constexpr uint32_t slot_bytes(uint32_t stride) { return 2 * 
 __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
 
 // Shared memory: tables at fixed offsets, then per warp: the exponent write
-// buffer and the chains' staging slots.
-struct Smem {
-    static constexpr uint32_t sym = 0;                       // uint32[4096]
-    static constexpr uint32_t luts = sym + kIdxEntries * 4;  // 17 * 256
+// buffer and the chains' staging slots.  R copies of the symbol table,
+// interleaved word by word (entry i of copy c at word R i + c): lane l reads
+// copy l mod R, so a lookup's 32 lanes spread over R groups of banks and
+// fewer of them meet in one bank.
+template <uint32_t R>
+struct SmemR {
+    static constexpr uint32_t sym = 0;                           // uint32[4096 R]
+    static constexpr uint32_t luts = sym + kIdxEntries * 4 * R;  // 17 * 256
     static constexpr uint32_t cl = luts + kLutBytes;         // 256
     static constexpr uint32_t zq = cl + 256;                 // uint8[16]
     static constexpr uint32_t ctr = zq + 16;                 // uint32 block counter (decoder), 16 B
@@ -63,7 +67,9 @@ struct Smem {
         return bufs + warps * per_warp(cap, stride);
     }
 };
-static_assert(Smem::bufs % 16 == 0, "buffers must be 16-byte aligned");
+using Smem = SmemR<1>;
+static_assert(SmemR<1>::bufs % 16 == 0 && SmemR<2>::bufs % 16 == 0 && SmemR<4>::bufs % 16 == 0,
+              "buffers must be 16-byte aligned");
 static_assert(slot_bytes(kSlotShort) % 16 == 0 && slot_bytes(kSlotLong) % 16 == 0,
               "slots keep the buffers 16-byte aligned");
 
@@ -179,8 +185,8 @@ struct Chain {
 #define DF11_DB_PASS(MA, WA, MB, WB, MASK)                                         \
     "@pa shr.u32 ea, %0, 20;\n\t"                                                 \
     "@pb shr.u32 eb, %7, 20;\n\t"                                                 \
-    "@pa mad.lo.u32 ea, ea, 4, %14;\n\t"                                          \
-    "@pb mad.lo.u32 eb, eb, 4, %14;\n\t"                                          \
+    "@pa mad.lo.u32 ea, ea, %15, %14;\n\t"                                        \
+    "@pb mad.lo.u32 eb, eb, %15, %14;\n\t"                                        \
     "@pa ld.shared.u32 ea, [ea];\n\t"                                             \
     "@pb ld.shared.u32 eb, [eb];\n\t"                                             \
     DF11_DB_CHAIN("pa", "ea", "%0", "%1", "%2", "%3", "%4", MA, WA, MASK)          \
@@ -213,6 +219,7 @@ __device__ __forceinline__ void chain_roles(Chain &c)
 
 // The loop, two passes per trip (mul and w exchanged between them); each
 // chain's values are sorted out afterwards by chain_roles.
+template <uint32_t R>
 __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_base)
 {
     asm volatile(
@@ -232,7 +239,7 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
         "}"
         : "+r"(A.h), "+r"(A.m), "+r"(A.l), "+r"(A.rem), "+r"(A.qa), "+r"(A.w), "+r"(A.mul), "+r"(B.h), "+r"(B.m),
           "+r"(B.l), "+r"(B.rem), "+r"(B.qa), "+r"(B.w), "+r"(B.mul)
-        : "r"(sym_base)
+        : "r"(sym_base), "n"(4 * R)
         : "memory");
     chain_roles(A);
     chain_roles(B);
@@ -501,15 +508,16 @@ __device__ __forceinline__ uint32_t table_word(uint32_t e, uint32_t min_bits, bo
 // Returns false (every thread alike) when the symbol table, stored or
 // derived, has an entry no such code set produces (table_word): the decode
 // loop's slot bound relies on every code taking at least min_bits bits.
-template <bool WORDS>
+template <bool WORDS, uint32_t R = 1>
 __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_t *cl_g, uint32_t num_luts,
                                              const uint32_t *sym_g, uint8_t *smem, uint32_t tid, uint32_t nthreads,
                                              uint32_t min_bits)
 {
-    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + Smem::sym);
-    uint8_t *luts = smem + Smem::luts;
-    uint8_t *cl = smem + Smem::cl;
-    uint8_t *zq = smem + Smem::zq;
+    using S = SmemR<R>;
+    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem + S::sym);
+    uint8_t *luts = smem + S::luts;
+    uint8_t *cl = smem + S::cl;
+    uint8_t *zq = smem + S::zq;
     const uint32_t lut_bytes = num_luts * 256u;
     for (uint32_t i = tid; i < lut_bytes; i += nthreads)
         luts[i] = luts_g[i];
@@ -521,20 +529,33 @@ __device__ __forceinline__ bool build_tables(const uint8_t *luts_g, const uint8_
         // and checked
         for (uint32_t i = tid; i < kIdxEntries / 4; i += nthreads) {
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(sym_g) + i);
-            reinterpret_cast<uint4 *>(sym_tab)[i] =
-                make_uint4(table_word<WORDS>(v.x, min_bits, bad), table_word<WORDS>(v.y, min_bits, bad),
-                           table_word<WORDS>(v.z, min_bits, bad), table_word<WORDS>(v.w, min_bits, bad));
+            const uint32_t t[4] = {table_word<WORDS>(v.x, min_bits, bad), table_word<WORDS>(v.y, min_bits, bad),
+                                   table_word<WORDS>(v.z, min_bits, bad), table_word<WORDS>(v.w, min_bits, bad)};
+            if (R == 1) {
+                reinterpret_cast<uint4 *>(sym_tab)[i] = make_uint4(t[0], t[1], t[2], t[3]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; k++)
+#pragma unroll
+                    for (uint32_t c = 0; c < R; c++)
+                        sym_tab[R * (4 * i + k) + c] = t[k];
+            }
         }
     } else {
         __syncthreads();
         // the first code of each 12-bit window (df11_symtab::first_code), in
         // scratch in the per-warp buffers, which are free until the blocks start
-        uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + Smem::bufs);
+        uint16_t *first_code = reinterpret_cast<uint16_t *>(smem + S::bufs);
         for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
             first_code[i] = df11_symtab::first_code(i, luts, cl, num_luts);
         __syncthreads();
         for (uint32_t i = tid; i < kIdxEntries; i += nthreads)
-            sym_tab[i] = table_word<WORDS>(df11_symtab::table_entry(i, first_code), min_bits, bad);
+        {
+            const uint32_t t = table_word<WORDS>(df11_symtab::table_entry(i, first_code), min_bits, bad);
+#pragma unroll
+            for (uint32_t c = 0; c < R; c++)
+                sym_tab[R * i + c] = t;
+        }
     }
     if (__syncthreads_or(bad))
         return false;
@@ -569,14 +590,15 @@ struct BlockOut {
 // sign/mantissa bytes first.  Returns false, after setting DF11_ERR_CORRUPT
 // in *p.status, when the block is inconsistent (nothing placed).  Called by
 // all 32 lanes of the warp.
-template <int C, uint32_t SLOT, bool WORDS, class P>
+template <int C, uint32_t SLOT, bool WORDS, uint32_t R, class P>
 __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, const BlockRegs<C> &cur,
                                              uint32_t sym_base, uint32_t exp_base, uint32_t slot_base, BlockOut &out)
 {
     // the LUTs, CodeLengths and zero-code table lie at fixed offsets from the
-    // symbol table (Smem)
-    const SharedBytes luts{sym_base + (Smem::luts - Smem::sym)}, cl{sym_base + (Smem::cl - Smem::sym)};
-    const uint32_t zq = sym_base + (Smem::zq - Smem::sym);
+    // symbol table (SmemR)
+    using S = SmemR<R>;
+    const SharedBytes luts{sym_base + (S::luts - S::sym)}, cl{sym_base + (S::cl - S::sym)};
+    const uint32_t zq = sym_base + (S::zq - S::sym);
     constexpr uint32_t T = 32 * C;
     const uint32_t o0 = cur.o0, o1 = cur.o1;
     const uint32_t lo_off = o0 & 15u;
@@ -644,7 +666,7 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
             ch[k].mul = 1u;
         }
         for (;;) {  // each pass resolves >= 1 code or ends both chains
-            decode_bulk2(ch[0], ch[1], sym_base);
+            decode_bulk2<R>(ch[0], ch[1], sym_base + 4u * ((uint32_t)lane % R));
             bool any_long = false;
 #pragma unroll
             for (int k = 0; k < 2; k++) {

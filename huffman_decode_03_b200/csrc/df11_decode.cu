@@ -362,7 +362,7 @@ __host__ __device__ constexpr uint32_t warp_bytes(uint32_t cap)
 // copied into shared memory by cp.async, with long slots it is loaded into
 // registers.
 // MODE 0: store the BF16 outputs; MODE 1: fused matrix-vector product.
-template <int C, int WARPS, int MODE, uint32_t SLOT>
+template <int C, int WARPS, int MODE, uint32_t SLOT, uint32_t R>
 __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params p)
 {
     static_assert(C == 1 || C == 2, "one or two chains per lane");
@@ -372,16 +372,18 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     // rebuild to memory), the byte-store loop where the ALU is (the fused
     // matrix-vector product)
     constexpr bool kWords = MODE == 0;
+    constexpr uint32_t kR = R;  // symbol-table copies (SmemR)
+    using S = SmemR<kR>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint8_t *exp_s = smem + Smem::bufs + warp * warp_bytes<C, SLOT>(p.cap);
+    uint8_t *exp_s = smem + S::bufs + warp * warp_bytes<C, SLOT>(p.cap);
     uint8_t *slots = exp_s + p.cap;
     const uint32_t nbuf = static_cast<uint32_t>(__cvta_generic_to_shared(slots + slot_bytes(SLOT)));
 
     // the CTA's blocks are a contiguous range; each warp takes its first one
     // here and every next one from a counter in shared memory, so that the
     // CTA's warps all finish within about one block of each other
-    uint32_t &next_block = *reinterpret_cast<uint32_t *>(smem + Smem::ctr);
+    uint32_t &next_block = *reinterpret_cast<uint32_t *>(smem + S::ctr);
     const uint32_t b_end = (uint32_t)(((uint64_t)p.nblocks * (blockIdx.x + 1)) / gridDim.x);
     uint32_t b = (uint32_t)(((uint64_t)p.nblocks * blockIdx.x) / gridDim.x) + (uint32_t)warp;
     if (tid == 0)
@@ -402,7 +404,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (early && b < b_end)
         prefetch_block<C>(p, b, lane, nbuf);
 
-    if (!build_tables<kWords>(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
+    if (!build_tables<kWords, kR>(p.luts, p.cl, p.num_luts, p.sym_table, smem, (uint32_t)tid, (uint32_t)kThreads,
                       SLOT < kSlotLong ? 2u : 1u)) {
         if (tid == 0)
             atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
         // short slots hold a segment's codes only when no code is 1 bit long
         // (the all-zero code is the shortest: canonical codes)
         bool bad = false;
-        const uint32_t lmin = lut_decode(0u, smem + Smem::luts, smem + Smem::cl, p.num_luts, &bad) >> 8;
+        const uint32_t lmin = lut_decode(0u, smem + S::luts, smem + S::cl, p.num_luts, &bad) >> 8;
         if (bad || lmin < 2) {
             if (tid == 0)
                 atomicOr(p.status, (uint32_t)DF11_ERR_CORRUPT);
@@ -426,7 +428,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     if (kCopy && !early && b < b_end)
         prefetch_block<C>(p, b, lane, nbuf);
 
-    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + Smem::sym));
+    const uint32_t sym_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem + S::sym));
     const uint32_t exp_base = static_cast<uint32_t>(__cvta_generic_to_shared(exp_s));
     const uint32_t slot_base = static_cast<uint32_t>(__cvta_generic_to_shared(slots)) + lane * SLOT;
 
@@ -441,7 +443,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
             load_block<C>(p, nb, lane, nxt);
         }
         BlockOut bo;
-        if (decode_block<C, SLOT, kWords>(p, b, lane, cur, sym_base, exp_base, slot_base, bo)) {
+        if (decode_block<C, SLOT, kWords, kR>(p, b, lane, cur, sym_base, exp_base, slot_base, bo)) {
             // ---- merge with sign/mantissa (from L2)
             const uint64_t g0 = bo.g0;
             const uint32_t lo_off = bo.lo_off, hi = bo.hi;
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
 struct DeviceFacts {
     int sms = 0;
     int smem_optin = 0;
-    uint32_t granted[2][2][2][4] = {};  // [MODE][C - 1][short slots][warps 32 / 24 / 16 / 8]
+    uint32_t granted[2][2][2][5] = {};  // [MODE][C - 1][short slots][warps 32 / 24 / 16 / 8, 32 with 2 tables]
     cudaStream_t up = nullptr, down = nullptr;  // copy streams of the host path, made on first use
 };
 std::mutex g_mu;
@@ -543,10 +545,10 @@ df11_status device_facts(DeviceFacts **out)
     return DF11_OK;
 }
 
-template <int C, int WARPS, int MODE, uint32_t SLOT>
+template <int C, int WARPS, int MODE, uint32_t SLOT, uint32_t R = 1>
 df11_status launch_warps(const Params &prm, cudaStream_t stream, uint32_t smem, DeviceFacts *f, uint32_t &granted)
 {
-    auto kern = df11_decode_kernel<C, WARPS, MODE, SLOT>;
+    auto kern = df11_decode_kernel<C, WARPS, MODE, SLOT, R>;
     if (smem > granted) {
         std::lock_guard<std::mutex> lock(g_mu);
         if (smem > granted) {
@@ -576,14 +578,19 @@ df11_status launch_slots(const Params &prm, cudaStream_t stream, DeviceFacts *f)
     const uint32_t optin = (uint32_t)f->smem_optin;
     auto &g = f->granted[MODE][C - 1][SLOT == kSlotShort ? 1 : 0];
     const uint32_t wb = warp_bytes<C, SLOT>(prm.cap);
-    if (Smem::bufs + 32 * wb <= optin)
-        return launch_warps<C, 32, MODE, SLOT>(prm, stream, Smem::bufs + 32 * wb, f, g[0]);
-    if (Smem::bufs + 24 * wb <= optin)
-        return launch_warps<C, 24, MODE, SLOT>(prm, stream, Smem::bufs + 24 * wb, f, g[1]);
-    if (Smem::bufs + 16 * wb <= optin)
-        return launch_warps<C, 16, MODE, SLOT>(prm, stream, Smem::bufs + 16 * wb, f, g[2]);
-    if (Smem::bufs + 8 * wb <= optin)
-        return launch_warps<C, 8, MODE, SLOT>(prm, stream, Smem::bufs + 8 * wb, f, g[3]);
+    // the rebuild to memory takes two copies of the symbol table (fewer bank
+    // conflicts in its lookups) when 32 warps still fit beside them
+    if (MODE == 0 && SmemR<2>::bufs + 32 * wb <= optin)
+        return launch_warps<C, 32, MODE, SLOT, 2>(prm, stream, SmemR<2>::bufs + 32 * wb, f, g[4]);
+    const uint32_t base = Smem::bufs;
+    if (base + 32 * wb <= optin)
+        return launch_warps<C, 32, MODE, SLOT>(prm, stream, base + 32 * wb, f, g[0]);
+    if (base + 24 * wb <= optin)
+        return launch_warps<C, 24, MODE, SLOT>(prm, stream, base + 24 * wb, f, g[1]);
+    if (base + 16 * wb <= optin)
+        return launch_warps<C, 16, MODE, SLOT>(prm, stream, base + 16 * wb, f, g[2]);
+    if (base + 8 * wb <= optin)
+        return launch_warps<C, 8, MODE, SLOT>(prm, stream, base + 8 * wb, f, g[3]);
     return DF11_ERR_INVALID_ARG;
 }
 

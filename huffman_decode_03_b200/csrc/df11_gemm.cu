@@ -484,7 +484,7 @@ __device__ __forceinline__ void decode_role(const GemmParams &p, const Roles &R,
             const uint64_t o0 = cur.o0, o1 = cur.o1 > cur.o0 ? cur.o1 : cur.o0;
             const uint64_t r0 = o0 > e0 ? o0 : e0, r1 = o1 < e1 ? o1 : e1;
             BlockOut bo;
-            const bool dok = decode_block<C, SLOT, false>(p, b, lane, cur, sym_base, exp_base, slot_base, bo);
+            const bool dok = decode_block<C, SLOT, false, 1>(p, b, lane, cur, sym_base, exp_base, slot_base, bo);
             if (r0 < r1) {
                 const uint32_t t_first = (uint32_t)((r0 - e0) >> kTileShift);
                 const uint32_t t_last = (uint32_t)((r1 - 1 - e0) >> kTileShift);
