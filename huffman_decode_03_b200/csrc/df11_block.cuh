@@ -247,8 +247,8 @@ __device__ __forceinline__ void decode_bulk2(Chain &A, Chain &B, uint32_t sym_ba
 #undef DF11_DB_PASS
 #undef DF11_DB_CHAIN
 
-// The byte-store form of the decode loop (the fused matrix-vector and GEMM
-// kernels, whose other work keeps the ALU busier than the L1): symbol-table
+// The byte-store form of the decode loop (the fused GEMM's decode warps, for
+// which the pending-word form measured no faster): symbol-table
 // entry as stored (table_entry): up to three rotated exponents in bytes
 // 0..2, their total length in bits 24..28, their number in bits 29..30
 // (0 = a code longer than 12 bits).

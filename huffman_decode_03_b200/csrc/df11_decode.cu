@@ -368,10 +368,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) df11_decode_kernel(const Params
     static_assert(C == 1 || C == 2, "one or two chains per lane");
     constexpr int kWarps = WARPS, kThreads = WARPS * 32;
     constexpr bool kCopy = SLOT == kSlotShort;  // metadata by cp.async
-    // the pending-word decode loop where the L1 is the busier unit (the
-    // rebuild to memory), the byte-store loop where the ALU is (the fused
-    // matrix-vector product)
-    constexpr bool kWords = MODE == 0;
+    // the pending-word decode loop in both modes (the fused GEMM's decode
+    // warps keep the byte-store loop)
+    constexpr bool kWords = true;
     constexpr uint32_t kR = R;  // symbol-table copies (SmemR)
     using S = SmemR<kR>;
     extern __shared__ __align__(128) uint8_t smem[];
