@@ -742,13 +742,20 @@ __device__ __forceinline__ bool decode_block(const P &p, uint32_t b, int lane, c
 #pragma unroll
     for (int k = 0; k < C; k++)
         packed |= (cnt[k] & 0xFFFFu) << (16 * k);
+    // (the shuffle's own predicate says whether the source lane exists)
     uint32_t incl = packed;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d)
-            incl += y;
-    }
+    asm("{\n\t.reg .pred q;\n\t.reg .u32 y;\n\t"
+        "shfl.sync.up.b32 y|q, %0, 1, 0, -1;\n\t"
+        "@q add.u32 %0, %0, y;\n\t"
+        "shfl.sync.up.b32 y|q, %0, 2, 0, -1;\n\t"
+        "@q add.u32 %0, %0, y;\n\t"
+        "shfl.sync.up.b32 y|q, %0, 4, 0, -1;\n\t"
+        "@q add.u32 %0, %0, y;\n\t"
+        "shfl.sync.up.b32 y|q, %0, 8, 0, -1;\n\t"
+        "@q add.u32 %0, %0, y;\n\t"
+        "shfl.sync.up.b32 y|q, %0, 16, 0, -1;\n\t"
+        "@q add.u32 %0, %0, y;\n\t}"
+        : "+r"(incl));
     const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
     uint32_t first[2] = {0u, 0u};
     uint32_t total = 0;
